@@ -1,0 +1,350 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself.
+
+What pins what:
+  * e4m3 / bf16 decoding: every code against torch's own dtype conversion.
+  * indexer: with one head, w = 1 it must equal ReLU(scale * q.k^T) computed
+    by a library matmul (the reduction stated in the path's definition);
+    one-hot and negated head weights, positive homogeneity in the scales and
+    head permutation then fix how heads, weights and scales enter; the
+    causal boundary is checked at an offset.
+  * top-k: equals a brute-force full sort (numpy lexsort) on tiny rows with
+    many ties; the short-context fallback selects every key.
+  * sparse MLA: when every causal key is selected it must equal dense causal
+    softmax attention from torch's scaled_dot_product_attention in float64;
+    a single selected row returns that row's latent exactly; the selection
+    order does not matter and unselected rows (even NaN) have no effect.
+  * paged decode: equals the contiguous path on the same logical sequence,
+    and a permutation of the physical blocks changes nothing.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+
+
+def e4m3_codes(rng, shape, lo=-8, hi=8):
+    v = torch.from_numpy(rng.integers(lo, hi + 1, size=shape)).float()
+    return v.to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def e4m3_random(rng, shape):
+    """Arbitrary finite e4m3 codes (not only integers)."""
+    codes = rng.integers(0, 256, size=shape).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x3C      # replace NaN codes by 1.5
+    return torch.from_numpy(codes)
+
+
+def lib_float(codes_u8):
+    return codes_u8.view(torch.float8_e4m3fn).double()
+
+
+# ----------------------------------------------------------------- decoding
+
+def test_e4m3_every_code_matches_torch():
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double()
+    for c in range(256):
+        got = oracle.e4m3(c)
+        if np.isnan(ref[c].item()):
+            assert np.isnan(got), c
+        else:
+            assert got == ref[c].item(), (c, got, ref[c].item())
+
+
+def test_bf16_decode_matches_torch():
+    rng = np.random.default_rng(7)
+    bits = rng.integers(0, 1 << 16, size=4096).astype(np.uint16)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).double().numpy()
+    got = np.array([oracle.bf16(int(b)) for b in bits])
+    same = (got == ref) | (np.isnan(got) & np.isnan(ref))
+    assert same.all()
+
+
+# ------------------------------------------------------------------ indexer
+
+def _single_head_library(q_f, k_f, scale, q_pos0):
+    """ReLU(scale * q.k^T) with the causal mask, via a library matmul."""
+    x = scale * (q_f @ k_f.T)
+    T, S = x.shape
+    pos = q_pos0 + torch.arange(T).unsqueeze(1)
+    x = torch.clamp(x, min=0.0)
+    return torch.where(torch.arange(S).unsqueeze(0) <= pos, x, torch.tensor(-np.inf, dtype=x.dtype))
+
+
+@pytest.mark.parametrize("grid", [True, False])
+def test_indexer_one_head_unit_weight_is_relu_qk(grid):
+    rng = np.random.default_rng(1)
+    T, S = 37, 53
+    mk = e4m3_codes if grid else e4m3_random
+    q8 = mk(rng, (T, 1, 128))
+    k8 = mk(rng, (S, 128))
+    w = torch.ones(T, 1)
+    scale, q_pos0 = 0.3125, 11
+    got = oracle.indexer(q8, None, k8, None, w, scale, q_pos0)
+    ref = _single_head_library(lib_float(q8[:, 0]), lib_float(k8), scale, q_pos0)
+    ref32 = ref.float().numpy()
+    fin = np.isfinite(ref32)
+    assert (np.isfinite(got) == fin).all()
+    if grid:
+        assert (got[fin] == ref32[fin]).all()
+    else:
+        np.testing.assert_allclose(got[fin], ref32[fin], rtol=2e-7, atol=0)
+
+
+def test_indexer_head_weights_and_sign():
+    """One-hot (+1 and -1) weights pick one head's ReLU score, with its sign."""
+    rng = np.random.default_rng(2)
+    T, S, Hi = 19, 40, 4
+    q8 = e4m3_codes(rng, (T, Hi, 128))
+    k8 = e4m3_codes(rng, (S, 128))
+    scale = 1.0 / 16
+    for h in range(Hi):
+        for sign in (1.0, -1.0):
+            w = torch.zeros(T, Hi)
+            w[:, h] = sign
+            got = oracle.indexer(q8, None, k8, None, w, scale)
+            ref = sign * _single_head_library(lib_float(q8[:, h]), lib_float(k8), scale, 0)
+            ref = torch.where(torch.isfinite(ref), ref, torch.tensor(-np.inf, dtype=ref.dtype))
+            ref32 = ref.float().numpy()
+            fin = np.isfinite(ref32)
+            assert (np.isfinite(got) == fin).all()
+            assert (got[fin] == ref32[fin]).all(), (h, sign)
+
+
+def test_indexer_linear_in_weights_and_head_permutation():
+    rng = np.random.default_rng(3)
+    T, S, Hi = 23, 31, 4
+    q8 = e4m3_codes(rng, (T, Hi, 128))
+    k8 = e4m3_codes(rng, (S, 128))
+    w1 = torch.from_numpy(rng.integers(-4, 5, size=(T, Hi)) / 4.0).float()
+    w2 = torch.from_numpy(rng.integers(-4, 5, size=(T, Hi)) / 4.0).float()
+    I1 = oracle.indexer(q8, None, k8, None, w1, 1 / 16)
+    I2 = oracle.indexer(q8, None, k8, None, w2, 1 / 16)
+    I12 = oracle.indexer(q8, None, k8, None, w1 + w2, 1 / 16)
+    fin = np.isfinite(I12)
+    assert (I1[fin] + I2[fin] == I12[fin]).all()       # exact on the grid
+    perm = torch.from_numpy(rng.permutation(Hi))
+    Ip = oracle.indexer(q8[:, perm].contiguous(), None, k8, None, w1[:, perm].contiguous(), 1 / 16)
+    assert np.array_equal(Ip, I1)
+
+
+def test_indexer_positive_homogeneity_in_scales():
+    """I scales by q_scale[t] * k_scale[s] * scale (all > 0): ReLU commutes with them."""
+    rng = np.random.default_rng(4)
+    T, S, Hi = 17, 29, 3
+    q8 = e4m3_random(rng, (T, Hi, 128))
+    k8 = e4m3_random(rng, (S, 128))
+    w = torch.from_numpy(rng.normal(size=(T, Hi))).float()
+    qs = torch.from_numpy(rng.uniform(0.01, 3.0, size=T)).float()
+    ks = torch.from_numpy(rng.uniform(0.01, 3.0, size=S)).float()
+    base = oracle.indexer(q8, None, k8, None, w, 1.0)
+    got = oracle.indexer(q8, qs, k8, ks, w, 0.125)
+    ref = base.astype(np.float64) * qs.double().numpy()[:, None] * ks.double().numpy()[None, :] * 0.125
+    fin = np.isfinite(base)
+    assert (np.isfinite(got) == fin).all()
+    np.testing.assert_allclose(got[fin], ref[fin], rtol=1e-6, atol=1e-30)
+
+
+def test_indexer_causal_boundary_and_row_subset():
+    rng = np.random.default_rng(5)
+    T, S, Hi = 8, 20, 2
+    q8 = e4m3_codes(rng, (T, Hi, 128))
+    k8 = e4m3_codes(rng, (S, 128))
+    w = torch.ones(T, Hi)
+    q_pos0 = 9
+    I = oracle.indexer(q8, None, k8, None, w, 1 / 16, q_pos0)
+    for t in range(T):
+        p = q_pos0 + t
+        assert np.isfinite(I[t, : min(p + 1, S)]).all()
+        assert np.isneginf(I[t, p + 1:]).all()
+    rows = np.array([6, 1, 3])
+    Ir = oracle.indexer(q8, None, k8, None, w, 1 / 16, q_pos0, rows=rows)
+    assert np.array_equal(Ir, I[rows])
+
+
+# -------------------------------------------------------------------- top-k
+
+def brute_topk(row, n, k):
+    if n <= k:
+        return np.concatenate([np.arange(n), -np.ones(k - n, np.int64)])
+    s = np.arange(n)
+    order = np.lexsort((s, -row[:n].astype(np.float64)))
+    return order[:k]
+
+
+def test_topk_equals_full_sort_with_ties():
+    rng = np.random.default_rng(6)
+    R, ld, k = 40, 300, 17
+    I = rng.integers(-6, 7, size=(R, ld)).astype(np.float32)   # many ties
+    I[:5] = rng.normal(size=(5, ld)).astype(np.float32)
+    n = rng.integers(1, ld + 1, size=R)
+    n[:3] = [1, k, k + 1]
+    got = oracle.topk(I, n, k)
+    for r in range(R):
+        assert np.array_equal(got[r], brute_topk(I[r], n[r], k)), r
+
+
+def test_topk_short_context_takes_every_key_and_scale_invariance():
+    rng = np.random.default_rng(8)
+    I = rng.normal(size=(6, 64)).astype(np.float32)
+    n = np.array([1, 5, 32, 33, 64, 2])
+    got = oracle.topk(I, n, 32)
+    for r in range(6):
+        if n[r] <= 32:
+            assert list(got[r, : n[r]]) == list(range(n[r]))
+            assert (got[r, n[r]:] == -1).all()
+    scaled = oracle.topk(I * np.float32(4.0), n, 32)     # power of two: exact
+    assert np.array_equal(scaled, got)
+
+
+# --------------------------------------------------------------- sparse MLA
+
+def _bf16(rng, shape):
+    return torch.from_numpy(rng.normal(size=shape)).to(torch.bfloat16)
+
+
+def dense_causal_sdpa(q, kv, sm_scale):
+    """Library dense causal attention in float64: K = kv (576), V = kv[:, :512]."""
+    T, H, _ = q.shape
+    qd = q.double().permute(1, 0, 2)                         # [H][T][576]
+    kd = kv.double().unsqueeze(0).expand(H, -1, -1)
+    vd = kv[:, :512].double().unsqueeze(0).expand(H, -1, -1)
+    o = torch.nn.functional.scaled_dot_product_attention(qd, kd, vd, is_causal=True, scale=sm_scale)
+    logits = (qd @ kd.transpose(1, 2)) * sm_scale
+    mask = torch.ones(T, T, dtype=torch.bool).tril()
+    lse = torch.logsumexp(logits.masked_fill(~mask, -np.inf), dim=-1)
+    return o.permute(1, 0, 2).numpy(), lse.T.numpy()
+
+
+def test_mla_all_keys_selected_is_dense_causal_attention():
+    rng = np.random.default_rng(9)
+    T, H, k = 24, 3, 32
+    q, kv = _bf16(rng, (T, H, 576)), _bf16(rng, (T, 576))
+    idx = np.full((T, k), -1, np.int32)
+    for t in range(T):
+        idx[t, : t + 1] = rng.permutation(t + 1)
+    out, lse = oracle.sparse_mla(q, kv, idx, 1 / 24)
+    ref, ref_lse = dense_causal_sdpa(q, kv, 1 / 24)
+    np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=1e-12, atol=1e-12)
+
+
+def test_mla_single_selected_row_is_that_row():
+    rng = np.random.default_rng(10)
+    T, H, k = 5, 4, 8
+    q, kv = _bf16(rng, (T, H, 576)), _bf16(rng, (11, 576))
+    idx = np.full((T, k), -1, np.int32)
+    for t in range(T):
+        idx[t, rng.integers(0, k)] = t + 3
+    out, lse = oracle.sparse_mla(q, kv, idx, 0.1)
+    for t in range(T):
+        row = kv[t + 3, :512].double().numpy()
+        assert (out[t] == row[None, :]).all()
+        z = 0.1 * (q[t].double() @ kv[t + 3].double()).numpy()
+        np.testing.assert_allclose(lse[t], z, rtol=1e-13)
+
+
+def test_mla_order_free_and_unselected_rows_have_no_effect():
+    rng = np.random.default_rng(11)
+    T, S, H, k = 6, 50, 2, 12
+    q, kv = _bf16(rng, (T, H, 576)), _bf16(rng, (S, 576))
+    idx = np.stack([rng.choice(S, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    idx[2, 5:] = -1
+    out, lse = oracle.sparse_mla(q, kv, idx, 1 / 24)
+    perm = np.stack([rng.permutation(k) for _ in range(T)])
+    out_p, lse_p = oracle.sparse_mla(q, kv, np.take_along_axis(idx, perm, 1), 1 / 24)
+    np.testing.assert_allclose(out_p, out, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(lse_p, lse, rtol=1e-13)
+    poisoned = kv.clone()
+    sel = set(idx[idx >= 0].tolist())
+    for s in range(S):
+        if s not in sel:
+            poisoned[s] = float("nan")
+    out_n, lse_n = oracle.sparse_mla(q, poisoned, idx, 1 / 24)
+    assert np.array_equal(out_n, out) and np.array_equal(lse_n, lse)
+
+
+# ---------------------------------------------------------------- full path
+
+def test_short_context_dsa_is_dense_causal_attention():
+    """Context <= k: the whole DSA path reproduces dense causal attention."""
+    cfg = W.CONFIGS[1]
+    inp = W.make_prefill(cfg, L=160)            # every row has <= 256 keys
+    r = oracle.forward(inp)
+    ref, ref_lse = dense_causal_sdpa(inp["q"], inp["kv"], inp["sm_scale"])
+    np.testing.assert_allclose(r["out"], ref, rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(r["lse"], ref_lse, rtol=1e-12, atol=1e-12)
+
+
+def test_long_context_selection_is_the_indexer_top_k():
+    """Past k keys, the output only depends on the selected rows."""
+    cfg = W.CONFIGS[1]
+    inp = W.make_prefill(cfg, L=400)
+    rows = np.array([399, 300, 257, 256, 255, 10])
+    r = oracle.forward(inp, rows=rows)
+    kv = inp["kv"].clone()
+    for i, t in enumerate(rows):
+        sel = set(r["idx"][i][r["idx"][i] >= 0].tolist())
+        assert len(sel) == min(t + 1, 256)
+    # shifting every unselected causal key of row 399 leaves its output alone
+    sel = set(r["idx"][0].tolist())
+    for s in range(400):
+        if s not in sel:
+            kv[s] = kv[s] + 3.0
+    out2, _ = oracle.sparse_mla(inp["q"], kv, np.tile(r["idx"][:1], (400, 1)), inp["sm_scale"], rows=[399])
+    assert np.array_equal(out2[0], r["out"][0])
+
+
+# ------------------------------------------------------------- paged decode
+
+def _small_decode(lens, seed=3, nq=2):
+    cfg = W.Config(99, "tiny_decode", "decode", k=48, Hi=4, H=3, seed=seed, nq=nq,
+                   ctx_lo=1, ctx_hi=2)
+    return W.make_decode(cfg, lens=torch.tensor(lens))
+
+
+def test_decode_equals_contiguous_prefill_rows():
+    inp = _small_decode([130, 40, 200], nq=2)
+    d = oracle.decode(inp)
+    for i, b in enumerate(range(inp["B"])):
+        n = int(inp["seq_len"][b])
+        k8 = oracle.gather_sequence(inp["k8_pool"].numpy(), inp["block_table"][b].numpy(), n)
+        ks = oracle.gather_sequence(inp["k_scale_pool"].numpy(), inp["block_table"][b].numpy(), n)
+        kv = oracle.gather_sequence(inp["kv_pool"].view(torch.int16).numpy(),
+                                    inp["block_table"][b].numpy(), n)
+        # contiguous prefill of n tokens whose last nq rows are the decode queries
+        T = n
+        q8 = torch.zeros(T, 4, 128, dtype=torch.uint8)
+        q8[n - 2:] = inp["q8"][b]
+        qs = torch.ones(T)
+        qs[n - 2:] = inp["q_scale"][b]
+        w = torch.zeros(T, 4)
+        w[n - 2:] = inp["w"][b]
+        q = torch.zeros(T, 3, 576, dtype=torch.bfloat16)
+        q[n - 2:] = inp["q"][b]
+        pre = dict(q8=q8, q_scale=qs, k8=torch.from_numpy(k8), k_scale=torch.from_numpy(ks),
+                   w=w, q=q, kv=torch.from_numpy(kv).view(torch.bfloat16), scale=inp["scale"],
+                   sm_scale=inp["sm_scale"], k=inp["k"], q_pos0=0, T=T, S=n)
+        r = oracle.forward(pre, rows=[n - 2, n - 1])
+        assert np.array_equal(np.sort(r["idx"], 1), np.sort(d["idx"][i], 1))
+        np.testing.assert_array_equal(r["out"], d["out"][i])
+
+
+def test_decode_invariant_under_physical_block_permutation():
+    inp = _small_decode([100, 64, 65], nq=1)
+    d = oracle.decode(inp)
+    rng = np.random.default_rng(12)
+    nblk = inp["nblk"]
+    perm = torch.from_numpy(rng.permutation(nblk))       # new physical slot of each block
+    inv = torch.empty_like(perm)
+    inv[perm] = torch.arange(nblk)
+    inp2 = dict(inp)
+    for key in ("k8_pool", "k_scale_pool", "kv_pool"):
+        inp2[key] = inp[key][inv].contiguous()
+    tab = inp["block_table"].clone()
+    tab[tab >= 0] = perm[tab[tab >= 0].long()].int()
+    inp2["block_table"] = tab
+    d2 = oracle.decode(inp2)
+    assert np.array_equal(d2["idx"], d["idx"])
+    assert np.array_equal(d2["out"], d["out"])
