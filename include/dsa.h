@@ -1,0 +1,205 @@
+/*
+ * dsa.h -- C ABI of libdsa.so: DeepSeek Sparse Attention (DSA) on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method has three stages, all on the GPU:
+ *   1. lightning indexer: for every causal (query t, key s) pair
+ *        I[t,s] = sum_h w[t,h] * ReLU(scale * q[t,h] . k[s])
+ *      over a 128-wide FP8 (e4m3) indexer key cache
+ *      ("DeepSeek-V3.2-Exp 模型优势与 DSA 工作原理", section 4, step 2;
+ *       FP8 and ReLU: "m.gxzdkb.com/media/457.html", section "秘密武器");
+ *   2. top-k: each query keeps its k best keys (k = 2048 by default), or
+ *      every key when it sees at most k of them (page 3, section 4, step 3
+ *      and section 2 "风险边界明确"); ties go to the smaller key index;
+ *   3. sparse MLA: softmax attention over the selected keys only, against a
+ *      512 + 64 wide bf16 latent cache whose first 512 dims are the values
+ *      (page 3, section 4, step 4 and section 3 "稀疏多潜在注意力").
+ *
+ * Conventions shared by every entry point
+ *  - All pointers are DEVICE pointers of the current CUDA device unless a
+ *    parameter says otherwise. The caller owns every buffer, including any
+ *    workspace; the library never allocates or frees device memory.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream) and the call returns without synchronising.
+ *  - Arguments are checked on the host before anything is launched; a call
+ *    that fails a check returns DSA_ERR_INVALID_ARG (or DSA_ERR_UNSUPPORTED)
+ *    and launches nothing. A failed launch returns DSA_ERR_CUDA.
+ *  - Faults found by the kernels (an index or block id out of range, which
+ *    is then skipped; a bounded wait that gave up, after which the kernel
+ *    returns early) are recorded in a per-device error word and reported by
+ *    dsa_get_device_error(). While a timeout is recorded, every kernel of
+ *    this library returns at once, so read and clear the word after a
+ *    failure.
+ *  - Buffers handed to the tensor memory accelerator must be 16-byte
+ *    aligned; row pitches are fixed by the layouts below (128 B for FP8
+ *    rows, 1152 B for 576-wide bf16 rows).
+ *  - Index sets are returned sorted by key index (ascending), then padded
+ *    with -1. Sets, not orders, are the result.
+ */
+#ifndef DSA_H
+#define DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = -1,     /* bad pointer, size, alignment or layout */
+  DSA_ERR_UNSUPPORTED = -2,     /* valid but not supported (e.g. head count) */
+  DSA_ERR_WORKSPACE = -3,       /* workspace missing or too small */
+  DSA_ERR_CUDA = -4,            /* a CUDA runtime call failed */
+  DSA_ERR_TIMEOUT = -5,         /* a kernel's bounded wait gave up */
+  DSA_ERR_DEVICE_BOUNDS = -6,   /* a kernel met an out-of-range index */
+  DSA_ERR_NOT_IMPLEMENTED = -7
+} dsa_status_t;
+
+typedef void *dsa_stream_t; /* cudaStream_t */
+
+/* Fixed widths of the caches. */
+#define DSA_D_INDEX 128   /* indexer key / query width (e4m3) */
+#define DSA_D_QK 576      /* MLA key width: 512 latent + 64 rope (bf16) */
+#define DSA_D_V 512       /* MLA value width: the latent dims */
+#define DSA_BLOCK 64      /* tokens per block of the paged cache */
+
+/* Human-readable name of a status code. Never NULL. */
+const char *dsa_status_string(int status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int dsa_version(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's error
+ * word. Returns DSA_OK, DSA_ERR_TIMEOUT (takes precedence) or
+ * DSA_ERR_DEVICE_BOUNDS; DSA_ERR_CUDA if the synchronisation itself failed.
+ */
+int dsa_get_device_error(dsa_stream_t stream);
+
+/*
+ * Stage 1, lightning indexer scores (section 4 step 2 of page 3).
+ *
+ *   q8      [T][Hi][128] e4m3 codes of the indexer queries
+ *   q_scale [T] fp32 per-token dequantisation scale, or NULL (= 1)
+ *   k8      [S][128] e4m3 codes of the indexer key cache
+ *   k_scale [S] fp32 per-token scale, or NULL (= 1); must be > 0
+ *   w       [T][Hi] fp32 per-head weights (any sign)
+ *   T, S    query rows and cached keys; query row t sits at position
+ *           q_pos0 + t and sees keys 0 .. min(q_pos0 + t, S - 1)
+ *   Hi      indexer heads: 1, 2, 4, 8, 16, 32 or 64
+ *   scale   positive score scale
+ *   scores  [T][ld] fp32 out: scores[t][s] = I[t,s] for every visible key
+ *           s; entries of later keys are unspecified (a key past the query
+ *           in the same 128-key tile reads -inf, others are not written)
+ *   ld      row pitch of `scores` in elements, >= S, multiple of 4
+ * All positive scales commute with ReLU, so they are applied after the
+ * head sum: I = k_scale[s] * sum_h (w * scale * q_scale[t]) * ReLU(q8 . k8).
+ */
+int dsa_indexer_scores(const void *q8, const float *q_scale, const void *k8,
+                       const float *k_scale, const float *w, int T, int S,
+                       int Hi, int q_pos0, float scale, float *scores,
+                       int64_t ld, dsa_stream_t stream);
+
+/*
+ * Stage 2, per-query top-k (section 4 step 3 of page 3).
+ *
+ *   scores  [T][ld] fp32 as written by dsa_indexer_scores; only the first
+ *           min(q_pos0 + t + 1, S) entries of row t are read
+ *   k       keys to keep per query, 1 .. 65536, multiple of 4
+ *   idx     [T][k] int32 out: the keys with the k largest scores (ties to
+ *           the smaller index), or every visible key when there are at
+ *           most k, sorted by key index and padded with -1
+ *   ld      multiple of 4; `scores` 16-byte aligned
+ */
+int dsa_topk(const float *scores, int T, int S, int64_t ld, int q_pos0, int k,
+             int32_t *idx, dsa_stream_t stream);
+
+/*
+ * Stage 3, sparse MLA forward (section 4 step 4 of page 3).
+ *
+ *   q       [T][H][576] bf16 queries (absorbed MLA form: every head
+ *           attends over the shared latent row)
+ *   kv      [S][576] bf16 latent cache; values are kv[:, :512]
+ *   idx     [T][k] int32 selected key positions in [0, S); -1 entries are
+ *           skipped; k multiple of 4
+ *   H       heads, 1 .. 128
+ *   out     [T][H][512] bf16 out: softmax(sm_scale * q . kv[idx]) kv[idx, :512]
+ *   lse     [T][H] fp32 out (natural log of the softmax denominator,
+ *           including the max), or NULL; -inf when no key is selected
+ */
+int dsa_sparse_mla_fwd(const void *q, const void *kv, const int32_t *idx,
+                       int T, int S, int H, int k, float sm_scale, void *out,
+                       float *lse, dsa_stream_t stream);
+
+/*
+ * Whole prefill path: indexer -> top-k -> sparse MLA for T query rows at
+ * positions q_pos0 .. q_pos0 + T - 1 against S cached keys (S >= q_pos0 + T
+ * for a self-contained prefill). Query rows are scored in chunks of `chunk`
+ * rows (0 = all rows at once); the workspace holds one chunk's scores.
+ *
+ *   idx_out [T][k] int32 out (the selection), or NULL to keep it in the
+ *           workspace only
+ *   workspace  at least dsa_forward_workspace_size() bytes, 256-byte aligned
+ *   other arguments as for the three stages.
+ */
+size_t dsa_forward_workspace_size(int T, int S, int Hi, int H, int k,
+                                  int chunk);
+int dsa_forward(const void *q8, const float *q_scale, const void *k8,
+                const float *k_scale, const float *w, const void *q,
+                const void *kv, int T, int S, int Hi, int H, int q_pos0, int k,
+                int chunk, float scale, float sm_scale, int32_t *idx_out,
+                void *out, float *lse, void *workspace, size_t ws_bytes,
+                dsa_stream_t stream);
+
+/*
+ * Batched decode over a paged cache (blocks of 64 tokens).
+ *
+ *   q8 [B][nq][Hi][128] e4m3, q_scale [B][nq] fp32 (or NULL), w [B][nq][Hi]
+ *   q  [B][nq][H][576] bf16
+ *   k8_pool      [nblk][64][128] e4m3; k_scale_pool [nblk][64] fp32 or NULL
+ *   kv_pool      [nblk][64][576] bf16
+ *   block_table  [B][max_blocks] int32: physical block of each logical
+ *                block of a sequence (entries past the end are not read)
+ *   seq_len      [B] int32: tokens of each sequence, nq <= seq_len[b] <=
+ *                64 * max_blocks (launches are sized from max_blocks, so
+ *                no host copy is needed)
+ *   nq           new query tokens per sequence; query j of sequence b sits
+ *                at position seq_len[b] - nq + j and sees keys 0 .. that
+ *                position (causal between the new tokens)
+ *   idx_out      [B][nq][k] logical key positions out, or NULL
+ *   out [B][nq][H][512] bf16, lse [B][nq][H] fp32 (or NULL)
+ *   workspace    scratch for the per-query score rows, at least
+ *                dsa_decode_paged_workspace_size() bytes, 256-byte aligned
+ */
+size_t dsa_decode_paged_workspace_size(int B, int nq, int max_blocks, int Hi,
+                                       int H, int k);
+int dsa_decode_paged(const void *q8, const float *q_scale, const float *w,
+                     const void *q, const void *k8_pool,
+                     const float *k_scale_pool, const void *kv_pool,
+                     const int32_t *block_table, const int32_t *seq_len,
+                     int B, int nq,
+                     int max_blocks, int nblk, int Hi, int H, int k,
+                     float scale, float sm_scale, int32_t *idx_out, void *out,
+                     float *lse, void *workspace, size_t ws_bytes,
+                     dsa_stream_t stream);
+
+/*
+ * The sparse MLA stage of the paged decode on its own: like
+ * dsa_sparse_mla_fwd, but `idx` [B*nq][k] holds logical positions of each
+ * sequence, translated through block_table into kv_pool rows. A position
+ * past the query's own position counts as out of range.
+ */
+int dsa_sparse_mla_decode_paged(const void *q, const void *kv_pool,
+                                const int32_t *block_table,
+                                const int32_t *seq_len, const int32_t *idx,
+                                int B, int nq, int max_blocks, int nblk, int H,
+                                int k, float sm_scale, void *out, float *lse,
+                                dsa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H */

@@ -1,0 +1,247 @@
+"""Python binding of libdsa.so: DeepSeek Sparse Attention on one B200.
+
+Argument marshalling only: every step of the path runs in the library's
+CUDA kernels (include/dsa.h documents each entry point). PyTorch provides
+device memory and the current stream. Importing this package loads
+libdsa.so and raises ImportError when it has not been built (build with
+``python sparse_attention_long_02_b200/build.py``); there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdsa.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "dsa.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python sparse_attention_long_02_b200/build.py`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+P, I32, I64, F32, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+
+
+def _sig(name, res, *args):
+    fn = getattr(_lib, name)
+    fn.restype = res
+    fn.argtypes = list(args)
+    return fn
+
+
+_sig("dsa_status_string", ctypes.c_char_p, I32)
+_sig("dsa_version", I32)
+_sig("dsa_get_device_error", I32, P)
+_sig("dsa_indexer_scores", I32, P, P, P, P, P, I32, I32, I32, I32, F32, P, I64, P)
+_sig("dsa_topk", I32, P, I32, I32, I64, I32, I32, P, P)
+_sig("dsa_sparse_mla_fwd", I32, P, P, P, I32, I32, I32, I32, F32, P, P, P)
+_sig("dsa_forward_workspace_size", SZ, I32, I32, I32, I32, I32, I32)
+_sig("dsa_forward", I32, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, F32, F32,
+     P, P, P, P, SZ, P)
+_sig("dsa_decode_paged_workspace_size", SZ, I32, I32, I32, I32, I32, I32)
+_sig("dsa_decode_paged", I32, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32,
+     F32, F32, P, P, P, P, SZ, P)
+_sig("dsa_sparse_mla_decode_paged", I32, P, P, P, P, P, I32, I32, I32, I32, I32, I32, F32, P,
+     P, P)
+
+DSA_OK = 0
+STATUS = {0: "DSA_OK", -1: "DSA_ERR_INVALID_ARG", -2: "DSA_ERR_UNSUPPORTED",
+          -3: "DSA_ERR_WORKSPACE", -4: "DSA_ERR_CUDA", -5: "DSA_ERR_TIMEOUT",
+          -6: "DSA_ERR_DEVICE_BOUNDS", -7: "DSA_ERR_NOT_IMPLEMENTED"}
+
+
+class DSAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.dsa_status_string(status).decode()
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({msg})")
+
+
+def lib():
+    """The loaded ctypes library (for callers that use the raw C ABI)."""
+    return _lib
+
+
+def declared_functions():
+    """Names of the functions include/dsa.h declares."""
+    text = open(HEADER_PATH).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]*?\b(dsa_\w+)\s*\(", text, re.M)))
+
+
+def _check(status, where):
+    if status != DSA_OK:
+        raise DSAError(status, where)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _u8(t):
+    if t.dtype == torch.float8_e4m3fn:
+        t = t.view(torch.uint8)
+    if t.dtype != torch.uint8:
+        raise TypeError("FP8 inputs must be uint8 codes or float8_e4m3fn")
+    return _dev(t)
+
+
+def _dev(t, dtype=None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t
+
+
+def _ld(S):
+    return (S + 3) // 4 * 4
+
+
+def get_device_error(stream=None) -> int:
+    """Synchronise and read-and-clear the device error word (a status code)."""
+    return _lib.dsa_get_device_error(_stream(stream))
+
+
+def check_device_error(stream=None):
+    _check(get_device_error(stream), "device")
+
+
+def indexer_scores(q8, q_scale, k8, k_scale, w, scale, q_pos0=0, scores=None, stream=None):
+    """I[t, s] for every visible key -> float32 [T][ld] (ld = S rounded up to 4)."""
+    q8, k8 = _u8(q8), _u8(k8)
+    w = _dev(w, torch.float32)
+    T, Hi = q8.shape[0], q8.shape[1]
+    S = k8.shape[0]
+    if scores is None:
+        scores = torch.empty(T, _ld(S), dtype=torch.float32, device=q8.device)
+    _check(_lib.dsa_indexer_scores(_p(q8), _p(_dev(q_scale, torch.float32)), _p(k8),
+                                   _p(_dev(k_scale, torch.float32)), _p(w), T, S, Hi, q_pos0,
+                                   float(scale), _p(_dev(scores, torch.float32)),
+                                   scores.shape[1], _stream(stream)), "dsa_indexer_scores")
+    return scores
+
+
+def topk(scores, S, k, q_pos0=0, idx=None, stream=None):
+    """Selected keys per row -> int32 [T][k], sorted by key, -1 padded."""
+    scores = _dev(scores, torch.float32)
+    T = scores.shape[0]
+    if idx is None:
+        idx = torch.empty(T, k, dtype=torch.int32, device=scores.device)
+    _check(_lib.dsa_topk(_p(scores), T, S, scores.shape[1], q_pos0, k, _p(_dev(idx, torch.int32)),
+                         _stream(stream)), "dsa_topk")
+    return idx
+
+
+def sparse_mla(q, kv, idx, sm_scale, out=None, lse=None, with_lse=True, stream=None):
+    """Sparse MLA over the selected rows -> (out bf16 [T][H][512], lse f32 [T][H])."""
+    q = _dev(q, torch.bfloat16)
+    kv = _dev(kv, torch.bfloat16)
+    idx = _dev(idx, torch.int32)
+    T, H = q.shape[0], q.shape[1]
+    S, k = kv.shape[0], idx.shape[1]
+    if out is None:
+        out = torch.empty(T, H, 512, dtype=torch.bfloat16, device=q.device)
+    if lse is None and with_lse:
+        lse = torch.empty(T, H, dtype=torch.float32, device=q.device)
+    _check(_lib.dsa_sparse_mla_fwd(_p(q), _p(kv), _p(idx), T, S, H, k, float(sm_scale), _p(out),
+                                   _p(lse), _stream(stream)), "dsa_sparse_mla_fwd")
+    return out, lse
+
+
+def forward_workspace_size(T, S, Hi, H, k, chunk=0) -> int:
+    return int(_lib.dsa_forward_workspace_size(T, S, Hi, H, k, chunk))
+
+
+def forward(q8, q_scale, k8, k_scale, w, q, kv, k, scale, sm_scale, q_pos0=0, chunk=0,
+            idx=None, out=None, lse=None, workspace=None, return_idx=True, stream=None):
+    """Whole prefill path -> (out, lse, idx or None)."""
+    q8, k8 = _u8(q8), _u8(k8)
+    q, kv = _dev(q, torch.bfloat16), _dev(kv, torch.bfloat16)
+    T, Hi = q8.shape[0], q8.shape[1]
+    S, H = k8.shape[0], q.shape[1]
+    dev = q.device
+    if out is None:
+        out = torch.empty(T, H, 512, dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty(T, H, dtype=torch.float32, device=dev)
+    if idx is None and return_idx:
+        idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+    need = forward_workspace_size(T, S, Hi, H, k, chunk)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _check(_lib.dsa_forward(_p(q8), _p(_dev(q_scale, torch.float32)), _p(k8),
+                            _p(_dev(k_scale, torch.float32)), _p(_dev(w, torch.float32)), _p(q),
+                            _p(kv), T, S, Hi, H, q_pos0, k, chunk, float(scale), float(sm_scale),
+                            _p(idx), _p(out), _p(lse), _p(workspace), workspace.numel(),
+                            _stream(stream)), "dsa_forward")
+    return out, lse, idx
+
+
+def decode_workspace_size(B, nq, max_blocks, Hi, H, k) -> int:
+    return int(_lib.dsa_decode_paged_workspace_size(B, nq, max_blocks, Hi, H, k))
+
+
+def decode_paged(q8, q_scale, w, q, k8_pool, k_scale_pool, kv_pool, block_table, seq_len, k,
+                 scale, sm_scale, idx=None, out=None, lse=None, workspace=None,
+                 return_idx=True, stream=None):
+    """Paged decode -> (out [B][nq][H][512], lse [B][nq][H], idx [B][nq][k] or None)."""
+    q8, k8_pool = _u8(q8), _u8(k8_pool)
+    q, kv_pool = _dev(q, torch.bfloat16), _dev(kv_pool, torch.bfloat16)
+    block_table = _dev(block_table, torch.int32)
+    seq_len = _dev(seq_len, torch.int32)
+    B, nq, Hi = q8.shape[0], q8.shape[1], q8.shape[2]
+    H = q.shape[2]
+    nblk, max_blocks = k8_pool.shape[0], block_table.shape[1]
+    dev = q.device
+    if out is None:
+        out = torch.empty(B, nq, H, 512, dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty(B, nq, H, dtype=torch.float32, device=dev)
+    if idx is None and return_idx:
+        idx = torch.empty(B, nq, k, dtype=torch.int32, device=dev)
+    need = decode_workspace_size(B, nq, max_blocks, Hi, H, k)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _check(_lib.dsa_decode_paged(_p(q8), _p(_dev(q_scale, torch.float32)),
+                                 _p(_dev(w, torch.float32)), _p(q), _p(k8_pool),
+                                 _p(_dev(k_scale_pool, torch.float32)), _p(kv_pool),
+                                 _p(block_table), _p(seq_len), B, nq, max_blocks, nblk, Hi, H, k,
+                                 float(scale), float(sm_scale), _p(idx), _p(out), _p(lse),
+                                 _p(workspace), workspace.numel(), _stream(stream)),
+           "dsa_decode_paged")
+    return out, lse, idx
+
+
+def sparse_mla_decode_paged(q, kv_pool, block_table, seq_len, idx, sm_scale, out=None, lse=None,
+                            stream=None):
+    """Sparse MLA of the paged decode for given logical selections."""
+    q, kv_pool = _dev(q, torch.bfloat16), _dev(kv_pool, torch.bfloat16)
+    block_table, seq_len = _dev(block_table, torch.int32), _dev(seq_len, torch.int32)
+    idx = _dev(idx, torch.int32)
+    B, nq, H = q.shape[0], q.shape[1], q.shape[2]
+    k = idx.shape[-1]
+    dev = q.device
+    if out is None:
+        out = torch.empty(B, nq, H, 512, dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty(B, nq, H, dtype=torch.float32, device=dev)
+    _check(_lib.dsa_sparse_mla_decode_paged(_p(q), _p(kv_pool), _p(block_table), _p(seq_len),
+                                            _p(idx), B, nq, block_table.shape[1],
+                                            kv_pool.shape[0], H, k, float(sm_scale), _p(out),
+                                            _p(lse), _stream(stream)),
+           "dsa_sparse_mla_decode_paged")
+    return out, lse

@@ -1,0 +1,331 @@
+// api.cu -- the C ABI of libdsa.so (declared in include/dsa.h): host-side
+// argument checks, tensor-map construction, workspace carving and the launch
+// sequence of each entry point. No device memory is allocated here.
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/dsa.h"
+#include "common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+
+// Per-device error word; kernels get its address as an argument.
+__device__ unsigned g_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+unsigned* g_err_ptr[kMaxDevices] = {};
+std::mutex g_mu;
+
+// Address of the current device's error word (looked up once per device).
+unsigned* device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<unsigned*>(p);
+  }
+  return g_err_ptr[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+
+}  // namespace
+
+cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                         uint64_t inner, uint64_t rows, uint64_t row_stride, uint32_t box_inner,
+                         uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_stride};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace dsa
+
+using namespace dsa;
+
+namespace {
+
+bool valid_hi(int Hi) {
+  return Hi == 1 || Hi == 2 || Hi == 4 || Hi == 8 || Hi == 16 || Hi == 32 || Hi == 64;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int run_indexer(const void* q8, const float* q_scale, const void* k8, const float* k_scale,
+                const float* w, int T, int S, int Hi, int q_pos0, float scale, float* scores,
+                int64_t ld, cudaStream_t st) {
+  IndexerArgs a;
+  a.T = T;
+  a.S = S;
+  a.Hi = Hi;
+  a.q_pos0 = q_pos0;
+  a.scale = scale;
+  a.w = w;
+  a.q_scale = q_scale;
+  a.k_scale = k_scale;
+  a.scores = scores;
+  a.ld = ld;
+  a.err = device_error_word();
+  if (!a.err) return DSA_ERR_CUDA;
+  return status_of(launch_indexer(a, q8, k8, S, st));
+}
+
+int run_topk(const float* scores, int rows, int S, int64_t ld, int q_pos0, const int* seq_len,
+             int nq, int k, int32_t* idx, cudaStream_t st) {
+  TopkArgs a;
+  a.scores = scores;
+  a.ld = ld;
+  a.rows = rows;
+  a.k = k;
+  a.q_pos0 = q_pos0;
+  a.S = S;
+  a.seq_len = seq_len;
+  a.nq = nq;
+  a.idx = idx;
+  a.err = device_error_word();
+  if (!a.err) return DSA_ERR_CUDA;
+  return status_of(launch_topk(a, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dsa_status_string(int status) {
+  switch (status) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case DSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case DSA_ERR_CUDA: return "CUDA runtime error";
+    case DSA_ERR_TIMEOUT: return "kernel wait timed out";
+    case DSA_ERR_DEVICE_BOUNDS: return "kernel met an out-of-range index";
+    case DSA_ERR_NOT_IMPLEMENTED: return "not implemented";
+    default: return "unknown status";
+  }
+}
+
+int dsa_version(void) { return 100; }
+
+int dsa_get_device_error(dsa_stream_t stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  unsigned* p = device_error_word();
+  if (!p) return DSA_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpy(&v, p, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return DSA_ERR_CUDA;
+  if (v != 0 && cudaMemset(p, 0, sizeof v) != cudaSuccess) return DSA_ERR_CUDA;
+  if (v & kErrTimeout) return DSA_ERR_TIMEOUT;
+  if (v & kErrBounds) return DSA_ERR_DEVICE_BOUNDS;
+  return DSA_OK;
+}
+
+int dsa_indexer_scores(const void* q8, const float* q_scale, const void* k8, const float* k_scale,
+                       const float* w, int T, int S, int Hi, int q_pos0, float scale,
+                       float* scores, int64_t ld, dsa_stream_t stream) {
+  if (!q8 || !k8 || !w || !scores || T < 0 || S < 0 || q_pos0 < 0 || !(scale > 0.f) ||
+      ld < S || (ld & 3) || !aligned16(q8) || !aligned16(k8) || !aligned16(scores))
+    return DSA_ERR_INVALID_ARG;
+  if (!valid_hi(Hi)) return DSA_ERR_UNSUPPORTED;
+  if (T == 0 || S == 0) return DSA_OK;
+  return run_indexer(q8, q_scale, k8, k_scale, w, T, S, Hi, q_pos0, scale, scores, ld,
+                     static_cast<cudaStream_t>(stream));
+}
+
+int dsa_topk(const float* scores, int T, int S, int64_t ld, int q_pos0, int k, int32_t* idx,
+             dsa_stream_t stream) {
+  if (!scores || !idx || T < 0 || S < 0 || q_pos0 < 0 || k <= 0 || k > 65536 || (k & 3) ||
+      ld < S || (ld & 3) || !aligned16(scores) || !aligned16(idx))
+    return DSA_ERR_INVALID_ARG;
+  if (T == 0) return DSA_OK;
+  return run_topk(scores, T, S, ld, q_pos0, nullptr, 1, k, idx, static_cast<cudaStream_t>(stream));
+}
+
+static int mla_common(const void* q, const void* kv, const int32_t* idx, int T, int S, int H, int k,
+                      float sm_scale, void* out, float* lse, const int32_t* block_table,
+                      const int32_t* seq_len, int max_blocks, int nblk, int nq,
+                      cudaStream_t st) {
+  if (!q || !kv || !idx || !out || T < 0 || S < 0 || k <= 0 || (k & 3) || !(sm_scale > 0.f) ||
+      !aligned16(q) || !aligned16(kv) || !aligned16(idx) || !aligned16(out))
+    return DSA_ERR_INVALID_ARG;
+  if (H < 1 || H > 128) return DSA_ERR_UNSUPPORTED;
+  if (T == 0) return DSA_OK;
+  MlaArgs a;
+  a.T = T;
+  a.S = S;
+  a.H = H;
+  a.k = k;
+  a.sm_scale_log2 = sm_scale * 1.4426950408889634f;
+  a.idx = idx;
+  a.block_table = block_table;
+  a.seq_len = seq_len;
+  a.max_blocks = max_blocks;
+  a.nblk = nblk;
+  a.nq = nq;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  a.err = device_error_word();
+  if (!a.err) return DSA_ERR_CUDA;
+  const long long kv_rows = block_table ? static_cast<long long>(nblk) * 64 : S;
+  if (kv_rows <= 0) return DSA_ERR_INVALID_ARG;
+  return status_of(launch_sparse_mla(a, q, kv, kv_rows, static_cast<long long>(T) * H, st));
+}
+
+int dsa_sparse_mla_fwd(const void* q, const void* kv, const int32_t* idx, int T, int S, int H,
+                       int k, float sm_scale, void* out, float* lse, dsa_stream_t stream) {
+  if (S <= 0 && T > 0) return DSA_ERR_INVALID_ARG;
+  return mla_common(q, kv, idx, T, S, H, k, sm_scale, out, lse, nullptr, nullptr, 0, 0, 1,
+                    static_cast<cudaStream_t>(stream));
+}
+
+int dsa_sparse_mla_decode_paged(const void* q, const void* kv_pool, const int32_t* block_table,
+                                const int32_t* seq_len, const int32_t* idx, int B, int nq,
+                                int max_blocks, int nblk, int H, int k, float sm_scale, void* out,
+                                float* lse, dsa_stream_t stream) {
+  if (!block_table || !seq_len || B < 0 || nq < 1 || max_blocks < 1 || nblk < 1)
+    return DSA_ERR_INVALID_ARG;
+  return mla_common(q, kv_pool, idx, B * nq, max_blocks * 64, H, k, sm_scale, out, lse,
+                    block_table, seq_len, max_blocks, nblk, nq, static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_forward_workspace_size(int T, int S, int Hi, int H, int k, int chunk) {
+  (void)Hi;
+  (void)H;
+  if (T <= 0 || S <= 0 || k <= 0) return 0;
+  const size_t rows = chunk <= 0 ? T : std::min(chunk, T);
+  const size_t ld = round_up(static_cast<size_t>(S), 4);
+  return round_up(rows * ld * sizeof(float), 256) +
+         round_up(static_cast<size_t>(T) * k * sizeof(int32_t), 256);
+}
+
+int dsa_forward(const void* q8, const float* q_scale, const void* k8, const float* k_scale,
+                const float* w, const void* q, const void* kv, int T, int S, int Hi, int H,
+                int q_pos0, int k, int chunk, float scale, float sm_scale, int32_t* idx_out,
+                void* out, float* lse, void* workspace, size_t ws_bytes, dsa_stream_t stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!q8 || !k8 || !w || !q || !kv || !out || T < 0 || S < 0 || q_pos0 < 0 || k <= 0 ||
+      (k & 3) || !(scale > 0.f) || !(sm_scale > 0.f))
+    return DSA_ERR_INVALID_ARG;
+  if (!valid_hi(Hi)) return DSA_ERR_UNSUPPORTED;
+  if (H < 1 || H > 128) return DSA_ERR_UNSUPPORTED;
+  if (T == 0) return DSA_OK;
+  if (S == 0) return DSA_ERR_INVALID_ARG;
+  const size_t need = dsa_forward_workspace_size(T, S, Hi, H, k, chunk);
+  if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return DSA_ERR_WORKSPACE;
+  const int rows = chunk <= 0 ? T : std::min(chunk, T);
+  const int64_t ld = static_cast<int64_t>(round_up(static_cast<size_t>(S), 4));
+  float* scores = static_cast<float*>(workspace);
+  int32_t* idx = idx_out;
+  if (!idx)
+    idx = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) +
+                                     round_up(static_cast<size_t>(rows) * ld * 4, 256));
+  if (!aligned16(idx)) return DSA_ERR_INVALID_ARG;
+  const uint8_t* q8b = static_cast<const uint8_t*>(q8);
+  for (int c0 = 0; c0 < T; c0 += rows) {
+    const int n = std::min(rows, T - c0);
+    int s = dsa_indexer_scores(q8b + static_cast<size_t>(c0) * Hi * 128,
+                               q_scale ? q_scale + c0 : nullptr, k8, k_scale,
+                               w + static_cast<size_t>(c0) * Hi, n, S, Hi, q_pos0 + c0, scale,
+                               scores, ld, stream);
+    if (s != DSA_OK) return s;
+    s = dsa_topk(scores, n, S, ld, q_pos0 + c0, k, idx + static_cast<size_t>(c0) * k, stream);
+    if (s != DSA_OK) return s;
+  }
+  return dsa_sparse_mla_fwd(q, kv, idx, T, S, H, k, sm_scale, out, lse, st);
+}
+
+size_t dsa_decode_paged_workspace_size(int B, int nq, int max_blocks, int Hi, int H, int k) {
+  (void)Hi;
+  (void)H;
+  if (B <= 0 || nq <= 0 || max_blocks <= 0 || k <= 0) return 0;
+  const size_t rows = static_cast<size_t>(B) * nq;
+  return round_up(rows * max_blocks * 64 * sizeof(float), 256) +
+         round_up(rows * k * sizeof(int32_t), 256);
+}
+
+int dsa_decode_paged(const void* q8, const float* q_scale, const float* w, const void* q,
+                     const void* k8_pool, const float* k_scale_pool, const void* kv_pool,
+                     const int32_t* block_table, const int32_t* seq_len, int B, int nq,
+                     int max_blocks, int nblk, int Hi, int H, int k, float scale, float sm_scale,
+                     int32_t* idx_out, void* out, float* lse, void* workspace, size_t ws_bytes,
+                     dsa_stream_t stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!q8 || !w || !q || !k8_pool || !kv_pool || !block_table || !seq_len || !out || B < 0 ||
+      nq < 1 || max_blocks < 1 || nblk < 1 || k <= 0 || (k & 3) || !(scale > 0.f) ||
+      !(sm_scale > 0.f) || !aligned16(q8) || !aligned16(k8_pool) || !aligned16(kv_pool))
+    return DSA_ERR_INVALID_ARG;
+  if (!valid_hi(Hi) || nq * Hi > 256) return DSA_ERR_UNSUPPORTED;
+  if (H < 1 || H > 128) return DSA_ERR_UNSUPPORTED;
+  if (B == 0) return DSA_OK;
+  const size_t need = dsa_decode_paged_workspace_size(B, nq, max_blocks, Hi, H, k);
+  if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return DSA_ERR_WORKSPACE;
+  const int rows = B * nq;
+  const int64_t ld = static_cast<int64_t>(max_blocks) * 64;
+  float* scores = static_cast<float*>(workspace);
+  int32_t* idx = idx_out;
+  if (!idx)
+    idx = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) +
+                                     round_up(static_cast<size_t>(rows) * ld * 4, 256));
+  if (!aligned16(idx)) return DSA_ERR_INVALID_ARG;
+
+  IndexerArgs a;
+  a.Hi = Hi;
+  a.scale = scale;
+  a.w = w;
+  a.q_scale = q_scale;
+  a.k_scale = k_scale_pool;
+  a.scores = scores;
+  a.ld = ld;
+  a.block_table = block_table;
+  a.max_blocks = max_blocks;
+  a.nblk = nblk;
+  a.seq_len = seq_len;
+  a.nq = nq;
+  a.B = B;
+  a.max_ctx = max_blocks * 64;
+  a.err = device_error_word();
+  if (!a.err) return DSA_ERR_CUDA;
+  cudaError_t e = launch_indexer(a, q8, k8_pool, static_cast<long long>(nblk) * 64, st);
+  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  int s = run_topk(scores, rows, 0, ld, 0, seq_len, nq, k, idx, st);
+  if (s != DSA_OK) return s;
+  return dsa_sparse_mla_decode_paged(q, kv_pool, block_table, seq_len, idx, B, nq, max_blocks,
+                                     nblk, H, k, sm_scale, out, lse, stream);
+}
+
+}  // extern "C"

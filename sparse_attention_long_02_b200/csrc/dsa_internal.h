@@ -1,0 +1,68 @@
+// dsa_internal.h -- launch interfaces between the C ABI (api.cu) and the
+// kernels. Not installed; the public interface is include/dsa.h.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+namespace dsa {
+
+struct IndexerArgs {
+  int T = 0, S = 0, Hi = 0, q_pos0 = 0;   // prefill: query rows, keys, heads, first position
+  float scale = 1.f;
+  const float* w = nullptr;               // [queries][Hi]
+  const float* q_scale = nullptr;         // [queries] or null
+  const float* k_scale = nullptr;         // [keys] (contiguous) or [nblk*64] (paged) or null
+  float* scores = nullptr;                // [queries][ld]
+  long long ld = 0;
+  // paged (decode) cache; block_table == nullptr selects the contiguous cache
+  const int* block_table = nullptr;
+  int max_blocks = 0, nblk = 0, nq = 1, B = 0, max_ctx = 0;
+  const int* seq_len = nullptr;
+  unsigned* err = nullptr;
+  // filled in by launch_indexer
+  int n_mma = 0, q_box_rows = 0, tmem_cols = 0, tiles_per_cta = 0;
+};
+
+struct TopkArgs {
+  const float* scores = nullptr;
+  long long ld = 0;
+  int rows = 0, k = 0;
+  int q_pos0 = 0, S = 0;                  // prefill row length min(q_pos0 + r + 1, S)
+  const int* seq_len = nullptr;           // decode row length seq_len[r/nq] - nq + r%nq + 1
+  int nq = 1;
+  int* idx = nullptr;
+  unsigned* err = nullptr;
+};
+
+struct MlaArgs {
+  int T = 0, S = 0, H = 0, k = 0;         // query rows, keys (contiguous), heads, slots per row
+  float sm_scale_log2 = 0.f;              // sm_scale * log2(e)
+  const int* idx = nullptr;               // [T][k]
+  const int* block_table = nullptr;       // paged cache (decode) or null
+  int max_blocks = 0, nblk = 0, nq = 1;
+  const int* seq_len = nullptr;
+  __nv_bfloat16* out = nullptr;           // [T][H][512]
+  float* lse = nullptr;                   // [T][H] or null
+  int kv_rows = 0;                        // rows of the kv tensor map (filled by the launcher)
+  unsigned* err = nullptr;
+};
+
+// 2D tensor map: `rows` rows of `inner` elements, `row_stride` bytes apart.
+cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                         uint64_t inner, uint64_t rows, uint64_t row_stride, uint32_t box_inner,
+                         uint32_t box_rows, CUtensorMapSwizzle swizzle);
+
+cudaError_t launch_indexer(const IndexerArgs& a, const void* q8, const void* k8, long long k_rows,
+                           cudaStream_t st);
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st);
+cudaError_t launch_sparse_mla(const MlaArgs& a, const void* q, const void* kv, long long kv_rows,
+                              long long q_rows, cudaStream_t st);
+
+int indexer_queries_per_cta(int Hi);
+
+}  // namespace dsa

@@ -1,0 +1,330 @@
+// indexer.cu -- lightning indexer scores on sm_100a tensor cores.
+//
+// Computes, for every causal (query t, key s) pair,
+//     I[t,s] = k_scale[s] * sum_h (w[t,h] * scale * q_scale[t]) * ReLU(x[t,h,s]),
+//     x[t,h,s] = sum_{d<128} q8[t,h,d] * k8[s,d]           (e4m3 x e4m3 -> f32)
+// which equals sum_h w[t,h] * ReLU(scale * qf[t,h] . kf[s]) because the
+// scales are positive. Method: "DeepSeek-V3.2-Exp 模型优势与 DSA 工作原理",
+// section 4, step 2 (dot product, mask, scale, per-head weight); FP8 and
+// ReLU: "m.gxzdkb.com/media/457.html", section "秘密武器".
+//
+// Tiling: keys sit on the MMA's M dimension (128 keys = 128 TMEM lanes),
+// queries x heads on N (QB queries x HI heads <= 256 columns), K = 128 is
+// four e4m3 MMAs of K = 32. Each epilogue thread owns one key row of the
+// accumulator and reduces the heads of each query in registers, so the head
+// sum needs no cross-lane traffic. Two TMEM accumulator buffers and two
+// epilogue warpgroups let the MMA of key tile i+1 run under the epilogue of
+// tile i.
+//
+// Warp roles (384 threads): warp 0 = TMA producer, warp 1 = MMA issuer and
+// TMEM owner, warps 4-7 and 8-11 = epilogue groups 0 and 1 (a warp may only
+// touch TMEM lanes 32*(warp%4) .. +31).
+#include "common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+namespace {
+
+constexpr int kIdxThreads = 384;
+constexpr int kKeyTile = 128;      // keys per MMA tile (M)
+constexpr int kStages = 4;         // key-tile ring depth
+constexpr int kKTileBytes = kKeyTile * 128;
+
+struct IdxSmem {
+  // operand tiles first (1024-B aligned by construction of the offsets)
+  uint8_t q[256 * 128];                 // B operand: QB*HI rows x 128 B
+  uint8_t k[kStages][kKTileBytes];      // A operand ring
+  float w[256];                         // w[t,h]*scale*q_scale[t] for the CTA's queries
+  unsigned long long q_full;
+  unsigned long long k_full[kStages];
+  unsigned long long k_empty[kStages];
+  unsigned long long t_full[2];
+  unsigned long long t_empty[2];
+  unsigned long long mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int HI, bool PAGED>
+__global__ void __launch_bounds__(kIdxThreads, 1)
+indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const IndexerArgs a) {
+  constexpr int QB = (256 / HI) < 64 ? (256 / HI) : 64;   // queries per CTA (prefill)
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  IdxSmem& sm = *reinterpret_cast<IdxSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned* err = a.err;
+  if (launch_aborted(err)) return;
+
+  // ------------------------------------------------------------ work unit
+  // Queries [q0, q0+nqb) of sequence `seq` (decode) or of the prefill block;
+  // key tiles [tile0, tile1) of that sequence.
+  int q0, nqb, seq = 0;
+  long long pos0;            // position of query q0
+  long long key_limit;       // keys of this sequence / cache
+  if (PAGED) {
+    seq = blockIdx.y;
+    const int len = a.seq_len[seq];
+    nqb = a.nq;
+    q0 = seq * a.nq;
+    pos0 = static_cast<long long>(len) - a.nq;
+    key_limit = len;
+  } else {
+    const int qb = gridDim.y - 1 - blockIdx.y;     // longest rows first
+    q0 = qb * QB;
+    nqb = min(QB, a.T - q0);
+    pos0 = static_cast<long long>(a.q_pos0) + q0;
+    key_limit = a.S;
+  }
+  const long long last_key = min(pos0 + nqb - 1, key_limit - 1);
+  const int ntiles_total = static_cast<int>((last_key + kKeyTile) / kKeyTile);
+  const int tile0 = blockIdx.x * a.tiles_per_cta;
+  const int tile1 = min(ntiles_total, tile0 + a.tiles_per_cta);
+  if (nqb <= 0 || last_key < 0 || tile0 >= tile1) return;
+  const int ntiles = tile1 - tile0;
+  const int ncol = a.n_mma;                 // MMA N = padded QB*HI (or nq*HI)
+  const uint32_t idesc = idesc_e4m3(128, ncol);
+
+  const int warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&sm.q_full), 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&sm.k_full[i]), 1);
+      mbar_init(smem_u32(&sm.k_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&sm.t_full[i]), 1);
+      mbar_init(smem_u32(&sm.t_empty[i]), 4);
+    }
+    mbar_init(smem_u32(&sm.mma_done), 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  // folded per-(query, head) weights: w * scale * q_scale
+  for (int j = threadIdx.x; j < ncol; j += blockDim.x) {
+    const int qq = j / HI, h = j % HI;
+    float v = 0.f;
+    if (qq < nqb) {
+      const long long t = q0 + qq;
+      const float qs = a.q_scale ? a.q_scale[t] : 1.f;
+      v = a.w[t * HI + h] * (a.scale * qs);
+    }
+    sm.w[j] = v;
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&sm.tmem_base), a.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_expect_tx(smem_u32(&sm.q_full), a.q_box_rows * 128);
+      tma_load_2d(smem_u32(sm.q), &tm_q, smem_u32(&sm.q_full), 0, q0 * HI);
+      int issued = 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int st = i % kStages;
+        if (i >= kStages &&
+            !mbar_wait(smem_u32(&sm.k_empty[st]), ((i / kStages) + 1) & 1, abort_flag, err))
+          break;
+        const uint32_t full = smem_u32(&sm.k_full[st]);
+        mbar_expect_tx(full, kKTileBytes);
+        const int tile = tile0 + i;
+        if (PAGED) {
+          for (int half = 0; half < 2; ++half) {
+            const int lb = 2 * tile + half;               // logical block
+            int pb = 0;
+            if (lb * 64 < key_limit) {
+              pb = a.block_table[static_cast<long long>(seq) * a.max_blocks + lb];
+              if (pb < 0 || pb >= a.nblk) {
+                raise_error(err, kErrBounds);
+                pb = 0;
+              }
+            }
+            tma_load_2d(smem_u32(sm.k[st]) + half * 64 * 128, &tm_k, full, 0, pb * 64);
+          }
+        } else {
+          tma_load_2d(smem_u32(sm.k[st]), &tm_k, full, 0, tile * kKeyTile);
+        }
+        ++issued;
+      }
+      // make sure no copy is still landing when the CTA leaves
+      for (int i = max(0, issued - kStages); i < issued; ++i)
+        mbar_drain(smem_u32(&sm.k_full[i % kStages]), (i / kStages) & 1);
+      mbar_drain(smem_u32(&sm.q_full), 0);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(smem_u32(&sm.q_full), 0, abort_flag, err);
+      const uint64_t bdesc = sdesc_sw128(smem_u32(sm.q), 0, 1024);
+      for (int i = 0; ok && i < ntiles; ++i) {
+        const int st = i % kStages, buf = i & 1;
+        if (!mbar_wait(smem_u32(&sm.k_full[st]), (i / kStages) & 1, abort_flag, err)) break;
+        if (i >= 2 && !mbar_wait(smem_u32(&sm.t_empty[buf]), ((i >> 1) + 1) & 1, abort_flag, err))
+          break;
+        tc_fence_after();
+        const uint64_t adesc = sdesc_sw128(smem_u32(sm.k[st]), 0, 1024);
+        const uint32_t d = tmem + buf * ncol;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)     // 4 x K=32 (32 bytes each)
+          mma_f8f6f4(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0);
+        mma_commit(smem_u32(&sm.k_empty[st]));
+        mma_commit(smem_u32(&sm.t_full[buf]));
+      }
+      mma_commit(smem_u32(&sm.mma_done));
+      mbar_drain(smem_u32(&sm.mma_done), 0);
+    }
+  } else if (warp >= 4) {
+    // --------------------------------------------------------- epilogue
+    const int g = (warp - 4) >> 2;                 // epilogue group = TMEM buffer
+    const int row = 32 * (warp & 3) + lane;        // accumulator row = key in tile
+    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    for (int i = g; i < ntiles; i += 2) {
+      if (!warp_wait(smem_u32(&sm.t_full[g]), (i >> 1) & 1, abort_flag, err)) break;
+      tc_fence_after();
+      const long long s = static_cast<long long>(tile0 + i) * kKeyTile + row;   // logical key
+      const bool key_ok = s < key_limit;
+      float ks = 1.f;
+      if (a.k_scale && key_ok) {
+        if (PAGED) {
+          int pb = a.block_table[static_cast<long long>(seq) * a.max_blocks + (s >> 6)];
+          pb = (pb < 0 || pb >= a.nblk) ? 0 : pb;
+          ks = a.k_scale[static_cast<long long>(pb) * 64 + (s & 63)];
+        } else {
+          ks = a.k_scale[s];
+        }
+      }
+      const uint32_t taddr = tmem + lane_base + g * ncol;
+      auto emit = [&](int qq, float acc) {
+        if (qq >= nqb || !key_ok) return;
+        const long long t = q0 + qq;
+        const long long pos = pos0 + qq;
+        float* out = a.scores + t * a.ld;
+        out[s] = (s <= pos) ? acc * ks : -INFINITY;
+      };
+      if constexpr (HI >= 32) {
+        float acc = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < ncol / 32; ++c) {
+          float v[32];
+          tmem_ld32(taddr + c * 32, v);
+          const float* wp = sm.w + c * 32;
+          float part = 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) part = fmaf(wp[j], fmaxf(v[j], 0.f), part);
+          acc += part;
+          if (((c + 1) * 32) % HI == 0) {
+            emit((c * 32) / HI, acc);
+            acc = 0.f;
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < ncol / 32; ++c) {
+          float v[32];
+          tmem_ld32(taddr + c * 32, v);
+          const float* wp = sm.w + c * 32;
+#pragma unroll
+          for (int qq = 0; qq < 32 / HI; ++qq) {
+            float acc = 0.f;
+#pragma unroll
+            for (int h = 0; h < HI; ++h)
+              acc = fmaf(wp[qq * HI + h], fmaxf(v[qq * HI + h], 0.f), acc);
+            emit(c * (32 / HI) + qq, acc);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.t_empty[g]));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, a.tmem_cols);
+  }
+}
+
+template <int HI, bool PAGED>
+cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const IndexerArgs& a,
+                       dim3 grid, cudaStream_t st) {
+  // Above half the SM's shared memory, so one CTA per SM: a second resident
+  // CTA would only queue on the TMEM allocation.
+  const size_t smem = std::max<size_t>(sizeof(IdxSmem) + 1024, 120 * 1024);
+  auto kern = indexer_kernel<HI, PAGED>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kIdxThreads, smem, st>>>(tq, tk, a);
+  return cudaGetLastError();
+}
+
+template <bool PAGED>
+cudaError_t launch_hi(int Hi, const CUtensorMap& tq, const CUtensorMap& tk, const IndexerArgs& a,
+                      dim3 grid, cudaStream_t st) {
+  switch (Hi) {
+    case 1: return launch_one<1, PAGED>(tq, tk, a, grid, st);
+    case 2: return launch_one<2, PAGED>(tq, tk, a, grid, st);
+    case 4: return launch_one<4, PAGED>(tq, tk, a, grid, st);
+    case 8: return launch_one<8, PAGED>(tq, tk, a, grid, st);
+    case 16: return launch_one<16, PAGED>(tq, tk, a, grid, st);
+    case 32: return launch_one<32, PAGED>(tq, tk, a, grid, st);
+    case 64: return launch_one<64, PAGED>(tq, tk, a, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+int indexer_queries_per_cta(int Hi) {
+  const int qb = 256 / Hi;
+  return qb < 64 ? qb : 64;
+}
+
+static int indexer_tiles_per_cta() { return 64; }
+
+cudaError_t launch_indexer(const IndexerArgs& a_in, const void* q8, const void* k8,
+                           long long k_rows, cudaStream_t st) {
+  IndexerArgs a = a_in;
+  const bool paged = a.block_table != nullptr;
+  const int qb = paged ? a.nq : indexer_queries_per_cta(a.Hi);
+  int n = qb * a.Hi;
+  n = (n + 31) / 32 * 32;                   // the epilogue reads TMEM 32 columns at a time
+  if (n < 32 || n > 256) return cudaErrorInvalidValue;
+  a.n_mma = n;
+  a.q_box_rows = n;
+  a.tmem_cols = 2 * n <= 32 ? 32 : 2 * n <= 64 ? 64 : 2 * n <= 128 ? 128 : 2 * n <= 256 ? 256 : 512;
+  a.tiles_per_cta = indexer_tiles_per_cta();
+
+  CUtensorMap tq, tk;
+  const long long q_rows = paged ? static_cast<long long>(a.B) * a.nq * a.Hi
+                                 : static_cast<long long>(a.T) * a.Hi;
+  cudaError_t e = make_tmap_2d(&tq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, q_rows, 128, 128, n,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_2d(&tk, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, k_rows, 128, 128,
+                   paged ? 64 : kKeyTile, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+
+  dim3 grid;
+  if (paged) {
+    const int max_tiles = (a.max_ctx + kKeyTile - 1) / kKeyTile;
+    grid = dim3((max_tiles + a.tiles_per_cta - 1) / a.tiles_per_cta, a.B);
+    return launch_hi<true>(a.Hi, tq, tk, a, grid, st);
+  }
+  const int nblocks = (a.T + qb - 1) / qb;
+  const long long max_key = std::min<long long>(static_cast<long long>(a.q_pos0) + a.T, a.S);
+  const int max_tiles = static_cast<int>((max_key + kKeyTile - 1) / kKeyTile);
+  grid = dim3((max_tiles + a.tiles_per_cta - 1) / a.tiles_per_cta, nblocks);
+  return launch_hi<false>(a.Hi, tq, tk, a, grid, st);
+}
+
+}  // namespace dsa

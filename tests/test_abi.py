@@ -1,0 +1,80 @@
+"""The C ABI without a GPU: the library loads, exports every declared entry
+point, and rejects bad arguments on the host before touching the device."""
+import ctypes
+import importlib.util
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _build():
+    spec = importlib.util.spec_from_file_location(
+        "dsa_build", os.path.join(ROOT, "sparse_attention_long_02_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    _build()
+    import sparse_attention_long_02_b200 as d
+    return d
+
+
+def test_every_declared_function_is_exported(dsa):
+    names = dsa.declared_functions()
+    header = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(dsa.lib(), n), n
+    # every entry point in the header is extern "C" (no mangling)
+    assert 'extern "C"' in header
+
+
+def test_status_strings(dsa):
+    for s in range(-7, 1):
+        assert dsa.lib().dsa_status_string(s)
+    assert dsa.lib().dsa_status_string(42) == b"unknown status"
+    assert dsa.lib().dsa_version() >= 100
+
+
+def test_host_validation_rejects_before_launch(dsa):
+    L = dsa.lib()
+    # null pointers
+    assert L.dsa_indexer_scores(None, None, None, None, None, 4, 4, 4, 0, 1.0, None, 4, None) == -1
+    assert L.dsa_topk(None, 4, 4, 4, 0, 4, None, None) == -1
+    assert L.dsa_sparse_mla_fwd(None, None, None, 1, 1, 8, 4, 0.1, None, None, None) == -1
+    fake = ctypes.c_void_p(1 << 20)       # aligned, never dereferenced
+    # unsupported indexer head count
+    assert L.dsa_indexer_scores(fake, None, fake, None, fake, 4, 4, 3, 0, 1.0, fake, 4, None) == -2
+    # k not a multiple of 4, ld not a multiple of 4, ld < S
+    assert L.dsa_topk(fake, 4, 4, 4, 0, 6, fake, None) == -1
+    assert L.dsa_topk(fake, 4, 6, 6, 0, 4, fake, None) == -1
+    assert L.dsa_topk(fake, 4, 8, 4, 0, 4, fake, None) == -1
+    # misaligned pointer
+    assert L.dsa_topk(ctypes.c_void_p((1 << 20) + 4), 4, 4, 4, 0, 4, fake, None) == -1
+    # MLA head count out of range
+    assert L.dsa_sparse_mla_fwd(fake, fake, fake, 1, 1, 129, 4, 0.1, fake, None, None) == -2
+    # non-positive scales
+    assert L.dsa_indexer_scores(fake, None, fake, None, fake, 4, 4, 4, 0, 0.0, fake, 4, None) == -1
+    # forward: workspace missing / too small
+    assert L.dsa_forward(fake, None, fake, None, fake, fake, fake, 8, 8, 4, 8, 0, 4, 0, 1.0, 0.1,
+                         None, fake, None, None, 0, None) == -3
+    # empty problems are a no-op
+    assert L.dsa_topk(fake, 0, 4, 4, 0, 4, fake, None) == 0
+
+
+def test_workspace_sizes(dsa):
+    L = dsa.lib()
+    # one chunk of fp32 scores (pitch rounded to 4) + the index rows, each 256-B rounded
+    assert L.dsa_forward_workspace_size(1024, 1024, 4, 8, 256, 0) == 1024 * 1024 * 4 + 1024 * 256 * 4
+    assert L.dsa_forward_workspace_size(131072, 131072, 64, 128, 2048, 4096) == \
+        4096 * 131072 * 4 + 131072 * 2048 * 4
+    assert L.dsa_forward_workspace_size(10, 7, 4, 8, 4, 3) == 256 + 256
+    assert L.dsa_decode_paged_workspace_size(64, 1, 512, 64, 128, 2048) == \
+        64 * 512 * 64 * 4 + 64 * 2048 * 4
+    assert L.dsa_forward_workspace_size(0, 8, 4, 8, 4, 0) == 0

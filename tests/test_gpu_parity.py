@@ -1,0 +1,260 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Tolerances (from the path's definition):
+  * indexer scores: |gpu - oracle| <= 1e-3 * max(|oracle|, A), A = sum_h |w| ReLU(.)
+    (bit-exact on the integer FP8 grid, where every fp32 partial sum is exact);
+  * top-k: identical sets on the grid; on random inputs a key may differ only
+    if its oracle score is within 1e-3 * |tau| of the oracle's k-th score tau;
+  * sparse MLA (bf16 in/out, fp32 accumulate): max-abs <= 2e-2 and
+    mean-abs <= 2e-3 against the float64 oracle on identical selections.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+MLA_MAX_ABS = 2e-2
+MLA_MEAN_ABS = 2e-3
+IDX_REL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    import sparse_attention_long_02_b200 as d
+    return d
+
+
+def cuda(inp):
+    return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+
+
+def no_device_error(dsa):
+    st = dsa.get_device_error()
+    assert st == 0, dsa.STATUS.get(st, st)
+
+
+def assert_mla_close(got, ref, lse=None, ref_lse=None):
+    got = got.float().cpu().numpy().astype(np.float64)
+    err = np.abs(got - ref)
+    assert np.isfinite(got).all()
+    assert err.max() <= MLA_MAX_ABS, err.max()
+    assert err.mean() <= MLA_MEAN_ABS, err.mean()
+    if lse is not None:
+        l = lse.cpu().numpy().astype(np.float64)
+        fin = np.isfinite(ref_lse)
+        assert (np.isfinite(l) == fin).all()
+        np.testing.assert_allclose(l[fin], ref_lse[fin], rtol=1e-4, atol=1e-4)
+
+
+def assert_sets_within_tolerance(gpu_idx, ref_idx, ref_I, k):
+    """Index sets agree except where the oracle score ties the k-th within 1e-3."""
+    for r in range(ref_idx.shape[0]):
+        g = set(int(x) for x in gpu_idx[r] if x >= 0)
+        o = set(int(x) for x in ref_idx[r] if x >= 0)
+        assert len(g) == len(o), r
+        if g == o:
+            continue
+        row = ref_I[r]
+        tau = min(row[i] for i in o)
+        for i in g ^ o:
+            assert abs(row[i] - tau) <= IDX_REL * abs(tau) + 1e-30, (r, i, row[i], tau)
+
+
+# ------------------------------------------------------------ config 1 grid
+
+@pytest.fixture(scope="module")
+def cfg1():
+    inp = W.make_prefill(W.CONFIGS[1])
+    ref = oracle.forward(inp)
+    return inp, ref
+
+
+def test_indexer_bit_exact_on_grid(dsa, cfg1):
+    inp, ref = cfg1
+    g = cuda(inp)
+    sc = dsa.indexer_scores(g["q8"], None, g["k8"], None, g["w"], inp["scale"])
+    no_device_error(dsa)
+    got = sc[:, : inp["S"]].cpu().numpy()
+    vis = np.isfinite(ref["I"])
+    assert np.array_equal(got[vis], ref["I"][vis])
+
+
+def test_topk_bit_exact_on_grid(dsa, cfg1):
+    inp, ref = cfg1
+    scores = torch.from_numpy(ref["I"]).cuda()
+    idx = dsa.topk(scores, inp["S"], inp["k"])
+    no_device_error(dsa)
+    exp = np.sort(np.where(ref["idx"] < 0, np.iinfo(np.int32).max, ref["idx"]), axis=1)
+    exp = np.where(exp == np.iinfo(np.int32).max, -1, exp)
+    assert np.array_equal(idx.cpu().numpy(), exp)
+
+
+def test_sparse_mla_on_oracle_selection(dsa, cfg1):
+    inp, ref = cfg1
+    g = cuda(inp)
+    out, lse = dsa.sparse_mla(g["q"], g["kv"], torch.from_numpy(ref["idx"]).cuda(), inp["sm_scale"])
+    no_device_error(dsa)
+    assert_mla_close(out, ref["out"], lse, ref["lse"])
+
+
+def test_forward_end_to_end_on_grid(dsa, cfg1):
+    inp, ref = cfg1
+    g = cuda(inp)
+    out, lse, idx = dsa.forward(g["q8"], None, g["k8"], None, g["w"], g["q"], g["kv"], inp["k"],
+                                inp["scale"], inp["sm_scale"], chunk=300)
+    no_device_error(dsa)
+    got = idx.cpu().numpy()
+    for r in range(inp["T"]):
+        assert set(got[r][got[r] >= 0]) == set(ref["idx"][r][ref["idx"][r] >= 0]), r
+    assert_mla_close(out, ref["out"], lse, ref["lse"])
+
+
+# ------------------------------------------------------ random FP8 inputs
+
+def _random_prefill(L, Hi, H, k, seed, plant=True):
+    cfg = W.Config(90, "random", "prefill", k=k, Hi=Hi, H=H, seed=seed, L=L,
+                   plant_block=256 if plant else 0, plant_n=16)
+    return W.make_prefill(cfg)
+
+
+@pytest.mark.parametrize("L,Hi,H,k,rows", [
+    (2500, 64, 128, 2048, [0, 1, 777, 2046, 2047, 2048, 2049, 2300, 2499]),
+    (1111, 4, 8, 256, [0, 255, 256, 600, 1110]),
+    (700, 1, 1, 64, [0, 63, 64, 65, 699]),
+    (300, 32, 16, 512, [0, 150, 299]),
+])
+def test_random_prefill_stages(dsa, L, Hi, H, k, rows):
+    inp = _random_prefill(L, Hi, H, k, seed=L + Hi)
+    g = cuda(inp)
+    rows = np.array(rows)
+    sc = dsa.indexer_scores(g["q8"], g["q_scale"], g["k8"], g["k_scale"], g["w"], inp["scale"])
+    out, lse, idx = dsa.forward(g["q8"], g["q_scale"], g["k8"], g["k_scale"], g["w"], g["q"],
+                                g["kv"], k, inp["scale"], inp["sm_scale"])
+    no_device_error(dsa)
+    I, A = oracle.indexer(inp["q8"], inp["q_scale"], inp["k8"], inp["k_scale"], inp["w"],
+                          inp["scale"], rows=rows, with_mag=True)
+    got = sc[rows, :L].cpu().numpy()
+    vis = np.isfinite(I)
+    tol = IDX_REL * np.maximum(np.abs(I), A)
+    assert (np.abs(got[vis] - I[vis]) <= tol[vis] + 1e-30).all()
+    ref_idx = oracle.topk(I, oracle.prefill_row_len(L, L, 0, rows), k)
+    gidx = idx[rows].cpu().numpy()
+    assert_sets_within_tolerance(gidx, ref_idx, I, k)
+    # attention on the GPU's own selection, oracle fed the identical selection
+    full_idx = np.full((L, k), -1, np.int32)
+    full_idx[rows] = gidx
+    ref_out, ref_lse = oracle.sparse_mla(inp["q"], inp["kv"], full_idx, inp["sm_scale"], rows=rows)
+    assert_mla_close(out[rows], ref_out, lse[rows], ref_lse)
+
+
+def test_indexer_offset_chunk_and_ragged_edges(dsa):
+    """Query rows at an offset into the cache; S not a multiple of 128."""
+    inp = _random_prefill(777, 64, 8, 128, seed=5, plant=False)
+    g = cuda(inp)
+    T0, T = 300, 213                       # rows 300..512 as a chunk
+    sc = dsa.indexer_scores(g["q8"][T0:T0 + T].contiguous(), g["q_scale"][T0:T0 + T].contiguous(),
+                            g["k8"], g["k_scale"], g["w"][T0:T0 + T].contiguous(), inp["scale"],
+                            q_pos0=T0)
+    no_device_error(dsa)
+    rows = np.array([0, 1, 100, 212])
+    I, A = oracle.indexer(inp["q8"][T0:T0 + T], inp["q_scale"][T0:T0 + T], inp["k8"],
+                          inp["k_scale"], inp["w"][T0:T0 + T], inp["scale"], q_pos0=T0,
+                          rows=rows, with_mag=True)
+    got = sc[rows, :777].cpu().numpy()
+    vis = np.isfinite(I)
+    assert (np.abs(got[vis] - I[vis]) <= IDX_REL * np.maximum(np.abs(I), A)[vis] + 1e-30).all()
+
+
+def test_mla_short_rows_single_key_and_all_padding(dsa):
+    rng = np.random.default_rng(3)
+    T, S, H, k = 5, 97, 8, 16
+    q = torch.from_numpy(rng.normal(size=(T, H, 576))).to(torch.bfloat16)
+    kv = torch.from_numpy(rng.normal(size=(S, 576))).to(torch.bfloat16)
+    idx = np.full((T, k), -1, np.int32)
+    idx[0, 0] = 96                         # one key: output is that row exactly
+    idx[1, :16] = rng.choice(S, 16, replace=False)
+    idx[2, :3] = [5, 6, 7]
+    # row 3: no key at all -> zeros, lse = -inf
+    idx[4, :7] = rng.choice(S, 7, replace=False)
+    out, lse = dsa.sparse_mla(q.cuda(), kv.cuda(), torch.from_numpy(idx).cuda(), 1 / 24)
+    no_device_error(dsa)
+    ref, ref_lse = oracle.sparse_mla(q, kv, idx, 1 / 24)
+    assert torch.equal(out[0].cpu(), kv[96, :512].expand(H, 512))
+    assert (out[3].float().cpu() == 0).all() and torch.isneginf(lse[3].cpu()).all()
+    assert_mla_close(out, ref, lse, ref_lse)
+
+
+def test_unselected_nan_rows_never_read(dsa):
+    """Poisoning every key outside the selection leaves the output bit-identical."""
+    rng = np.random.default_rng(4)
+    T, S, H, k = 9, 400, 128, 128
+    q = torch.from_numpy(rng.normal(size=(T, H, 576))).to(torch.bfloat16).cuda()
+    kv = torch.from_numpy(rng.normal(size=(S, 576))).to(torch.bfloat16).cuda()
+    idx = torch.from_numpy(np.stack([rng.choice(S, k, replace=False) for _ in range(T)])
+                           .astype(np.int32)).cuda()
+    out, lse = dsa.sparse_mla(q, kv, idx, 1 / 24)
+    poisoned = kv.clone()
+    keep = torch.zeros(S, dtype=torch.bool, device="cuda")
+    keep[idx.flatten().long()] = True
+    poisoned[~keep] = float("nan")
+    out2, lse2 = dsa.sparse_mla(q, poisoned, idx, 1 / 24)
+    no_device_error(dsa)
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+
+
+def test_out_of_range_index_is_reported_and_skipped(dsa):
+    rng = np.random.default_rng(5)
+    T, S, H, k = 2, 64, 8, 8
+    q = torch.from_numpy(rng.normal(size=(T, H, 576))).to(torch.bfloat16).cuda()
+    kv = torch.from_numpy(rng.normal(size=(S, 576))).to(torch.bfloat16).cuda()
+    idx = torch.tensor([[1, 2, 3, 999, -1, -1, -1, -1], [4, 5, -7, 6, -1, -1, -1, -1]],
+                       dtype=torch.int32).cuda()
+    out, _ = dsa.sparse_mla(q, kv, idx, 1 / 24)
+    st = dsa.get_device_error()
+    assert st == -6, st                              # DSA_ERR_DEVICE_BOUNDS
+    assert torch.isfinite(out.float()).all()
+    clean = torch.tensor([[1, 2, 3, -1, -1, -1, -1, -1], [4, 5, 6, -1, -1, -1, -1, -1]],
+                         dtype=torch.int32).cuda()
+    out2, _ = dsa.sparse_mla(q, kv, clean, 1 / 24)
+    no_device_error(dsa)
+    # the -7 entry is simply skipped (slot order does not matter up to rounding)
+    assert (out[0] == out2[0]).all()
+    assert (out[1].float() - out2[1].float()).abs().max() < 1e-2
+
+
+# ------------------------------------------------------------ paged decode
+
+def _small_decode(lens, nq, seed, Hi=64, H=128, k=2048):
+    cfg = W.Config(91, "decode_test", "decode", k=k, Hi=Hi, H=H, seed=seed, nq=nq,
+                   ctx_lo=1, ctx_hi=2)
+    return W.make_decode(cfg, lens=torch.tensor(lens))
+
+
+@pytest.mark.parametrize("lens,nq", [([100, 2048, 2049, 2050, 5000, 9000], 2),
+                                     ([64, 65, 4097, 3000], 1)])
+def test_decode_paged_vs_oracle(dsa, lens, nq):
+    inp = _small_decode(lens, nq, seed=len(lens) + nq)
+    g = cuda(inp)
+    out, lse, idx = dsa.decode_paged(g["q8"], g["q_scale"], g["w"], g["q"], g["k8_pool"],
+                                     g["k_scale_pool"], g["kv_pool"], g["block_table"],
+                                     g["seq_len"], inp["k"], inp["scale"], inp["sm_scale"])
+    no_device_error(dsa)
+    ref = oracle.decode(inp)
+    gidx = idx.cpu().numpy()
+    for b in range(inp["B"]):
+        assert_sets_within_tolerance(gidx[b], ref["idx"][b], ref["I"][b], inp["k"])
+    # MLA on the oracle's selection through the paged stage entry point
+    o2, l2 = dsa.sparse_mla_decode_paged(g["q"], g["kv_pool"], g["block_table"], g["seq_len"],
+                                         torch.from_numpy(ref["idx"]).cuda(), inp["sm_scale"])
+    no_device_error(dsa)
+    assert_mla_close(o2, ref["out"], l2, ref["lse"])
+    same = [b for b in range(inp["B"])
+            if all(set(gidx[b, j]) == set(ref["idx"][b, j]) for j in range(nq))]
+    assert same
+    assert_mla_close(out[same], ref["out"][same], lse[same], ref["lse"][same])
