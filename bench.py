@@ -1,0 +1,487 @@
+"""Benchmark of the DSA hot path on B200: prefill tokens/s at 128K and decode
+queries/s at B=64 x 32K, with roofline fractions and the CPU oracle beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole hot path (indexer -> top-k -> sparse MLA)
+over the prefill workload: one causal prefill of L = 131072 tokens, queries
+scored in 4096-row chunks against the full causal prefix (inputs resident in
+HBM, far larger than L2, so no flush is needed). Under torchrun each rank
+runs its own independent prefill (weak scaling, no data-path collective);
+the reported time is the max over ranks. The decode workload (64 sequences
+x 32768 tokens, paged cache) is timed in the same run, with an L2 flush
+before every iteration, and reported under "decode".
+
+--impl reference times the CPU oracle (the plain C implementation the tests
+compare against) on the host cores, on a stratified sample of query rows of
+the same workload, and prints the same JSON line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "DSA tokens/s: prefill@128K & decode queries/s B=64@32K; % of FP8/HBM roofline"
+PREFILL_CFG = 4
+DECODE_CFG = 3
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--L", type=int, default=0, help="override the prefill length (testing)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ ranks
+
+class Ranks:
+    def __init__(self, gpus):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+        elif torch.cuda.is_available():
+            torch.cuda.set_device(0)
+        self.gpus = gpus
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.barrier()
+            self.pg.destroy_process_group()
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        mhz, maxm, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                maxm = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": maxm,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ------------------------------------------------------------ work counts
+
+def prefill_work(L, Hi, H, k):
+    """Algorithmic work of one causal prefill (no masked pairs, no re-reads)."""
+    pairs = L * (L + 1) // 2                               # causal (t, s) pairs
+    sel = sum(min(t + 1, k) for t in range(L))             # selected (t, key) pairs
+    idx_flops = 2 * 128 * Hi * pairs
+    mla_flops = 2 * (576 + 512) * H * sel
+    # bytes each stage must move at least once
+    idx_bytes = L * Hi * 128 + L * 128 + L * 4 * 2 + L * Hi * 4 + L * k * 4
+    mla_bytes = L * H * 576 * 2 + L * 576 * 2 + L * k * 4 + L * H * 512 * 2 + L * H * 4
+    return dict(pairs=pairs, sel=sel, idx_flops=idx_flops, mla_flops=mla_flops,
+                idx_bytes=idx_bytes, mla_bytes=mla_bytes)
+
+
+def decode_work(lens, nq, Hi, H, k):
+    ctx = [int(n) for n in lens]
+    idx_bytes = sum(n * (128 + 4) for n in ctx) + len(ctx) * nq * (Hi * 128 + Hi * 4 + 4)
+    sel = sum(min(n - nq + j + 1, k) for n in ctx for j in range(nq))
+    mla_bytes = sel * 1152 + len(ctx) * nq * H * (576 * 2 + 512 * 2 + 4)
+    idx_flops = sum(2 * 128 * Hi * (n - nq + j + 1) for n in ctx for j in range(nq))
+    mla_flops = 2 * (576 + 512) * H * sel
+    return dict(idx_bytes=idx_bytes, mla_bytes=mla_bytes, idx_flops=idx_flops,
+                mla_flops=mla_flops, sel=sel)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# --------------------------------------------------------- GPU measurement
+
+def _ev():
+    return torch.cuda.Event(enable_timing=True)
+
+
+def prefill_inputs(L, rank):
+    import dataclasses
+    cfg = dataclasses.replace(W.CONFIGS[PREFILL_CFG], seed=W.CONFIGS[PREFILL_CFG].seed + 1000 * rank)
+    return cfg, W.make_prefill(cfg, device="cuda", L=L)
+
+
+class Prefill:
+    """Preallocated buffers and one call of the whole path per step."""
+
+    def __init__(self, dsa, cfg, inp):
+        self.dsa, self.cfg, self.inp = dsa, cfg, inp
+        T, H, k = inp["T"], inp["H"], inp["k"]
+        self.chunk = cfg.chunk or T
+        self.ws = torch.empty(dsa.forward_workspace_size(T, inp["S"], inp["Hi"], H, k, self.chunk),
+                              dtype=torch.uint8, device="cuda")
+        self.out = torch.empty(T, H, 512, dtype=torch.bfloat16, device="cuda")
+        self.lse = torch.empty(T, H, dtype=torch.float32, device="cuda")
+        self.idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+        self.launches = 2 * math.ceil(T / self.chunk) + 1
+
+    def step(self):
+        i = self.inp
+        self.dsa.forward(i["q8"], i["q_scale"], i["k8"], i["k_scale"], i["w"], i["q"], i["kv"],
+                         i["k"], i["scale"], i["sm_scale"], chunk=self.chunk, idx=self.idx,
+                         out=self.out, lse=self.lse, workspace=self.ws)
+
+    def stages(self, reps=2):
+        """Per-stage device time of one step (ms), events around each stage call."""
+        d, i = self.dsa, self.inp
+        T, S, Hi, k = i["T"], i["S"], i["Hi"], i["k"]
+        ld = (S + 3) // 4 * 4
+        scores = self.ws[: self.chunk * ld * 4].view(torch.float32).view(self.chunk, ld)
+        tot = {"indexer": 0.0, "topk": 0.0, "sparse_mla": 0.0}
+        for _ in range(reps):
+            for c0 in range(0, T, self.chunk):
+                n = min(self.chunk, T - c0)
+                e0, e1, e2 = _ev(), _ev(), _ev()
+                e0.record()
+                d.indexer_scores(i["q8"][c0:c0 + n], i["q_scale"][c0:c0 + n], i["k8"], i["k_scale"],
+                                 i["w"][c0:c0 + n], i["scale"], q_pos0=c0, scores=scores[:n])
+                e1.record()
+                d.topk(scores[:n], S, k, q_pos0=c0, idx=self.idx[c0:c0 + n])
+                e2.record()
+                e2.synchronize()
+                tot["indexer"] += e0.elapsed_time(e1)
+                tot["topk"] += e1.elapsed_time(e2)
+            e0, e1 = _ev(), _ev()
+            e0.record()
+            d.sparse_mla(i["q"], i["kv"], self.idx, i["sm_scale"], out=self.out, lse=self.lse)
+            e1.record()
+            e1.synchronize()
+            tot["sparse_mla"] += e0.elapsed_time(e1)
+        return {s: v / reps for s, v in tot.items()}
+
+
+def time_steps(fn, steps, warmup, ranks, dsa, clock_gpu):
+    for _ in range(warmup):
+        fn()
+    st = dsa.get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error during warm-up: {dsa.STATUS.get(st, st)}")
+    torch.cuda.synchronize()
+    ranks.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(clock_gpu) as clk:
+        e0, e1 = _ev(), _ev()
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        e1.synchronize()
+    torch.cuda.synchronize()
+    ranks.barrier()
+    st = dsa.get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the timed region: {dsa.STATUS.get(st, st)}")
+    return ranks.max(e0.elapsed_time(e1) / steps), clk.summary()
+
+
+def e2e_prefill(pf, steps):
+    """Same path through the binding from pinned host buffers, copies timed."""
+    i = pf.inp
+    names = ["q8", "q_scale", "k8", "k_scale", "w", "q", "kv"]
+    host = {}
+    for n in names:
+        h = torch.empty(i[n].shape, dtype=i[n].dtype, pin_memory=True)
+        h.copy_(i[n])
+        host[n] = h
+    out_h = torch.empty(pf.out.shape, dtype=pf.out.dtype, pin_memory=True)
+    lse_h = torch.empty(pf.lse.shape, dtype=pf.lse.dtype, pin_memory=True)
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+
+    def step():
+        for n in names:
+            i[n].copy_(host[n], non_blocking=True)
+        pf.step()
+        out_h.copy_(pf.out, non_blocking=True)
+        lse_h.copy_(pf.lse, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    e0, e1 = _ev(), _ev()
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del host
+    return ms, h2d, d2h
+
+
+def time_decode(dsa, steps, warmup):
+    cfg = W.CONFIGS[DECODE_CFG]
+    inp = W.make_decode(cfg, device="cuda")
+    g = inp
+    B, nq, k = inp["B"], inp["nq"], inp["k"]
+    ws = torch.empty(dsa.decode_workspace_size(B, nq, inp["max_blocks"], inp["Hi"], inp["H"], k),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.empty(B, nq, inp["H"], 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, nq, inp["H"], dtype=torch.float32, device="cuda")
+    idx = torch.empty(B, nq, k, dtype=torch.int32, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def full():
+        dsa.decode_paged(g["q8"], g["q_scale"], g["w"], g["q"], g["k8_pool"], g["k_scale_pool"],
+                         g["kv_pool"], g["block_table"], g["seq_len"], k, inp["scale"],
+                         inp["sm_scale"], idx=idx, out=out, lse=lse, workspace=ws)
+
+    def mla():
+        dsa.sparse_mla_decode_paged(g["q"], g["kv_pool"], g["block_table"], g["seq_len"], idx,
+                                    inp["sm_scale"], out=out, lse=lse)
+
+    res = {}
+    for name, fn in (("total", full), ("sparse_mla", mla)):
+        for _ in range(warmup):
+            fn()
+        times = []
+        for _ in range(steps):
+            flush.zero_()                                   # L2 flush, outside the events
+            e0, e1 = _ev(), _ev()
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+        res[name] = statistics.median(times)
+    st = dsa.get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in decode: {dsa.STATUS.get(st, st)}")
+    work = decode_work(inp["seq_len"].cpu().tolist(), nq, inp["Hi"], inp["H"], k)
+    return res, work, B * nq
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def oracle_sample(inp, n_rows=32, threads=None):
+    """Time the CPU oracle on query rows spread evenly over t (incl. the last).
+
+    Each row runs the whole path (indexer over its causal prefix, top-k, sparse
+    MLA). Rows are independent; they are shared out over host threads (the C
+    oracle releases the GIL). Since the sample is stratified in t, rows/s
+    estimates the oracle's tokens/s on the full workload.
+    """
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    threads = threads or os.cpu_count() or 1
+    T, k = inp["T"], inp["k"]
+    rows = sorted(set(min(T - 1, int((i + 0.5) * T / n_rows)) for i in range(n_rows)) | {T - 1})
+    r = torch.tensor(rows)
+    host = dict(k8=inp["k8"].cpu(), k_scale=None if inp["k_scale"] is None else inp["k_scale"].cpu(),
+                kv=inp["kv"].cpu(), q8=inp["q8"][r.to(inp["q8"].device)].cpu(),
+                w=inp["w"][r.to(inp["w"].device)].cpu(), q=inp["q"][r.to(inp["q"].device)].cpu(),
+                q_scale=None if inp["q_scale"] is None else inp["q_scale"][r.to(inp["q8"].device)].cpu())
+
+    def one(i):
+        t = rows[i]
+        qs = None if host["q_scale"] is None else host["q_scale"][i:i + 1]
+        I = oracle.indexer(host["q8"][i:i + 1], qs, host["k8"], host["k_scale"], host["w"][i:i + 1],
+                           inp["scale"], q_pos0=t)
+        sel = oracle.topk(I, [min(t + 1, inp["S"])], k)
+        oracle.sparse_mla(host["q"][i:i + 1], host["kv"], sel, inp["sm_scale"])
+
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(one, range(len(rows))))
+    wall = time.perf_counter() - t0
+    return dict(value=len(rows) / wall, unit="tokens/s", cores=threads, kind="oracle",
+                sample=f"{len(rows)} query rows of the L={T} prefill, evenly spaced in t "
+                       f"(incl. the last), whole path per row, {threads} threads; "
+                       f"{wall:.1f} s wall", wall_s=wall)
+
+
+# ------------------------------------------------------------------- main
+
+def config_obj(L, chunk):
+    return {"workload": f"prefill L={L} causal, 4096-row chunks, k=2048, indexer 64x128 FP8, "
+                        "MLA 128 heads x (512+64) bf16; decode B=64 x 32768 paged",
+            "L": L, "chunk": chunk, "k": 2048, "Hi": 64, "H": 128,
+            "l2": "prefill inputs exceed L2 (no flush); decode: 256 MB L2 flush per iteration"}
+
+
+def run_reference(args):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    L = args.L or W.CONFIGS[PREFILL_CFG].L
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    cfg = W.CONFIGS[PREFILL_CFG]
+    inp = W.make_prefill(cfg, device=dev, L=L)
+    for _ in range(args.warmup):
+        oracle_sample(inp, n_rows=8)
+    vals, walls, last = [], [], None
+    for _ in range(args.steps):
+        last = oracle_sample(inp)
+        vals.append(last["value"])
+        walls.append(last["wall_s"])
+    v = statistics.mean(vals)
+    last["value"] = v
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * statistics.mean(walls), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_obj(L, cfg.chunk), "cpu_baseline": last,
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    ranks = Ranks(args.gpus)
+    import sparse_attention_long_02_b200 as dsa
+    pk = peaks()
+    fp8_sus = 2 * pk["bf16_sus"]
+    cfg, inp = prefill_inputs(args.L or W.CONFIGS[PREFILL_CFG].L, ranks.rank)
+    L = inp["T"]
+    pf = Prefill(dsa, cfg, inp)
+    ms, clocks = time_steps(pf.step, args.steps, args.warmup, ranks, dsa, ranks.local)
+    tokens = L * ranks.world
+    value = tokens / (ms / 1e3)
+
+    work = prefill_work(L, inp["Hi"], inp["H"], inp["k"])
+    st = pf.stages()
+    stages = {
+        "indexer": {"ms": st["indexer"], "bound": "tensor", "unit": "TFLOP/s",
+                    "achieved": work["idx_flops"] / (st["indexer"] * 1e-3) / 1e12, "peak": fp8_sus},
+        "topk": {"ms": st["topk"]},
+        "sparse_mla": {"ms": st["sparse_mla"], "bound": "tensor", "unit": "TFLOP/s",
+                       "achieved": work["mla_flops"] / (st["sparse_mla"] * 1e-3) / 1e12,
+                       "peak": pk["bf16_sus"]},
+    }
+    for s in stages.values():
+        if "peak" in s:
+            s["frac"] = s["achieved"] / s["peak"]
+    dom = max(("indexer", "sparse_mla"), key=lambda s: st[s])
+    launches_per_step = {"indexer": math.ceil(L / pf.chunk), "sparse_mla": 1}[dom]
+    roof = {"kernel": dom, "bound": "tensor", "achieved": stages[dom]["achieved"],
+            "peak": stages[dom]["peak"], "unit": "TFLOP/s", "frac": stages[dom]["frac"],
+            "traffic": None, "launches_per_step": launches_per_step,
+            "peak_src": f"{pk['src']} sustained bf16" + (" x2 (FP8/BF16 nominal ratio)"
+                                                         if dom == "indexer" else "")}
+    t_roof = max(work["idx_flops"] / (fp8_sus * 1e12), work["idx_bytes"] / (pk["hbm"] * 1e9)) + \
+        max(work["mla_flops"] / (pk["bf16_sus"] * 1e12), work["mla_bytes"] / (pk["hbm"] * 1e9))
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ranks.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8 indexer / bf16 MLA, fp32 accumulate", "data": "synthetic",
+            "config": config_obj(L, pf.chunk), "clocks": clocks,
+            "gpu_launches": pf.launches * args.steps,
+            "roofline": roof, "stages": stages,
+            "end_to_end_roofline": {"ms": 1e3 * t_roof, "frac": 1e3 * t_roof / ms}}
+    if not args.no_decode:
+        dres, dwork, nqueries = time_decode(dsa, max(args.steps, 10), args.warmup)
+        mla_gbs = dwork["mla_bytes"] / (dres["sparse_mla"] * 1e-3) / 1e9
+        line["decode"] = {
+            "workload": "B=64 x 32768, nq=1, paged (block 64), k=2048, 64x128 FP8 indexer, "
+                        "MLA 128 heads", "value": nqueries * ranks.world / (dres["total"] * 1e-3),
+            "unit": "queries/s", "ms": dres["total"],
+            "sparse_mla": {"ms": dres["sparse_mla"], "bound": "hbm", "achieved": mla_gbs,
+                           "peak": pk["hbm"], "unit": "GB/s", "frac": mla_gbs / pk["hbm"]},
+            "indexer_topk_ms": dres["total"] - dres["sparse_mla"]}
+    if not args.no_e2e:
+        e_ms, h2d, d2h = e2e_prefill(pf, max(1, min(args.steps, 3)))
+        line["e2e"] = {"value": tokens / (ranks.max(e_ms) / 1e3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    if ranks.rank == 0 and ranks.world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = oracle_sample(inp)
+    ranks.close()
+    if ranks.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

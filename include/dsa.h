@@ -72,6 +72,13 @@ const char *dsa_status_string(int status);
 int dsa_version(void);
 
 /*
+ * Text of the last CUDA runtime error an entry point of this thread turned
+ * into DSA_ERR_CUDA ("" if none). The string is owned by the library and
+ * stays valid until the next failing call on the same thread.
+ */
+const char *dsa_last_error_string(void);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's error
  * word. Returns DSA_OK, DSA_ERR_TIMEOUT (takes precedence) or
  * DSA_ERR_DEVICE_BOUNDS; DSA_ERR_CUDA if the synchronisation itself failed.

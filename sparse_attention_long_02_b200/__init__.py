@@ -36,6 +36,7 @@ def _sig(name, res, *args):
 
 _sig("dsa_status_string", ctypes.c_char_p, I32)
 _sig("dsa_version", I32)
+_sig("dsa_last_error_string", ctypes.c_char_p)
 _sig("dsa_get_device_error", I32, P)
 _sig("dsa_indexer_scores", I32, P, P, P, P, P, I32, I32, I32, I32, F32, P, I64, P)
 _sig("dsa_topk", I32, P, I32, I32, I64, I32, I32, P, P)
@@ -59,6 +60,8 @@ class DSAError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         msg = _lib.dsa_status_string(status).decode()
+        if status == -4:
+            msg += ": " + _lib.dsa_last_error_string().decode()
         super().__init__(f"{where}: {STATUS.get(status, status)} ({msg})")
 
 

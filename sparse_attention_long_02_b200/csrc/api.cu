@@ -53,7 +53,13 @@ EncodeTiledFn encode_tiled() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-int status_of(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+thread_local char g_last_error[256] = "";
+
+int status_of(cudaError_t e) {
+  if (e == cudaSuccess) return DSA_OK;
+  snprintf(g_last_error, sizeof g_last_error, "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return DSA_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -139,6 +145,8 @@ const char* dsa_status_string(int status) {
 }
 
 int dsa_version(void) { return 100; }
+
+const char* dsa_last_error_string(void) { return g_last_error; }
 
 int dsa_get_device_error(dsa_stream_t stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -320,9 +328,9 @@ int dsa_decode_paged(const void* q8, const float* q_scale, const float* w, const
   a.max_ctx = max_blocks * 64;
   a.err = device_error_word();
   if (!a.err) return DSA_ERR_CUDA;
-  cudaError_t e = launch_indexer(a, q8, k8_pool, static_cast<long long>(nblk) * 64, st);
-  if (e != cudaSuccess) return DSA_ERR_CUDA;
-  int s = run_topk(scores, rows, 0, ld, 0, seq_len, nq, k, idx, st);
+  int s = status_of(launch_indexer(a, q8, k8_pool, static_cast<long long>(nblk) * 64, st));
+  if (s != DSA_OK) return s;
+  s = run_topk(scores, rows, 0, ld, 0, seq_len, nq, k, idx, st);
   if (s != DSA_OK) return s;
   return dsa_sparse_mla_decode_paged(q, kv_pool, block_table, seq_len, idx, B, nq, max_blocks,
                                      nblk, H, k, sm_scale, out, lse, stream);

@@ -63,14 +63,14 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   long long pos0;            // position of query q0
   long long key_limit;       // keys of this sequence / cache
   if (PAGED) {
-    seq = blockIdx.y;
+    seq = blockIdx.x;
     const int len = a.seq_len[seq];
     nqb = a.nq;
     q0 = seq * a.nq;
     pos0 = static_cast<long long>(len) - a.nq;
     key_limit = len;
   } else {
-    const int qb = gridDim.y - 1 - blockIdx.y;     // longest rows first
+    const int qb = gridDim.x - 1 - blockIdx.x;     // longest rows first
     q0 = qb * QB;
     nqb = min(QB, a.T - q0);
     pos0 = static_cast<long long>(a.q_pos0) + q0;
@@ -78,7 +78,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   }
   const long long last_key = min(pos0 + nqb - 1, key_limit - 1);
   const int ntiles_total = static_cast<int>((last_key + kKeyTile) / kKeyTile);
-  const int tile0 = blockIdx.x * a.tiles_per_cta;
+  const int tile0 = blockIdx.y * a.tiles_per_cta;
   const int tile1 = min(ntiles_total, tile0 + a.tiles_per_cta);
   if (nqb <= 0 || last_key < 0 || tile0 >= tile1) return;
   const int ntiles = tile1 - tile0;
@@ -317,13 +317,13 @@ cudaError_t launch_indexer(const IndexerArgs& a_in, const void* q8, const void* 
   dim3 grid;
   if (paged) {
     const int max_tiles = (a.max_ctx + kKeyTile - 1) / kKeyTile;
-    grid = dim3((max_tiles + a.tiles_per_cta - 1) / a.tiles_per_cta, a.B);
+    grid = dim3(a.B, (max_tiles + a.tiles_per_cta - 1) / a.tiles_per_cta);
     return launch_hi<true>(a.Hi, tq, tk, a, grid, st);
   }
   const int nblocks = (a.T + qb - 1) / qb;
   const long long max_key = std::min<long long>(static_cast<long long>(a.q_pos0) + a.T, a.S);
   const int max_tiles = static_cast<int>((max_key + kKeyTile - 1) / kKeyTile);
-  grid = dim3((max_tiles + a.tiles_per_cta - 1) / a.tiles_per_cta, nblocks);
+  grid = dim3(nblocks, (max_tiles + a.tiles_per_cta - 1) / a.tiles_per_cta);
   return launch_hi<false>(a.Hi, tq, tk, a, grid, st);
 }
 

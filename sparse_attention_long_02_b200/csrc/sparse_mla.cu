@@ -94,7 +94,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const uint32_t rank = cluster_rank();
   const uint32_t peer = rank ^ 1u;
   const int nat = rank == 0 ? 5 : 4;
-  const int r = blockIdx.y;                      // query row
+  const int r = blockIdx.x >> 1;                 // query row (one cluster per row)
   const int seq = A.block_table ? r / A.nq : 0;
   // keys a slot may name: the causal prefix of the query (paged) or the cache
   int limit = A.S;
@@ -375,7 +375,7 @@ cudaError_t launch_sparse_mla(const MlaArgs& a_in, const void* q, const void* kv
   e = cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid(2, a.T);
+  dim3 grid(2 * a.T);      // x has no 65535 limit; cluster pairs are consecutive x
   sparse_mla_kernel<<<grid, kMlaThreads, smem, st>>>(tq, tkv, a);
   return cudaGetLastError();
 }
