@@ -193,6 +193,37 @@ int dsa_decode_paged(const void *q8, const float *q_scale, const float *w,
                      dsa_stream_t stream);
 
 /*
+ * Paged decode that allocates nothing, for callers that cannot allocate
+ * device memory: code running where cudaMalloc is not allowed or not safe
+ * (a host callback, a plugin living inside another framework's memory
+ * pool, a tool with no device allocator of its own). The pages describe no
+ * such entry point; it is a convenience of this library.
+ *
+ * Same arguments and results as dsa_decode_paged(), without the workspace.
+ * The scratch is a fixed 32 MiB array inside the library, present on every
+ * GPU that loads libdsa.so until the process exits. A call whose scratch
+ * need, dsa_decode_paged_workspace_size(B, nq, max_blocks, Hi, H, k), is
+ * above 32 MiB is rejected with DSA_ERR_WORKSPACE before anything is
+ * launched (dsa_last_error_string() says why).
+ *  - The first call on each device looks up the array's device address
+ *    with that device current; make that first call before any stream
+ *    capture begins.
+ *  - All calls on a device share the one array. Calls whose GPU work
+ *    overlaps (different streams, or different host threads, without
+ *    ordering between them) race on it; serialise them. Every byte a call
+ *    reads from the scratch is written earlier in the same call, so the
+ *    previous call's leftovers never leak into a result.
+ */
+int dsa_decode_paged_noalloc(const void *q8, const float *q_scale,
+                             const float *w, const void *q,
+                             const void *k8_pool, const float *k_scale_pool,
+                             const void *kv_pool, const int32_t *block_table,
+                             const int32_t *seq_len, int B, int nq,
+                             int max_blocks, int nblk, int Hi, int H, int k,
+                             float scale, float sm_scale, int32_t *idx_out,
+                             void *out, float *lse, dsa_stream_t stream);
+
+/*
  * The sparse MLA stage of the paged decode on its own: like
  * dsa_sparse_mla_fwd, but `idx` [B*nq][k] holds logical positions of each
  * sequence, translated through block_table into kv_pool rows. A position

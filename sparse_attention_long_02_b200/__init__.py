@@ -47,6 +47,8 @@ _sig("dsa_forward", I32, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32,
 _sig("dsa_decode_paged_workspace_size", SZ, I32, I32, I32, I32, I32, I32)
 _sig("dsa_decode_paged", I32, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32,
      F32, F32, P, P, P, P, SZ, P)
+_sig("dsa_decode_paged_noalloc", I32, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32,
+     I32, F32, F32, P, P, P, P)
 _sig("dsa_sparse_mla_decode_paged", I32, P, P, P, P, P, I32, I32, I32, I32, I32, I32, F32, P,
      P, P)
 
@@ -248,3 +250,31 @@ def sparse_mla_decode_paged(q, kv_pool, block_table, seq_len, idx, sm_scale, out
                                             _p(lse), _stream(stream)),
            "dsa_sparse_mla_decode_paged")
     return out, lse
+
+
+def decode_paged_noalloc(q8, q_scale, w, q, k8_pool, k_scale_pool, kv_pool, block_table, seq_len,
+                         k, scale, sm_scale, idx=None, out=None, lse=None, stream=None):
+    """Paged decode whose scratch is the library's fixed device array (no workspace).
+
+    For callers that cannot allocate device memory; see dsa_decode_paged_noalloc
+    in include/dsa.h for the size limit and the sharing rules.
+    """
+    q8, k8_pool = _u8(q8), _u8(k8_pool)
+    q, kv_pool = _dev(q, torch.bfloat16), _dev(kv_pool, torch.bfloat16)
+    block_table = _dev(block_table, torch.int32)
+    seq_len = _dev(seq_len, torch.int32)
+    B, nq, Hi = q8.shape[0], q8.shape[1], q8.shape[2]
+    H = q.shape[2]
+    dev = q.device
+    if out is None:
+        out = torch.empty(B, nq, H, 512, dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty(B, nq, H, dtype=torch.float32, device=dev)
+    _check(_lib.dsa_decode_paged_noalloc(_p(q8), _p(_dev(q_scale, torch.float32)),
+                                         _p(_dev(w, torch.float32)), _p(q), _p(k8_pool),
+                                         _p(_dev(k_scale_pool, torch.float32)), _p(kv_pool),
+                                         _p(block_table), _p(seq_len), B, nq,
+                                         block_table.shape[1], k8_pool.shape[0], Hi, H, k,
+                                         float(scale), float(sm_scale), _p(idx), _p(out), _p(lse),
+                                         _stream(stream)), "dsa_decode_paged_noalloc")
+    return out, lse, idx

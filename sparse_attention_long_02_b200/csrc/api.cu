@@ -63,6 +63,8 @@ int status_of(cudaError_t e) {
 
 }  // namespace
 
+void set_last_error(const char* msg) { snprintf(g_last_error, sizeof g_last_error, "%s", msg); }
+
 cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
                          uint64_t inner, uint64_t rows, uint64_t row_stride, uint32_t box_inner,
                          uint32_t box_rows, CUtensorMapSwizzle swizzle) {

@@ -65,4 +65,7 @@ cudaError_t launch_sparse_mla(const MlaArgs& a, const void* q, const void* kv, l
 
 int indexer_queries_per_cta(int Hi);
 
+// Records a message for dsa_last_error_string() on this thread.
+void set_last_error(const char* msg);
+
 }  // namespace dsa
