@@ -11,22 +11,25 @@
 //
 // Layout of the work. One query (all H <= 128 heads on the MMA's M) runs on a
 // cluster of two CTAs. A 128-head x 512-dim fp32 output needs all 512 TMEM
-// columns of an SM, so the output is split by value dims: CTA 0 owns latent
-// dims [0,256) and CTA 1 owns [256,512). The logit contraction is split the
-// same way, CTA 0 also taking the 64 rope dims, so each CTA gathers only the
-// dims it uses and every selected byte crosses HBM once. Per tile of 64
-// selected keys:
-//   1. warp 0 gathers the CTA's dims of the 64 rows with TMA gather4 (the
-//      block table is applied here for the paged cache);
-//   2. warp 1 issues S_c = Q_c K_c^T (M=128 heads, N=64 keys) into TMEM;
+// columns of an SM, so the output is split by value dims: CTA c owns latent
+// dims [256c, 256c+256). The logit contraction is split the same way, each
+// CTA also taking half of the 64 rope dims ([512+32c, 512+32c+32)), so both
+// CTAs do the same work, each gathers only the dims it uses, and every
+// selected byte crosses HBM once. Per tile of 64 selected keys:
+//   1. warp 0 stages the tile's indices in shared memory and gathers the
+//      CTA's dims of the 64 rows with TMA gather4 (through the block table
+//      for the paged cache), three tiles ahead;
+//   2. warp 1 issues S_c = Q_c K_c^T (M=128 heads, N=64 keys, K=288) into
+//      one of two TMEM logit buffers;
 //   3. warps 4-7 (one thread per head) read their partial logits, push them
 //      to the peer CTA's shared memory, add the peer's partials (fp32 adds
-//      commute, so both CTAs see identical logits), run the online softmax
-//      in the exp2 domain and write P (bf16) for the tensor core; the
-//      running maximum is re-based only when it grows by more than 8 (log2
-//      units), and only then is the TMEM output rescaled;
-//   4. warp 1 issues O_c += P V_c (M=128, N=256 dims, K=64 keys), reading V
-//      from the same gathered tile (MN-major view).
+//      commute, so both CTAs see identical logits), mask unselected slots,
+//      run the online softmax in the exp2 domain and store P (bf16) into one
+//      of two TMEM P buffers; the running maximum is re-based only when it
+//      grows by more than 8 (log2 units), and only then is the output in
+//      TMEM rescaled;
+//   4. warp 1 issues O_c += P V_c with P read from TMEM (M=128, N=256 dims,
+//      K=64 keys) and V from the same gathered tile (MN-major view).
 // The final output is O / l in bf16 and lse = (m + log2 l) * ln 2.
 #include "common.cuh"
 #include "dsa_internal.h"
@@ -36,39 +39,40 @@ namespace {
 
 constexpr int kMlaThreads = 256;
 constexpr int kTileKeys = 64;
-constexpr int kStages = 2;
-constexpr int kAtomBytesQ = 128 * 128;          // 128 heads x 64 dims bf16
-constexpr int kAtomBytesKV = kTileKeys * 128;   // 64 keys x 64 dims bf16
-constexpr int kMaxAtoms = 5;
-constexpr uint32_t kColO = 0;                   // TMEM columns [0,256): output
-constexpr uint32_t kColS = 256;                 // [256,384): two logit buffers
-constexpr float kRebase = 8.0f;                 // lazy rescale threshold (log2 units)
+constexpr int kStages = 3;
+constexpr int kAtoms = 4;                        // 128-B swizzled atoms of 64 dims
+constexpr int kAtomBytesQ = 128 * 128;           // 128 heads x 64 dims bf16
+constexpr int kRopeBytesQ = 128 * 64;            // 128 heads x 32 dims bf16 (64-B swizzle)
+constexpr int kAtomBytesKV = kTileKeys * 128;    // 64 keys x 64 dims bf16
+constexpr int kRopeBytesKV = kTileKeys * 64;     // 64 keys x 32 dims bf16
+constexpr int kStageTx = kAtoms * kAtomBytesKV + kRopeBytesKV;
+constexpr uint32_t kColO = 0;                    // TMEM columns [0,256): output
+constexpr uint32_t kColS = 256;                  // [256,384): two logit buffers
+constexpr uint32_t kColP = 384;                  // [384,448): two P buffers (bf16 pairs)
+constexpr float kRebase = 8.0f;                  // lazy rescale threshold (log2 units)
 
 struct MlaSmem {
-  uint8_t q[kMaxAtoms][kAtomBytesQ];
-  uint8_t kv[kStages][kMaxAtoms][kAtomBytesKV];
-  uint8_t p[128 * 128];                         // P: 128 heads x 64 keys bf16, SW128
-  float x[128 * 64];                            // peer's partial logits (swizzled rows)
+  uint8_t q[kAtoms][kAtomBytesQ];
+  uint8_t q_rope[kRopeBytesQ];
+  uint8_t kv[kStages][kAtoms][kAtomBytesKV];
+  uint8_t kv_rope[kStages][kRopeBytesKV];
+  float x[128 * 64];                             // peer's partial logits (swizzled rows)
+  int sidx[kStages][kTileKeys];                  // the tile's slots, -1 where skipped
   unsigned long long q_full;
   unsigned long long kv_full[kStages];
   unsigned long long kv_empty[kStages];
   unsigned long long s_full[2];
   unsigned long long s_empty[2];
-  unsigned long long p_full;
-  unsigned long long p_empty;
-  unsigned long long x_full;                    // peer wrote into x
-  unsigned long long x_free;                    // peer finished reading its own x
+  unsigned long long p_full[2];
+  unsigned long long p_empty[2];
+  unsigned long long x_full;                     // peer wrote into x
+  unsigned long long x_free;                     // peer finished reading its own x
   unsigned long long o_done;
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// 64-dim atom a of this CTA -> first dim of the atom in the 576-dim row.
-__device__ __forceinline__ int atom_dim(int rank, int a) {
-  return rank == 0 ? (a < 4 ? 64 * a : 512) : 256 + 64 * a;
-}
-
-// Physical row of selected slot `v` (a logical position), or -1 if skipped.
+// Physical row of slot value `v` (a logical position), or -1 if skipped.
 __device__ __forceinline__ int kv_row(const MlaArgs& A, int v, int seq, int limit) {
   if (v < 0) return -1;
   if (v >= limit) {
@@ -84,8 +88,20 @@ __device__ __forceinline__ int kv_row(const MlaArgs& A, int v, int seq, int limi
   return pb * 64 + (v & 63);
 }
 
+// Slot values of the lane's four rows of tile i (-1 past the end of the row).
+__device__ __forceinline__ int4 load_slots(const int* sel, int k, int i, int lane) {
+  const int j = i * kTileKeys + 4 * lane;
+  if (j + 3 < k) return __ldg(reinterpret_cast<const int4*>(sel + j));
+  int4 v = make_int4(-1, -1, -1, -1);
+  if (j < k) v.x = __ldg(sel + j);
+  if (j + 1 < k) v.y = __ldg(sel + j + 1);
+  if (j + 2 < k) v.z = __ldg(sel + j + 2);
+  return v;
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaThreads, 1)
-sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
+                  const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_kvr,
                   const MlaArgs A) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   MlaSmem& sm = *reinterpret_cast<MlaSmem*>(
@@ -93,7 +109,6 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   unsigned* err = A.err;
   const uint32_t rank = cluster_rank();
   const uint32_t peer = rank ^ 1u;
-  const int nat = rank == 0 ? 5 : 4;
   const int r = blockIdx.x >> 1;                 // query row (one cluster per row)
   const int seq = A.block_table ? r / A.nq : 0;
   // keys a slot may name: the causal prefix of the query (paged) or the cache
@@ -102,21 +117,24 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const int ntiles = (A.k + kTileKeys - 1) / kTileKeys;
   const int* sel = A.idx + static_cast<long long>(r) * A.k;
   const int warp = warp_id(), lane = lane_id();
-  // Both CTAs of the pair take the same early exit, so neither waits alone.
+  const int dim0 = 256 * static_cast<int>(rank);             // first latent dim of this CTA
+  const int rope0 = 512 + 32 * static_cast<int>(rank);       // first rope dim of this CTA
+  // Both CTAs of the pair normally take the same early exit; if they did not,
+  // the working one times out on the peer's barriers and still returns.
   const bool aborted = launch_aborted(err);
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&sm.q_full), 1);
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(smem_u32(&sm.kv_full[i]), 1);
+      mbar_init(smem_u32(&sm.kv_full[i]), 16);   // the 16 gathering lanes
       mbar_init(smem_u32(&sm.kv_empty[i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.s_full[i]), 1);
       mbar_init(smem_u32(&sm.s_empty[i]), 128);
+      mbar_init(smem_u32(&sm.p_full[i]), 128);
+      mbar_init(smem_u32(&sm.p_empty[i]), 1);
     }
-    mbar_init(smem_u32(&sm.p_full), 128);
-    mbar_init(smem_u32(&sm.p_empty), 1);
     mbar_init(smem_u32(&sm.x_full), 128);
     mbar_init(smem_u32(&sm.x_free), 128);
     mbar_init(smem_u32(&sm.o_done), 1);
@@ -136,31 +154,45 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   if (warp == 0 && !aborted) {
     // ------------------------------------------------------- gather warp
     if (lane == 0) {
-      mbar_expect_tx(smem_u32(&sm.q_full), nat * kAtomBytesQ);
-      for (int a = 0; a < nat; ++a)
-        tma_load_2d(smem_u32(sm.q[a]), &tm_q, smem_u32(&sm.q_full), atom_dim(rank, a), r * A.H);
+      const uint32_t qf = smem_u32(&sm.q_full);
+      mbar_expect_tx(qf, kAtoms * kAtomBytesQ + kRopeBytesQ);
+      for (int a = 0; a < kAtoms; ++a)
+        tma_load_2d(smem_u32(sm.q[a]), &tm_q, qf, dim0 + 64 * a, r * A.H);
+      tma_load_2d(smem_u32(sm.q_rope), &tm_qr, qf, rope0, r * A.H);
     }
+    int4 next = lane < 16 ? load_slots(sel, A.k, 0, lane) : make_int4(-1, -1, -1, -1);
     int issued = 0;
     for (int i = 0; i < ntiles; ++i) {
       const int st = i % kStages;
+      const int4 cur = next;
+      if (lane < 16 && i + 1 < ntiles) next = load_slots(sel, A.k, i + 1, lane);   // prefetch
+      int rows[4] = {-1, -1, -1, -1};
+      const int vals[4] = {cur.x, cur.y, cur.z, cur.w};
+      if (lane < 16) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) rows[c] = kv_row(A, vals[c], seq, limit);
+      }
       if (i >= kStages &&
           !warp_wait(smem_u32(&sm.kv_empty[st]), ((i / kStages) + 1) & 1, abort_flag, err))
         break;
-      const uint32_t full = smem_u32(&sm.kv_full[st]);
-      if (lane == 0) mbar_expect_tx(full, nat * kAtomBytesKV);
-      __syncwarp();
       if (lane < 16) {
-        int rows[4];
+        const uint32_t full = smem_u32(&sm.kv_full[st]);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int j = i * kTileKeys + 4 * lane + c;
-          const int v = j < A.k ? sel[j] : -1;
-          const int pr = kv_row(A, v, seq, limit);
-          rows[c] = pr < 0 ? A.kv_rows : pr;     // past the end: TMA fills zeros
-        }
-        for (int a = 0; a < nat; ++a)
-          tma_gather4(smem_u32(sm.kv[st][a]) + lane * 512, &tm_kv, full, atom_dim(rank, a),
-                      rows[0], rows[1], rows[2], rows[3]);
+        for (int c = 0; c < 4; ++c) sm.sidx[st][4 * lane + c] = rows[c] >= 0 ? vals[c] : -1;
+        // each gathering lane arrives once (releasing its slot writes); lane 0 also
+        // announces the stage's byte count
+        if (lane == 0)
+          mbar_expect_tx(full, kStageTx);
+        else
+          mbar_arrive(full);
+        int y[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) y[c] = rows[c] < 0 ? A.kv_rows : rows[c];   // past the end: zeros
+        for (int a = 0; a < kAtoms; ++a)
+          tma_gather4(smem_u32(sm.kv[st][a]) + lane * 512, &tm_kv, full, dim0 + 64 * a, y[0], y[1],
+                      y[2], y[3]);
+        tma_gather4(smem_u32(sm.kv_rope[st]) + lane * 256, &tm_kvr, full, rope0, y[0], y[1], y[2],
+                    y[3]);
       }
       ++issued;
     }
@@ -174,18 +206,17 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16(128, kTileKeys, false);
       const uint32_t id_pv = idesc_bf16(128, 256, true);
-      const uint64_t pdesc = sdesc_sw128(smem_u32(sm.p), 0, 1024);
       bool ok = mbar_wait(smem_u32(&sm.q_full), 0, abort_flag, err);
       auto issue_pv = [&](int i) -> bool {
-        const int st = i % kStages;
-        if (!mbar_wait(smem_u32(&sm.p_full), i & 1, abort_flag, err)) return false;
+        const int st = i % kStages, b = i & 1;
+        if (!mbar_wait(smem_u32(&sm.p_full[b]), (i >> 1) & 1, abort_flag, err)) return false;
         tc_fence_after();
         const uint64_t vdesc = sdesc_sw128(smem_u32(sm.kv[st][0]), kAtomBytesKV, 1024);
 #pragma unroll
-        for (int kk = 0; kk < kTileKeys / 16; ++kk)   // 16 keys = 2 groups of 8 rows
-          mma_bf16(tmem + kColO, pdesc + 2 * kk, vdesc + (kk * 2048 >> 4), id_pv,
-                   (i > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(smem_u32(&sm.p_empty));
+        for (int kk = 0; kk < kTileKeys / 16; ++kk)   // 16 keys: 8 P columns, 2 V row groups
+          mma_bf16_ts(tmem + kColO, tmem + kColP + 32 * b + 8 * kk, vdesc + (kk * 2048 >> 4),
+                      id_pv, (i > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(smem_u32(&sm.p_empty[b]));
         mma_commit(smem_u32(&sm.kv_empty[st]));
         return true;
       };
@@ -196,13 +227,19 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (i >= 2 && !mbar_wait(smem_u32(&sm.s_empty[b]), ((i >> 1) + 1) & 1, abort_flag, err))
           break;
         tc_fence_after();
-        for (int a = 0; a < nat; ++a) {
+        const uint32_t d = tmem + kColS + b * kTileKeys;
+        for (int a = 0; a < kAtoms; ++a) {
           const uint64_t qd = sdesc_sw128(smem_u32(sm.q[a]), 0, 1024);
           const uint64_t kd = sdesc_sw128(smem_u32(sm.kv[st][a]), 0, 1024);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)          // 4 x K=16 dims (32 bytes)
-            mma_bf16(tmem + kColS + b * kTileKeys, qd + 2 * kk, kd + 2 * kk, id_qk,
-                     (a > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16(d, qd + 2 * kk, kd + 2 * kk, id_qk, (a > 0 || kk > 0) ? 1u : 0u);
+        }
+        {
+          const uint64_t qd = sdesc_sw64(smem_u32(sm.q_rope), 512);
+          const uint64_t kd = sdesc_sw64(smem_u32(sm.kv_rope[st]), 512);
+          mma_bf16(d, qd, kd, id_qk, 1u);
+          mma_bf16(d, qd + 2, kd + 2, id_qk, 1u);
         }
         mma_commit(smem_u32(&sm.s_full[b]));
         if (i > 0) {
@@ -225,7 +262,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int i = 0; ok && i < ntiles; ++i) {
-      const int b = i & 1;
+      const int b = i & 1, st = i % kStages;
       float s[64];
       if (!(ok = warp_wait(smem_u32(&sm.s_full[b]), (i >> 1) & 1, abort_flag, err))) break;
       tc_fence_after();
@@ -243,6 +280,16 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         st_cluster_v4(peer_x + pc * 16, s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
       }
       mbar_arrive_remote(peer_x_full);
+      // which slots of the tile are selected (staged by the gather warp)
+      if (!(ok = warp_wait(smem_u32(&sm.kv_full[st]), (i / kStages) & 1, abort_flag, err))) break;
+      unsigned long long valid = 0;
+#pragma unroll
+      for (int c = 0; c < kTileKeys / 4; ++c) {
+        const int4 v = *reinterpret_cast<const int4*>(&sm.sidx[st][4 * c]);
+        valid |= static_cast<unsigned long long>((v.x >= 0) | ((v.y >= 0) << 1) |
+                                                 ((v.z >= 0) << 2) | ((v.w >= 0) << 3))
+                 << (4 * c);
+      }
       if (!(ok = warp_wait<true>(smem_u32(&sm.x_full), i & 1, abort_flag, err))) break;
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
@@ -254,50 +301,45 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         s[4 * c + 3] += v.w;
       }
       mbar_arrive_remote(peer_x_free);
-      // mask unselected slots, scale into the log2 domain
-      float mt = -INFINITY;
-      const int* tsel = sel + i * kTileKeys;
+      // mask unselected slots, scale into the log2 domain, tile maximum
+      float pm[8];
 #pragma unroll
-      for (int c = 0; c < kTileKeys; c += 4) {
-        int4 v4 = make_int4(-1, -1, -1, -1);
-        if (i * kTileKeys + c + 3 < A.k) v4 = __ldg(reinterpret_cast<const int4*>(tsel + c));
-        else {
-          int* pv = reinterpret_cast<int*>(&v4);
-          for (int e = 0; e < 4; ++e)
-            if (i * kTileKeys + c + e < A.k) pv[e] = __ldg(tsel + c + e);
-        }
-        const int vv[4] = {v4.x, v4.y, v4.z, v4.w};
+      for (int e = 0; e < 8; ++e) pm[e] = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const bool valid = vv[e] >= 0 && vv[e] < limit;
-          s[c + e] = valid ? s[c + e] * A.sm_scale_log2 : -INFINITY;
-          mt = fmaxf(mt, s[c + e]);
-        }
+      for (int j = 0; j < kTileKeys; ++j) {
+        s[j] = ((valid >> j) & 1ull) ? s[j] * A.sm_scale_log2 : -INFINITY;
+        pm[j & 7] = fmaxf(pm[j & 7], s[j]);
       }
+      const float mt = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       float alpha = 1.f;
       bool rescale = false;
-      if (mt > m_ref + kRebase) {        // also the first tile with a valid key
-        const float m_new = fmaxf(mt, m_ref);
+      if (mt > m_ref + kRebase) {        // also the first tile with a selected key
         if (m_ref > -INFINITY) {
-          alpha = exp2f(m_ref - m_new);
+          alpha = fast_exp2(m_ref - mt);
           rescale = true;
         }
-        m_ref = m_new;
+        m_ref = mt;
       }
-      float psum = 0.f;
+      float ps[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ps[e] = 0.f;
       uint32_t pk[32];
+      const bool live = m_ref > -INFINITY;
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        const float p0 = m_ref > -INFINITY ? exp2f(s[2 * c] - m_ref) : 0.f;
-        const float p1 = m_ref > -INFINITY ? exp2f(s[2 * c + 1] - m_ref) : 0.f;
-        psum += p0 + p1;
+        const float p0 = live ? fast_exp2(s[2 * c] - m_ref) : 0.f;
+        const float p1 = live ? fast_exp2(s[2 * c + 1] - m_ref) : 0.f;
+        ps[c & 7] += p0 + p1;
         const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
         pk[c] = *reinterpret_cast<const uint32_t*>(&pb);
       }
-      l = l * alpha + psum;
-      // P buffer and the output are free once PV(i-1) has finished
-      if (i > 0 && !(ok = warp_wait(smem_u32(&sm.p_empty), (i - 1) & 1, abort_flag, err))) break;
+      l = l * alpha + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
+      // a new reference maximum: rescale the output once PV(i-1) has finished
       if (rescale && i > 0) {
+        if (!(ok = warp_wait(smem_u32(&sm.p_empty[(i - 1) & 1]), ((i - 1) >> 1) & 1, abort_flag,
+                             err)))
+          break;
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
@@ -308,25 +350,23 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           tmem_st32(tmem + lane_base + kColO + 32 * c, o);
         }
       }
-      // P row h: 64 bf16 = 128 B in the 128-B swizzle (chunk c at c ^ (h % 8))
-      uint8_t* prow = sm.p + (h >> 3) * 1024 + (h & 7) * 128;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int pc = c ^ (h & 7);
-        *reinterpret_cast<uint4*>(prow + pc * 16) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      }
-      fence_proxy_async_smem();
+      // P buffer b is free once PV(i-2) has finished
+      if (i >= 2 &&
+          !(ok = warp_wait(smem_u32(&sm.p_empty[b]), ((i - 2) >> 1) & 1, abort_flag, err)))
+        break;
+      tc_fence_after();
+      tmem_st32(tmem + lane_base + kColP + 32 * b, *reinterpret_cast<const float(*)[32]>(pk));
       tc_fence_before();
-      mbar_arrive(smem_u32(&sm.p_full));
+      mbar_arrive(smem_u32(&sm.p_full[b]));
     }
     // ------------------------------------------------------- epilogue
     if (ok && ntiles > 0 &&
-        warp_wait(smem_u32(&sm.p_empty), (ntiles - 1) & 1, abort_flag, err)) {
+        warp_wait(smem_u32(&sm.p_empty[(ntiles - 1) & 1]), ((ntiles - 1) >> 1) & 1, abort_flag,
+                  err)) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const bool head_ok = h < A.H;
-      __nv_bfloat16* orow = A.out + (static_cast<long long>(r) * A.H + h) * 512 + rank * 256;
+      __nv_bfloat16* orow = A.out + (static_cast<long long>(r) * A.H + h) * 512 + dim0;
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
         float o[32];
@@ -364,22 +404,24 @@ cudaError_t launch_sparse_mla(const MlaArgs& a_in, const void* q, const void* kv
                               long long q_rows, cudaStream_t st) {
   MlaArgs a = a_in;
   a.kv_rows = static_cast<int>(kv_rows);
-  CUtensorMap tq, tkv;
-  cudaError_t e = make_tmap_2d(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 576, q_rows, 576 * 2, 64,
-                               128, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (e != cudaSuccess) return e;
-  e = make_tmap_2d(&tkv, kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 576, kv_rows, 576 * 2, 64, 1,
-                   CU_TENSOR_MAP_SWIZZLE_128B);
+  CUtensorMap tq, tqr, tkv, tkvr;
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  cudaError_t e =
+      make_tmap_2d(&tq, q, bf, 576, q_rows, 576 * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e == cudaSuccess)
+    e = make_tmap_2d(&tqr, q, bf, 576, q_rows, 576 * 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (e == cudaSuccess)
+    e = make_tmap_2d(&tkv, kv, bf, 576, kv_rows, 576 * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e == cudaSuccess)
+    e = make_tmap_2d(&tkvr, kv, bf, 576, kv_rows, 576 * 2, 32, 1, CU_TENSOR_MAP_SWIZZLE_64B);
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(MlaSmem) + 1024;
   e = cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(2 * a.T);      // x has no 65535 limit; cluster pairs are consecutive x
-  sparse_mla_kernel<<<grid, kMlaThreads, smem, st>>>(tq, tkv, a);
+  sparse_mla_kernel<<<grid, kMlaThreads, smem, st>>>(tq, tqr, tkv, tkvr, a);
   return cudaGetLastError();
 }
-
-size_t sparse_mla_smem_bytes() { return sizeof(MlaSmem) + 1024; }
 
 }  // namespace dsa
