@@ -48,6 +48,7 @@ struct MlaArgs {
   const int* seq_len = nullptr;
   __nv_bfloat16* out = nullptr;           // [T][H][512]
   float* lse = nullptr;                   // [T][H] or null
+  const __nv_bfloat16* kv = nullptr;      // [kv_rows][576] (filled by the launcher)
   int kv_rows = 0;                        // rows of the kv tensor map (filled by the launcher)
   unsigned* err = nullptr;
 };

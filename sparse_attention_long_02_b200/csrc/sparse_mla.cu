@@ -16,9 +16,9 @@
 // CTA also taking half of the 64 rope dims ([512+32c, 512+32c+32)), so both
 // CTAs do the same work, each gathers only the dims it uses, and every
 // selected byte crosses HBM once. Per tile of 64 selected keys:
-//   1. warp 0 stages the tile's indices in shared memory and gathers the
-//      CTA's dims of the 64 rows with TMA gather4 (through the block table
-//      for the paged cache), three tiles ahead;
+//   1. six gather warps copy the CTA's dims of the 64 rows with coalesced
+//      cp.async (through the block table for the paged cache), up to three
+//      tiles ahead, and stage the tile's slots in shared memory;
 //   2. warp 1 issues S_c = Q_c K_c^T (M=128 heads, N=64 keys, K=288) into
 //      one of two TMEM logit buffers;
 //   3. warps 4-7 (one thread per head) read their partial logits, push them
@@ -33,11 +33,12 @@
 // The final output is O / l in bf16 and lse = (m + log2 l) * ln 2.
 #include "common.cuh"
 #include "dsa_internal.h"
+#include <cuda_fp16.h>
 
 namespace dsa {
 namespace {
 
-constexpr int kMlaThreads = 256;
+constexpr int kMlaThreads = 384;
 constexpr int kTileKeys = 64;
 constexpr int kStages = 3;
 constexpr int kAtoms = 4;                        // 128-B swizzled atoms of 64 dims
@@ -45,7 +46,7 @@ constexpr int kAtomBytesQ = 128 * 128;           // 128 heads x 64 dims bf16
 constexpr int kRopeBytesQ = 128 * 64;            // 128 heads x 32 dims bf16 (64-B swizzle)
 constexpr int kAtomBytesKV = kTileKeys * 128;    // 64 keys x 64 dims bf16
 constexpr int kRopeBytesKV = kTileKeys * 64;     // 64 keys x 32 dims bf16
-constexpr int kStageTx = kAtoms * kAtomBytesKV + kRopeBytesKV;
+constexpr int kGatherWarps = 6;                 // warps 0, 2, 3, 8, 9, 10
 constexpr uint32_t kColO = 0;                    // TMEM columns [0,256): output
 constexpr uint32_t kColS = 256;                  // [256,384): two logit buffers
 constexpr uint32_t kColP = 384;                  // [384,448): two P buffers (bf16 pairs)
@@ -56,7 +57,7 @@ struct MlaSmem {
   uint8_t q_rope[kRopeBytesQ];
   uint8_t kv[kStages][kAtoms][kAtomBytesKV];
   uint8_t kv_rope[kStages][kRopeBytesKV];
-  float x[128 * 64];                             // peer's partial logits (swizzled rows)
+  uint4 x[128 * 8];                              // peer's partial logits, fp16 (swizzled rows)
   int sidx[kStages][kTileKeys];                  // the tile's slots, -1 where skipped
   unsigned long long q_full;
   unsigned long long kv_full[kStages];
@@ -65,8 +66,9 @@ struct MlaSmem {
   unsigned long long s_empty[2];
   unsigned long long p_full[2];
   unsigned long long p_empty[2];
-  unsigned long long x_full;                     // peer wrote into x
-  unsigned long long x_free;                     // peer finished reading its own x
+  unsigned long long x_full;                     // the peer's partial logits have landed in x
+  unsigned long long x_free;                     // the peer has read what this CTA sent it
+  unsigned long long x_read;                     // the four softmax warps have read x
   unsigned long long o_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -86,17 +88,6 @@ __device__ __forceinline__ int kv_row(const MlaArgs& A, int v, int seq, int limi
     return -1;
   }
   return pb * 64 + (v & 63);
-}
-
-// Slot values of the lane's four rows of tile i (-1 past the end of the row).
-__device__ __forceinline__ int4 load_slots(const int* sel, int k, int i, int lane) {
-  const int j = i * kTileKeys + 4 * lane;
-  if (j + 3 < k) return __ldg(reinterpret_cast<const int4*>(sel + j));
-  int4 v = make_int4(-1, -1, -1, -1);
-  if (j < k) v.x = __ldg(sel + j);
-  if (j + 1 < k) v.y = __ldg(sel + j + 1);
-  if (j + 2 < k) v.z = __ldg(sel + j + 2);
-  return v;
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaThreads, 1)
@@ -126,7 +117,8 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&sm.q_full), 1);
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(smem_u32(&sm.kv_full[i]), 16);   // the 16 gathering lanes
+      // one cp.async-completion arrival per gathering thread + the slot writer
+      mbar_init(smem_u32(&sm.kv_full[i]), 32 * kGatherWarps + 1);
       mbar_init(smem_u32(&sm.kv_empty[i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -135,8 +127,9 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       mbar_init(smem_u32(&sm.p_full[i]), 128);
       mbar_init(smem_u32(&sm.p_empty[i]), 1);
     }
-    mbar_init(smem_u32(&sm.x_full), 128);
-    mbar_init(smem_u32(&sm.x_free), 128);
+    mbar_init(smem_u32(&sm.x_full), 1);          // own expect_tx + the peer's st.async bytes
+    mbar_init(smem_u32(&sm.x_free), 1);          // one release from the peer per tile
+    mbar_init(smem_u32(&sm.x_read), 4);
     mbar_init(smem_u32(&sm.o_done), 1);
     sm.abort_flag = aborted ? 1 : 0;
     fence_barrier_init();
@@ -151,56 +144,63 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
 
-  if (warp == 0 && !aborted) {
-    // ------------------------------------------------------- gather warp
-    if (lane == 0) {
+  const int gw = warp == 0 ? 0 : (warp == 2 || warp == 3) ? warp - 1 : warp - 5;   // 0..5
+  if ((warp == 0 || warp == 2 || warp == 3 || (warp >= 8 && warp <= 10)) && !aborted) {
+    // ------------------------------------------------------- gather warps
+    // Each warp copies whole rows: one cp.async per lane covers the 512-B latent
+    // slice of a row (coalesced), lanes 0-3 add its 64-B rope slice; rows land
+    // in the 128-B (latent) and 64-B (rope) swizzled layouts the MMA reads.
+    if (warp == 0 && lane == 0) {
       const uint32_t qf = smem_u32(&sm.q_full);
       mbar_expect_tx(qf, kAtoms * kAtomBytesQ + kRopeBytesQ);
       for (int a = 0; a < kAtoms; ++a)
         tma_load_2d(smem_u32(sm.q[a]), &tm_q, qf, dim0 + 64 * a, r * A.H);
       tma_load_2d(smem_u32(sm.q_rope), &tm_qr, qf, rope0, r * A.H);
     }
-    int4 next = lane < 16 ? load_slots(sel, A.k, 0, lane) : make_int4(-1, -1, -1, -1);
-    int issued = 0;
+    int v0 = lane < A.k ? __ldg(sel + lane) : -1;
+    int v1 = lane + 32 < A.k ? __ldg(sel + lane + 32) : -1;
     for (int i = 0; i < ntiles; ++i) {
       const int st = i % kStages;
-      const int4 cur = next;
-      if (lane < 16 && i + 1 < ntiles) next = load_slots(sel, A.k, i + 1, lane);   // prefetch
-      int rows[4] = {-1, -1, -1, -1};
-      const int vals[4] = {cur.x, cur.y, cur.z, cur.w};
-      if (lane < 16) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) rows[c] = kv_row(A, vals[c], seq, limit);
+      const int c0 = v0, c1 = v1;
+      const int j0 = (i + 1) * kTileKeys + lane;                    // prefetch the next tile
+      if (i + 1 < ntiles) {
+        v0 = j0 < A.k ? __ldg(sel + j0) : -1;
+        v1 = j0 + 32 < A.k ? __ldg(sel + j0 + 32) : -1;
       }
+      const int r0 = kv_row(A, c0, seq, limit), r1 = kv_row(A, c1, seq, limit);
       if (i >= kStages &&
           !warp_wait(smem_u32(&sm.kv_empty[st]), ((i / kStages) + 1) & 1, abort_flag, err))
         break;
-      if (lane < 16) {
-        const uint32_t full = smem_u32(&sm.kv_full[st]);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) sm.sidx[st][4 * lane + c] = rows[c] >= 0 ? vals[c] : -1;
-        // each gathering lane arrives once (releasing its slot writes); lane 0 also
-        // announces the stage's byte count
-        if (lane == 0)
-          mbar_expect_tx(full, kStageTx);
-        else
-          mbar_arrive(full);
-        int y[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) y[c] = rows[c] < 0 ? A.kv_rows : rows[c];   // past the end: zeros
-        for (int a = 0; a < kAtoms; ++a)
-          tma_gather4(smem_u32(sm.kv[st][a]) + lane * 512, &tm_kv, full, dim0 + 64 * a, y[0], y[1],
-                      y[2], y[3]);
-        tma_gather4(smem_u32(sm.kv_rope[st]) + lane * 256, &tm_kvr, full, rope0, y[0], y[1], y[2],
-                    y[3]);
+      const uint32_t full = smem_u32(&sm.kv_full[st]);
+      if (gw == 0) {
+        sm.sidx[st][lane] = r0 >= 0 ? c0 : -1;
+        sm.sidx[st][32 + lane] = r1 >= 0 ? c1 : -1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(full);
       }
-      ++issued;
+      const uint32_t kv0 = smem_u32(sm.kv[st][lane >> 3]);
+      const uint32_t rope = smem_u32(sm.kv_rope[st]);
+      for (int row = gw; row < kTileKeys; row += kGatherWarps) {
+        const int pr = __shfl_sync(0xffffffffu, row < 32 ? r0 : r1, row & 31);
+        const __nv_bfloat16* src = A.kv + static_cast<long long>(pr < 0 ? 0 : pr) * 576;
+        const uint32_t nb = pr < 0 ? 0u : 16u;               // skipped slot: zero fill
+        cp_async16(kv0 + row * 128 + (((lane & 7) ^ (row & 7)) << 4), src + dim0 + lane * 8, nb);
+        if (lane < 4)
+          cp_async16(rope + row * 64 + ((lane ^ ((row >> 1) & 3)) << 4), src + rope0 + lane * 8, nb);
+      }
+      cp_async_arrive(full);
     }
-    if (lane == 0) {
-      for (int i = max(0, issued - kStages); i < issued; ++i)
-        mbar_drain(smem_u32(&sm.kv_full[i % kStages]), (i / kStages) & 1);
-      mbar_drain(smem_u32(&sm.q_full), 0);
-    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (warp == 0 && lane == 0) mbar_drain(smem_u32(&sm.q_full), 0);
+  } else if (warp == 11 && !aborted) {
+    // ------------------------------------------ release x back to the peer
+    // This warp issues no remote stores, so its cluster-scope release does
+    // not wait behind the softmax warps' outgoing partials.
+    if (lane == 0)
+      for (int i = 0; i < ntiles; ++i) {
+        if (!mbar_wait(smem_u32(&sm.x_read), i & 1, abort_flag, err)) break;
+        mbar_arrive_remote(mapa(smem_u32(&sm.x_free), peer));
+      }
   } else if (warp == 1 && !aborted) {
     // ------------------------------------------------------- MMA thread
     if (lane == 0) {
@@ -226,6 +226,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (!mbar_wait(smem_u32(&sm.kv_full[st]), (i / kStages) & 1, abort_flag, err)) break;
         if (i >= 2 && !mbar_wait(smem_u32(&sm.s_empty[b]), ((i >> 1) + 1) & 1, abort_flag, err))
           break;
+        fence_proxy_async_smem();         // cp.async (generic) writes -> tensor-core reads
         tc_fence_after();
         const uint32_t d = tmem + kColS + b * kTileKeys;
         for (int a = 0; a < kAtoms; ++a) {
@@ -255,10 +256,9 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // ------------------------------------------------- softmax warpgroup
     const int h = 32 * (warp & 3) + lane;               // head = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    const uint32_t peer_x = mapa(smem_u32(sm.x), peer) + h * 256;
+    const uint32_t peer_x = mapa(smem_u32(sm.x), peer) + h * 128;
     const uint32_t peer_x_full = mapa(smem_u32(&sm.x_full), peer);
-    const uint32_t peer_x_free = mapa(smem_u32(&sm.x_free), peer);
-    const float* my_x = sm.x + h * 64;
+    const uint4* my_x = sm.x + h * 8;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int i = 0; ok && i < ntiles; ++i) {
@@ -271,15 +271,28 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 *reinterpret_cast<float(*)[32]>(s + 32));
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.s_empty[b]));
-      // exchange partial logits with the peer CTA
+      // exchange partial logits with the peer CTA: this CTA's x receives the
+      // peer's 128 x 64 partials for tile i as fp16 (16 KB, credited to x_full);
+      // the shared-memory network between SMs is the scarce resource here, and
+      // fp16 keeps 11 bits of each partial (relative error 2^-11, below the
+      // bf16 rounding P gets before the PV product)
+      if (h == 0) mbar_expect_tx(smem_u32(&sm.x_full), 128 * 64 * 2);
       if (i > 0 && !(ok = warp_wait<true>(smem_u32(&sm.x_free), (i - 1) & 1, abort_flag, err)))
         break;
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
+      for (int c = 0; c < 8; ++c) {
         const int pc = c ^ (h & 7);
-        st_cluster_v4(peer_x + pc * 16, s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
+        uint4 v;
+        __half2 h0 = __floats2half2_rn(s[8 * c], s[8 * c + 1]);
+        __half2 h1 = __floats2half2_rn(s[8 * c + 2], s[8 * c + 3]);
+        __half2 h2 = __floats2half2_rn(s[8 * c + 4], s[8 * c + 5]);
+        __half2 h3 = __floats2half2_rn(s[8 * c + 6], s[8 * c + 7]);
+        v.x = *reinterpret_cast<uint32_t*>(&h0);
+        v.y = *reinterpret_cast<uint32_t*>(&h1);
+        v.z = *reinterpret_cast<uint32_t*>(&h2);
+        v.w = *reinterpret_cast<uint32_t*>(&h3);
+        st_async_v4_b32(peer_x + pc * 16, v, peer_x_full);
       }
-      mbar_arrive_remote(peer_x_full);
       // which slots of the tile are selected (staged by the gather warp)
       if (!(ok = warp_wait(smem_u32(&sm.kv_full[st]), (i / kStages) & 1, abort_flag, err))) break;
       unsigned long long valid = 0;
@@ -292,15 +305,20 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       if (!(ok = warp_wait<true>(smem_u32(&sm.x_full), i & 1, abort_flag, err))) break;
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
+      for (int c = 0; c < 8; ++c) {
         const int pc = c ^ (h & 7);
-        const float4 v = *reinterpret_cast<const float4*>(my_x + pc * 4);
-        s[4 * c] += v.x;
-        s[4 * c + 1] += v.y;
-        s[4 * c + 2] += v.z;
-        s[4 * c + 3] += v.w;
+        const uint4 v = my_x[pc];
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[e]));
+          s[8 * c + 2 * e] += f.x;
+          s[8 * c + 2 * e + 1] += f.y;
+        }
       }
-      mbar_arrive_remote(peer_x_free);
+      // warp 11 hands x back to the peer once all four warps have read it
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.x_read));
       // mask unselected slots, scale into the log2 domain, tile maximum
       float pm[8];
 #pragma unroll
@@ -321,21 +339,32 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         m_ref = mt;
       }
+      // P buffer b is free once PV(i-2) has finished
+      if (i >= 2 &&
+          !(ok = warp_wait(smem_u32(&sm.p_empty[b]), ((i - 2) >> 1) & 1, abort_flag, err)))
+        break;
+      tc_fence_after();
       float ps[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) ps[e] = 0.f;
-      uint32_t pk[32];
       const bool live = m_ref > -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = live ? fast_exp2(s[2 * c] - m_ref) : 0.f;
-        const float p1 = live ? fast_exp2(s[2 * c + 1] - m_ref) : 0.f;
-        ps[c & 7] += p0 + p1;
-        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-        pk[c] = *reinterpret_cast<const uint32_t*>(&pb);
+      for (int half = 0; half < 2; ++half) {     // 32 keys -> 16 packed columns at a time
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int j = 32 * half + 2 * c;
+          const float p0 = live ? fast_exp2(s[j] - m_ref) : 0.f;
+          const float p1 = live ? fast_exp2(s[j + 1] - m_ref) : 0.f;
+          ps[c & 7] += p0 + p1;
+          const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+          pk[c] = *reinterpret_cast<const uint32_t*>(&pb);
+        }
+        tmem_st16(tmem + lane_base + kColP + 32 * b + 16 * half, pk);
       }
       l = l * alpha + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
       // a new reference maximum: rescale the output once PV(i-1) has finished
+      // (PV(i) cannot start before this warpgroup arrives on p_full below)
       if (rescale && i > 0) {
         if (!(ok = warp_wait(smem_u32(&sm.p_empty[(i - 1) & 1]), ((i - 1) >> 1) & 1, abort_flag,
                              err)))
@@ -350,12 +379,6 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           tmem_st32(tmem + lane_base + kColO + 32 * c, o);
         }
       }
-      // P buffer b is free once PV(i-2) has finished
-      if (i >= 2 &&
-          !(ok = warp_wait(smem_u32(&sm.p_empty[b]), ((i - 2) >> 1) & 1, abort_flag, err)))
-        break;
-      tc_fence_after();
-      tmem_st32(tmem + lane_base + kColP + 32 * b, *reinterpret_cast<const float(*)[32]>(pk));
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.p_full[b]));
     }
@@ -404,6 +427,7 @@ cudaError_t launch_sparse_mla(const MlaArgs& a_in, const void* q, const void* kv
                               long long q_rows, cudaStream_t st) {
   MlaArgs a = a_in;
   a.kv_rows = static_cast<int>(kv_rows);
+  a.kv = static_cast<const __nv_bfloat16*>(kv);
   CUtensorMap tq, tqr, tkv, tkvr;
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   cudaError_t e =

@@ -80,7 +80,7 @@ def test_noalloc_decode_matches_workspace_decode_twice():
         assert err.max().item() <= 2e-2 and err.mean().item() <= 2e-3
         fin = torch.isfinite(lse_r)
         assert torch.equal(fin, torch.isfinite(lse))
-        assert (lse[fin] - lse_r[fin]).abs().max().item() <= 1e-4
+        assert (lse[fin] - lse_r[fin]).abs().max().item() <= 2e-3
 
 
 def test_noalloc_rejects_requests_beyond_its_scratch():
