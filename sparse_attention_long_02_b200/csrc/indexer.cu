@@ -209,19 +209,30 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         out[s] = (s <= pos) ? acc * ks : -INFINITY;
       };
       if constexpr (HI >= 32) {
-        float acc = 0.f;
+        // 64 columns per TMEM round trip; ReLU, then the weighted head sum in
+        // packed f32x2 FMAs over four independent accumulators
+        float2 acc[4];
 #pragma unroll 1
-        for (int c = 0; c < ncol / 32; ++c) {
-          float v[32];
-          tmem_ld32(taddr + c * 32, v);
-          const float* wp = sm.w + c * 32;
-          float part = 0.f;
+        for (int c = 0; c < ncol / 64; ++c) {
+          float v[64];
+          tmem_ld64(taddr + c * 64, v);
+          const float2* wp = reinterpret_cast<const float2*>(sm.w + c * 64);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) part = fmaf(wp[j], fmaxf(v[j], 0.f), part);
-          acc += part;
-          if (((c + 1) * 32) % HI == 0) {
-            emit((c * 32) / HI, acc);
-            acc = 0.f;
+          for (int sub = 0; sub < 2; ++sub) {
+            const int col0 = c * 64 + sub * 32;
+            if (col0 % HI == 0) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) acc[e] = make_float2(0.f, 0.f);
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float2 x =
+                  make_float2(fmaxf(v[32 * sub + 2 * j], 0.f), fmaxf(v[32 * sub + 2 * j + 1], 0.f));
+              acc[j & 3] = __ffma2_rn(wp[16 * sub + j], x, acc[j & 3]);
+            }
+            if ((col0 + 32) % HI == 0)
+              emit(col0 / HI, ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                                  ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y)));
           }
         }
       } else {
@@ -297,8 +308,8 @@ cudaError_t launch_indexer(const IndexerArgs& a_in, const void* q8, const void* 
   const bool paged = a.block_table != nullptr;
   const int qb = paged ? a.nq : indexer_queries_per_cta(a.Hi);
   int n = qb * a.Hi;
-  n = (n + 31) / 32 * 32;                   // the epilogue reads TMEM 32 columns at a time
-  if (n < 32 || n > 256) return cudaErrorInvalidValue;
+  n = (n + 63) / 64 * 64;                   // the epilogue reads TMEM 64 columns at a time
+  if (n < 64 || n > 256) return cudaErrorInvalidValue;
   a.n_mma = n;
   a.q_box_rows = n;
   a.tmem_cols = 2 * n <= 32 ? 32 : 2 * n <= 64 ? 64 : 2 * n <= 128 ? 128 : 2 * n <= 256 ? 256 : 512;
