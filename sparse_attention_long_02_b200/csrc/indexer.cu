@@ -185,21 +185,26 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int g = (warp - 4) >> 2;                 // epilogue group = TMEM buffer
     const int row = 32 * (warp & 3) + lane;        // accumulator row = key in tile
     const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    // k_scale of this thread's key in tile i, fetched one tile ahead so the
+    // load's latency hides behind the previous tile's epilogue
+    auto key_scale = [&](int i) -> float {
+      const long long s = static_cast<long long>(tile0 + i) * kKeyTile + row;
+      if (!a.k_scale || i >= ntiles || s >= key_limit) return 1.f;
+      if (PAGED) {
+        int pb = a.block_table[static_cast<long long>(seq) * a.max_blocks + (s >> 6)];
+        pb = (pb < 0 || pb >= a.nblk) ? 0 : pb;
+        return __ldg(a.k_scale + static_cast<long long>(pb) * 64 + (s & 63));
+      }
+      return __ldg(a.k_scale + s);
+    };
+    float ks_next = key_scale(g);
     for (int i = g; i < ntiles; i += 2) {
+      const float ks = ks_next;
+      ks_next = key_scale(i + 2);
       if (!warp_wait(smem_u32(&sm.t_full[g]), (i >> 1) & 1, abort_flag, err)) break;
       tc_fence_after();
       const long long s = static_cast<long long>(tile0 + i) * kKeyTile + row;   // logical key
       const bool key_ok = s < key_limit;
-      float ks = 1.f;
-      if (a.k_scale && key_ok) {
-        if (PAGED) {
-          int pb = a.block_table[static_cast<long long>(seq) * a.max_blocks + (s >> 6)];
-          pb = (pb < 0 || pb >= a.nblk) ? 0 : pb;
-          ks = a.k_scale[static_cast<long long>(pb) * 64 + (s & 63)];
-        } else {
-          ks = a.k_scale[s];
-        }
-      }
       const uint32_t taddr = tmem + lane_base + g * ncol;
       auto emit = [&](int qq, float acc) {
         if (qq >= nqb || !key_ok) return;
