@@ -5,12 +5,18 @@
 // it sees at most k of them (page 3, section 2 "风险边界明确"). Ties are
 // broken by the smaller key index, which makes the selected set unique.
 //
-// One CTA per row. Scores map to order-preserving 32-bit keys; a radix
-// select with three histogram passes (11 + 11 + 10 bits, shared-memory
-// histograms) finds the k-th largest key T and how many keys equal to T
-// are still needed. A last pass walks the row in index order with a
-// block-wide scan and writes every index whose key is > T plus the first
-// `need` indices whose key == T. The output is therefore sorted by index.
+// One CTA per row. Scores map to order-preserving 32-bit keys.
+//   pass 1: a 4096-bin histogram of the top 12 key bits locates the bucket
+//           holding the k-th largest key;
+//   pass 2: one ordered sweep of the row (block-wide scans) appends every
+//           index above that bucket to a "sure" list and every member of the
+//           bucket (key, index) to a candidate list, both in index order;
+//   then, in shared memory only, a two-level radix select on the low 20 bits
+//   picks the candidates still needed (ties to the first in index order) and
+//   the two index-sorted lists are merged into the output.
+// Rows whose bucket holds more candidates than the buffer, or calls with
+// k > 4096, take the general path: three histogram passes over the row and
+// an ordered selection pass. Either way the output is sorted by index.
 #include "common.cuh"
 #include "dsa_internal.h"
 
@@ -19,6 +25,18 @@ namespace {
 
 constexpr int kTopkThreads = 512;
 constexpr int kWarps = kTopkThreads / 32;
+constexpr int kBins = 4096;          // 12-bit first-level histogram
+constexpr int kFastMaxK = 4096;      // capacity of the "sure" list
+constexpr int kCandCap = 4096;       // capacity of the bucket's candidate list
+
+struct TopkSmem {
+  unsigned hist[kBins];              // also the chosen-candidate list after pass 2
+  int sure[kFastMaxK];
+  unsigned cand_key[kCandCap];       // low 20 key bits
+  int cand_idx[kCandCap];
+  unsigned warp_tot[kWarps];
+  unsigned s_bucket, s_above;
+};
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t b = __float_as_uint(f);
@@ -33,7 +51,6 @@ __device__ __forceinline__ long long row_length(const TopkArgs& a, int r) {
   return min(static_cast<long long>(a.q_pos0) + r + 1, static_cast<long long>(a.S));
 }
 
-// Inclusive prefix sum over a warp.
 __device__ __forceinline__ unsigned warp_incl_scan(unsigned v) {
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -43,12 +60,235 @@ __device__ __forceinline__ unsigned warp_incl_scan(unsigned v) {
   return v;
 }
 
+// Exclusive prefix sum over the block; `total` gets the block sum. Two syncs.
+__device__ __forceinline__ unsigned block_excl_scan(unsigned v, unsigned* warp_tot,
+                                                    unsigned& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned incl = warp_incl_scan(v);
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  unsigned base = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const unsigned t = warp_tot[w];
+    base += (w < warp) ? t : 0u;
+    tot += t;
+  }
+  __syncthreads();
+  total = tot;
+  return base + incl - v;
+}
+
+// With hist[0..nb) filled, find (from the top) the bucket where the count
+// reaches `want`; writes the bucket and the count strictly above it.
+__device__ __forceinline__ void find_bucket(const unsigned* hist, int nb, unsigned want,
+                                            unsigned* s_bucket, unsigned* s_above) {
+  if ((threadIdx.x >> 5) == 0) {
+    const int lane = threadIdx.x & 31;
+    const int per = nb / 32;
+    const int top = nb - 1 - lane * per;
+    unsigned local = 0;
+    for (int j = 0; j < per; ++j) local += hist[top - j];
+    const unsigned incl = warp_incl_scan(local);
+    const unsigned excl = incl - local;
+    const unsigned hit = __ballot_sync(0xffffffffu, incl >= want);
+    const int first = __ffs(hit) - 1;
+    if (lane == first) {
+      unsigned cum = excl;
+      for (int j = 0; j < per; ++j) {
+        const unsigned c = hist[top - j];
+        if (cum + c >= want) {
+          *s_bucket = top - j;
+          *s_above = cum;
+          break;
+        }
+        cum += c;
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// Writes the row's selection in index order: every key whose order key is
+// above `thr`, plus the first `need` keys equal to `thr`.
+__device__ void write_selection(const float4* x4, long long n, long long n4, uint32_t thr,
+                                unsigned need, int* out, int k, TopkSmem& sm) {
+  const int tid = threadIdx.x;
+  unsigned base_gt = 0, base_eq = 0;
+  for (long long i0 = 0; i0 < n4; i0 += kTopkThreads) {
+    const long long i = i0 + tid;
+    unsigned gt_m = 0, eq_m = 0;
+    if (i < n4) {
+      const float4 v = x4[i];
+      const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (4 * i + c < n) {
+          const uint32_t u = order_key(e[c]);
+          gt_m |= static_cast<unsigned>(u > thr) << c;
+          eq_m |= static_cast<unsigned>(u == thr) << c;
+        }
+    }
+    unsigned tot;
+    const unsigned ex = block_excl_scan(__popc(gt_m) | (__popc(eq_m) << 16), sm.warp_tot, tot);
+    unsigned gt_before = base_gt + (ex & 0xffffu), eq_before = base_eq + (ex >> 16);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (gt_m & (1u << c)) {
+        const unsigned p = gt_before + min(eq_before, need);
+        if (p < static_cast<unsigned>(k)) out[p] = static_cast<int>(4 * i + c);
+        ++gt_before;
+      } else if (eq_m & (1u << c)) {
+        if (eq_before < need) {
+          const unsigned p = gt_before + eq_before;
+          if (p < static_cast<unsigned>(k)) out[p] = static_cast<int>(4 * i + c);
+        }
+        ++eq_before;
+      }
+    }
+    base_gt += tot & 0xffffu;
+    base_eq += tot >> 16;
+  }
+}
+
+// General path: 11 + 11 + 10-bit radix select over the row, then the ordered
+// selection pass.
+__device__ void select_general(const float4* x4, long long n, long long n4, int k, int* out,
+                               TopkSmem& sm) {
+  const int tid = threadIdx.x;
+  uint32_t prefix = 0;
+  unsigned want = static_cast<unsigned>(k);
+  const int bits[3] = {11, 11, 10};
+  int shift = 32;
+  for (int p = 0; p < 3; ++p) {
+    const int nb = 1 << bits[p];
+    shift -= bits[p];
+    const int hi_shift = shift + bits[p];
+    for (int i = tid; i < nb; i += kTopkThreads) sm.hist[i] = 0;
+    __syncthreads();
+    for (long long i = tid; i < n4; i += kTopkThreads) {
+      const float4 v = x4[i];
+      const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (4 * i + c >= n) break;
+        const uint32_t u = order_key(e[c]);
+        if (p == 0 || (u >> hi_shift) == prefix) atomicAdd(&sm.hist[(u >> shift) & (nb - 1)], 1u);
+      }
+    }
+    __syncthreads();
+    find_bucket(sm.hist, nb, want, &sm.s_bucket, &sm.s_above);
+    prefix = (prefix << bits[p]) | sm.s_bucket;
+    want -= sm.s_above;
+    __syncthreads();
+  }
+  write_selection(x4, n, n4, prefix, want, out, k, sm);
+}
+
+// Number of entries of the ascending array a[0..m) that are below v.
+__device__ __forceinline__ int count_below(const int* a, int m, int v) {
+  int lo = 0, hi = m;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (a[mid] < v) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+// Fast path: the bucket `b` of the top 12 bits holds the k-th key; `above`
+// keys lie in higher buckets.
+__device__ void select_fast(const float4* x4, long long n, long long n4, int k, int* out,
+                            TopkSmem& sm, unsigned b, unsigned above) {
+  const int tid = threadIdx.x;
+  const unsigned want = static_cast<unsigned>(k) - above;   // still needed from the bucket
+  // pass 2: ordered sweep collecting the sure keys and the bucket's members
+  unsigned base_sure = 0, base_cand = 0;
+  for (long long i0 = 0; i0 < n4; i0 += kTopkThreads) {
+    const long long i = i0 + tid;
+    unsigned sure_m = 0, cand_m = 0;
+    uint32_t keys[4] = {0, 0, 0, 0};
+    if (i < n4) {
+      const float4 v = x4[i];
+      const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (4 * i + c < n) {
+          const uint32_t u = order_key(e[c]);
+          keys[c] = u;
+          sure_m |= static_cast<unsigned>((u >> 20) > b) << c;
+          cand_m |= static_cast<unsigned>((u >> 20) == b) << c;
+        }
+    }
+    unsigned tot;
+    const unsigned ex = block_excl_scan(__popc(sure_m) | (__popc(cand_m) << 16), sm.warp_tot, tot);
+    unsigned ps = base_sure + (ex & 0xffffu), pc = base_cand + (ex >> 16);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (sure_m & (1u << c)) sm.sure[ps++] = static_cast<int>(4 * i + c);
+      if (cand_m & (1u << c)) {
+        sm.cand_key[pc] = keys[c] & 0xfffffu;
+        sm.cand_idx[pc] = static_cast<int>(4 * i + c);
+        ++pc;
+      }
+    }
+    base_sure += tot & 0xffffu;
+    base_cand += tot >> 16;
+  }
+  __syncthreads();
+  const int ncand = static_cast<int>(base_cand);
+  // radix select on the low 20 bits, inside shared memory (10 + 10 bits)
+  for (int j = tid; j < 1024; j += kTopkThreads) sm.hist[j] = 0;
+  __syncthreads();
+  for (int j = tid; j < ncand; j += kTopkThreads) atomicAdd(&sm.hist[sm.cand_key[j] >> 10], 1u);
+  __syncthreads();
+  find_bucket(sm.hist, 1024, want, &sm.s_bucket, &sm.s_above);
+  const unsigned bA = sm.s_bucket;
+  const unsigned want2 = want - sm.s_above;
+  __syncthreads();
+  for (int j = tid; j < 1024; j += kTopkThreads) sm.hist[j] = 0;
+  __syncthreads();
+  for (int j = tid; j < ncand; j += kTopkThreads)
+    if ((sm.cand_key[j] >> 10) == bA) atomicAdd(&sm.hist[sm.cand_key[j] & 1023u], 1u);
+  __syncthreads();
+  find_bucket(sm.hist, 1024, want2, &sm.s_bucket, &sm.s_above);
+  const uint32_t thr = (bA << 10) | sm.s_bucket;
+  const unsigned need = want2 - sm.s_above;
+  __syncthreads();
+  // chosen candidates, compacted in index order into list2 (reusing hist)
+  int* list2 = reinterpret_cast<int*>(sm.hist);
+  unsigned base_gt = 0, base_eq = 0;
+  for (int j0 = 0; j0 < ncand; j0 += kTopkThreads) {
+    const int j = j0 + tid;
+    const bool in = j < ncand;
+    const uint32_t key = in ? sm.cand_key[j] : 0u;
+    const bool gt = in && key > thr, eq = in && key == thr;
+    unsigned tot;
+    const unsigned ex = block_excl_scan(static_cast<unsigned>(gt) | (static_cast<unsigned>(eq) << 16),
+                                        sm.warp_tot, tot);
+    const unsigned gt_before = base_gt + (ex & 0xffffu), eq_before = base_eq + (ex >> 16);
+    if (gt) list2[gt_before + min(eq_before, need)] = sm.cand_idx[j];
+    else if (eq && eq_before < need) list2[gt_before + eq_before] = sm.cand_idx[j];
+    base_gt += tot & 0xffffu;
+    base_eq += tot >> 16;
+  }
+  __syncthreads();
+  // merge the two index-sorted lists (disjoint) into the output
+  const int na = static_cast<int>(above), nb2 = static_cast<int>(want);
+  for (int i = tid; i < na; i += kTopkThreads) {
+    const int v = sm.sure[i];
+    out[i + count_below(list2, nb2, v)] = v;
+  }
+  for (int j = tid; j < nb2; j += kTopkThreads) {
+    const int v = list2[j];
+    out[j + count_below(sm.sure, na, v)] = v;
+  }
+}
+
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkArgs a) {
-  __shared__ unsigned hist[2048];
-  __shared__ unsigned warp_tot[kWarps];
-  __shared__ unsigned s_bucket, s_above;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
   const int r = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   int* out = a.idx + static_cast<long long>(r) * a.k;
   long long n = row_length(a, r);
   if (n < 0) n = 0;
@@ -60,132 +300,38 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkArgs a) {
     for (int j = tid; j < a.k; j += kTopkThreads) out[j] = j < n ? j : -1;
     return;
   }
-  const float* x = a.scores + static_cast<long long>(r) * a.ld;
-  const float4* x4 = reinterpret_cast<const float4*>(x);
+  const float4* x4 = reinterpret_cast<const float4*>(a.scores + static_cast<long long>(r) * a.ld);
   const long long n4 = (n + 3) >> 2;
-
-  // ----------------------------------------------------- radix select
-  uint32_t prefix = 0;                  // key bits fixed so far
-  unsigned want = static_cast<unsigned>(a.k);   // rank still to find within the prefix
-  const int bits[3] = {11, 11, 10};
-  int shift = 32;
-  for (int p = 0; p < 3; ++p) {
-    const int nb = 1 << bits[p];
-    shift -= bits[p];
-    for (int i = tid; i < nb; i += kTopkThreads) hist[i] = 0;
-    __syncthreads();
-    const int hi_shift = shift + bits[p];
-    for (long long i = tid; i < n4; i += kTopkThreads) {
-      const float4 v = x4[i];
-      const float e[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if (4 * i + c >= n) break;
-        const uint32_t u = order_key(e[c]);
-        if (p == 0 || (u >> hi_shift) == prefix)
-          atomicAdd(&hist[(u >> shift) & (nb - 1)], 1u);
-      }
-    }
-    __syncthreads();
-    if (warp == 0) {
-      // lane l owns bins [top - per*l - per + 1, top - per*l], scanned from the top
-      const int per = nb / 32;
-      const int top = nb - 1 - lane * per;
-      unsigned local = 0;
-      for (int j = 0; j < per; ++j) local += hist[top - j];
-      const unsigned incl = warp_incl_scan(local);
-      const unsigned excl = incl - local;
-      const unsigned hit = __ballot_sync(0xffffffffu, incl >= want);
-      const int first = __ffs(hit) - 1;
-      if (lane == first) {
-        unsigned cum = excl;
-        for (int j = 0; j < per; ++j) {
-          const unsigned c = hist[top - j];
-          if (cum + c >= want) {
-            s_bucket = top - j;
-            s_above = cum;
-            break;
-          }
-          cum += c;
-        }
-      }
-    }
-    __syncthreads();
-    prefix = (prefix << bits[p]) | s_bucket;
-    want -= s_above;
-    __syncthreads();
-  }
-  const uint32_t thr = prefix;          // k-th largest key
-  const unsigned need = want;           // keys == thr to take, smallest indices first
-
-  // ------------------------------------------- ordered final selection
-  unsigned base_sel = 0, base_eq = 0;
-  for (long long i0 = 0; i0 < n4; i0 += kTopkThreads) {
-    const long long i = i0 + tid;
-    unsigned gt_mask = 0, eq_mask = 0;
-    if (i < n4) {
-      const float4 v = x4[i];
-      const float e[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if (4 * i + c < n) {
-          const uint32_t u = order_key(e[c]);
-          gt_mask |= (u > thr) << c;
-          eq_mask |= (u == thr) << c;
-        }
-      }
-    }
-    // exclusive scan of (eq count) to rank equal keys in index order
-    const unsigned n_eq = __popc(eq_mask);
-    unsigned incl = warp_incl_scan(n_eq);
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    unsigned wbase = 0, total = 0;
-    for (int w = 0; w < kWarps; ++w) {
-      const unsigned t = warp_tot[w];
-      if (w < warp) wbase += t;
-      total += t;
-    }
-    unsigned eq_rank = base_eq + wbase + incl - n_eq;
-    unsigned sel_mask = gt_mask;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      if (eq_mask & (1u << c)) {
-        if (eq_rank < need) sel_mask |= 1u << c;
-        ++eq_rank;
-      }
-    }
-    base_eq += total;
-    __syncthreads();
-    const unsigned n_sel = __popc(sel_mask);
-    incl = warp_incl_scan(n_sel);
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    wbase = 0;
-    total = 0;
-    for (int w = 0; w < kWarps; ++w) {
-      const unsigned t = warp_tot[w];
-      if (w < warp) wbase += t;
-      total += t;
-    }
-    unsigned pos = base_sel + wbase + incl - n_sel;
+  // pass 1: 12-bit histogram of the whole row
+  for (int i = tid; i < kBins; i += kTopkThreads) sm.hist[i] = 0;
+  __syncthreads();
+#pragma unroll 2
+  for (long long i = tid; i < n4; i += kTopkThreads) {
+    const float4 v = x4[i];
+    const float e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int c = 0; c < 4; ++c)
-      if (sel_mask & (1u << c)) {
-        if (pos < static_cast<unsigned>(a.k)) out[pos] = static_cast<int>(4 * i + c);
-        ++pos;
-      }
-    base_sel += total;
-    __syncthreads();
+      if (4 * i + c < n) atomicAdd(&sm.hist[order_key(e[c]) >> 20], 1u);
   }
-  if (tid == 0 && base_sel != static_cast<unsigned>(a.k)) raise_error(a.err, kErrBounds);
+  __syncthreads();
+  find_bucket(sm.hist, kBins, static_cast<unsigned>(a.k), &sm.s_bucket, &sm.s_above);
+  const unsigned b = sm.s_bucket, above = sm.s_above, in_bucket = sm.hist[b];
+  __syncthreads();
+  if (a.k <= kFastMaxK && in_bucket <= static_cast<unsigned>(kCandCap))
+    select_fast(x4, n, n4, a.k, out, sm, b, above);
+  else
+    select_general(x4, n, n4, a.k, out, sm);
 }
 
 }  // namespace
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
   if (a.rows <= 0) return cudaSuccess;
-  topk_kernel<<<a.rows, kTopkThreads, 0, st>>>(a);
+  const size_t smem = sizeof(TopkSmem);
+  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  topk_kernel<<<a.rows, kTopkThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -262,3 +262,26 @@ def test_decode_paged_vs_oracle(dsa, lens, nq):
             if all(set(gidx[b, j]) == set(ref["idx"][b, j]) for j in range(nq))]
     assert same
     assert_mla_close(out[same], ref["out"][same], lse[same], ref["lse"][same])
+
+
+@pytest.mark.parametrize("kind,n,k", [("random", 20000, 2048), ("ties", 20000, 2048),
+                                      ("constant", 9000, 1024), ("random", 12000, 5000),
+                                      ("ties", 3000, 256)])
+def test_topk_fast_and_general_paths(dsa, kind, n, k):
+    """Random rows take the in-shared-memory path; rows whose k-th bucket is
+    crowded (heavy ties, constant rows) and k > 4096 take the general path."""
+    rng = np.random.default_rng(n + k)
+    R = 6
+    if kind == "random":
+        I = rng.normal(size=(R, n)).astype(np.float32)
+    elif kind == "ties":
+        I = (rng.integers(-3, 4, size=(R, n)) / 8.0).astype(np.float32)
+    else:
+        I = np.full((R, n), 0.5, np.float32)
+    q_pos0 = n - R                       # rows see n-R+1 .. n keys
+    idx = dsa.topk(torch.from_numpy(I).cuda(), n, k, q_pos0=q_pos0)
+    no_device_error(dsa)
+    ref = oracle.topk(I, oracle.prefill_row_len(R, n, q_pos0), k)
+    exp = np.sort(np.where(ref < 0, np.iinfo(np.int32).max, ref), axis=1)
+    exp = np.where(exp == np.iinfo(np.int32).max, -1, exp)
+    assert np.array_equal(idx.cpu().numpy(), exp)
