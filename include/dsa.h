@@ -144,7 +144,12 @@ int dsa_sparse_mla_fwd(const void *q, const void *kv, const int32_t *idx,
  * Whole prefill path: indexer -> top-k -> sparse MLA for T query rows at
  * positions q_pos0 .. q_pos0 + T - 1 against S cached keys (S >= q_pos0 + T
  * for a self-contained prefill). Query rows are scored in chunks of `chunk`
- * rows (0 = all rows at once); the workspace holds one chunk's scores.
+ * rows (0 = all rows at once); the workspace holds the scores of two chunks
+ * (one when there is a single chunk), so that the top-k of one chunk runs on
+ * a library-owned side stream beside the indexer of the next. The side stream
+ * and its events are created on the first multi-chunk call on a device (no
+ * device memory is allocated) and joined back into `stream` before the
+ * attention launch; concurrent calls on one device enqueue one at a time.
  *
  *   idx_out [T][k] int32 out (the selection), or NULL to keep it in the
  *           workspace only

@@ -92,6 +92,37 @@ bool valid_hi(int Hi) {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Per-device stream and events that let the top-k of one prefill chunk run
+// beside the indexer of the next (created once, no device memory). Calls on
+// one device enqueue under a lock so the events are recorded and waited on in
+// order.
+struct Overlap {
+  cudaStream_t side = nullptr;
+  cudaEvent_t start = nullptr;
+  cudaEvent_t idx_done[2] = {nullptr, nullptr};
+  cudaEvent_t topk_done[2] = {nullptr, nullptr};
+  bool ready = false;
+};
+constexpr int kMaxDev = 64;
+Overlap g_overlap[kMaxDev];
+std::mutex g_overlap_mu;
+
+Overlap* overlap_for_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  Overlap& o = g_overlap[dev];
+  if (!o.ready) {
+    bool ok = cudaStreamCreateWithFlags(&o.side, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&o.start, cudaEventDisableTiming) == cudaSuccess;
+    for (int b = 0; ok && b < 2; ++b)
+      ok = cudaEventCreateWithFlags(&o.idx_done[b], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&o.topk_done[b], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) return nullptr;
+    o.ready = true;
+  }
+  return &o;
+}
+
 int run_indexer(const void* q8, const float* q_scale, const void* k8, const float* k_scale,
                 const float* w, int T, int S, int Hi, int q_pos0, float scale, float* scores,
                 int64_t ld, cudaStream_t st) {
@@ -237,7 +268,8 @@ size_t dsa_forward_workspace_size(int T, int S, int Hi, int H, int k, int chunk)
   if (T <= 0 || S <= 0 || k <= 0) return 0;
   const size_t rows = chunk <= 0 ? T : std::min(chunk, T);
   const size_t ld = round_up(static_cast<size_t>(S), 4);
-  return round_up(rows * ld * sizeof(float), 256) +
+  const size_t nbuf = rows < static_cast<size_t>(T) ? 2 : 1;   // double-buffered chunks
+  return nbuf * round_up(rows * ld * sizeof(float), 256) +
          round_up(static_cast<size_t>(T) * k * sizeof(int32_t), 256);
 }
 
@@ -258,23 +290,58 @@ int dsa_forward(const void* q8, const float* q_scale, const void* k8, const floa
     return DSA_ERR_WORKSPACE;
   const int rows = chunk <= 0 ? T : std::min(chunk, T);
   const int64_t ld = static_cast<int64_t>(round_up(static_cast<size_t>(S), 4));
-  float* scores = static_cast<float*>(workspace);
+  const size_t chunk_bytes = round_up(static_cast<size_t>(rows) * ld * 4, 256);
+  const int nbuf = rows < T ? 2 : 1;
+  float* scores[2] = {static_cast<float*>(workspace),
+                      reinterpret_cast<float*>(static_cast<char*>(workspace) + chunk_bytes)};
   int32_t* idx = idx_out;
-  if (!idx)
-    idx = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) +
-                                     round_up(static_cast<size_t>(rows) * ld * 4, 256));
+  if (!idx) idx = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + nbuf * chunk_bytes);
   if (!aligned16(idx)) return DSA_ERR_INVALID_ARG;
   const uint8_t* q8b = static_cast<const uint8_t*>(q8);
-  for (int c0 = 0; c0 < T; c0 += rows) {
+  auto indexer_chunk = [&](int c0, float* sc) {
     const int n = std::min(rows, T - c0);
-    int s = dsa_indexer_scores(q8b + static_cast<size_t>(c0) * Hi * 128,
-                               q_scale ? q_scale + c0 : nullptr, k8, k_scale,
-                               w + static_cast<size_t>(c0) * Hi, n, S, Hi, q_pos0 + c0, scale,
-                               scores, ld, stream);
-    if (s != DSA_OK) return s;
-    s = dsa_topk(scores, n, S, ld, q_pos0 + c0, k, idx + static_cast<size_t>(c0) * k, stream);
-    if (s != DSA_OK) return s;
+    return dsa_indexer_scores(q8b + static_cast<size_t>(c0) * Hi * 128,
+                              q_scale ? q_scale + c0 : nullptr, k8, k_scale,
+                              w + static_cast<size_t>(c0) * Hi, n, S, Hi, q_pos0 + c0, scale, sc,
+                              ld, stream);
+  };
+  auto topk_chunk = [&](int c0, float* sc, cudaStream_t on) {
+    const int n = std::min(rows, T - c0);
+    return dsa_topk(sc, n, S, ld, q_pos0 + c0, k, idx + static_cast<size_t>(c0) * k, on);
+  };
+  std::unique_lock<std::mutex> lock(g_overlap_mu);
+  Overlap* ov = nbuf == 2 ? overlap_for_current_device() : nullptr;
+  if (!ov) {                               // one chunk (or no side stream): in order
+    lock.unlock();
+    for (int c0 = 0; c0 < T; c0 += rows) {
+      int s = indexer_chunk(c0, scores[0]);
+      if (s != DSA_OK) return s;
+      s = topk_chunk(c0, scores[0], st);
+      if (s != DSA_OK) return s;
+    }
+    return dsa_sparse_mla_fwd(q, kv, idx, T, S, H, k, sm_scale, out, lse, st);
   }
+  // top-k of chunk c (side stream) runs beside the indexer of chunk c+1
+  cudaError_t e = cudaEventRecord(ov->start, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(ov->side, ov->start, 0);
+  if (e != cudaSuccess) return status_of(e);
+  int c = 0;
+  for (int c0 = 0; c0 < T; c0 += rows, ++c) {
+    const int b = c & 1;
+    if (c >= 2 && (e = cudaStreamWaitEvent(st, ov->topk_done[b], 0)) != cudaSuccess)
+      return status_of(e);
+    int s = indexer_chunk(c0, scores[b]);
+    if (s != DSA_OK) return s;
+    if ((e = cudaEventRecord(ov->idx_done[b], st)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(ov->side, ov->idx_done[b], 0)) != cudaSuccess)
+      return status_of(e);
+    s = topk_chunk(c0, scores[b], ov->side);
+    if (s != DSA_OK) return s;
+    if ((e = cudaEventRecord(ov->topk_done[b], ov->side)) != cudaSuccess) return status_of(e);
+  }
+  for (int b = 0; b < std::min(c, 2); ++b)
+    if ((e = cudaStreamWaitEvent(st, ov->topk_done[b], 0)) != cudaSuccess) return status_of(e);
+  lock.unlock();
   return dsa_sparse_mla_fwd(q, kv, idx, T, S, H, k, sm_scale, out, lse, st);
 }
 

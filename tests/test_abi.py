@@ -72,9 +72,10 @@ def test_workspace_sizes(dsa):
     L = dsa.lib()
     # one chunk of fp32 scores (pitch rounded to 4) + the index rows, each 256-B rounded
     assert L.dsa_forward_workspace_size(1024, 1024, 4, 8, 256, 0) == 1024 * 1024 * 4 + 1024 * 256 * 4
+    # several chunks: two score chunks (the top-k of one overlaps the next indexer)
     assert L.dsa_forward_workspace_size(131072, 131072, 64, 128, 2048, 4096) == \
-        4096 * 131072 * 4 + 131072 * 2048 * 4
-    assert L.dsa_forward_workspace_size(10, 7, 4, 8, 4, 3) == 256 + 256
+        2 * 4096 * 131072 * 4 + 131072 * 2048 * 4
+    assert L.dsa_forward_workspace_size(10, 7, 4, 8, 4, 3) == 2 * 256 + 256
     assert L.dsa_decode_paged_workspace_size(64, 1, 512, 64, 128, 2048) == \
         64 * 512 * 64 * 4 + 64 * 2048 * 4
     assert L.dsa_forward_workspace_size(0, 8, 4, 8, 4, 0) == 0
