@@ -1,9 +1,9 @@
 // common.cuh -- sm_100a building blocks shared by the DSA kernels.
 //
-// Inline-PTX wrappers for mbarriers (every wait is bounded), TMA tile and
-// gather4 loads, the tcgen05 tensor-core path (TMEM allocation, MMA issue,
-// commit, TMEM loads/stores) and the shared-memory matrix descriptors the
-// MMA reads its operands through.
+// Inline-PTX wrappers for mbarriers (every wait is bounded), TMA tile loads,
+// cp.async, bulk copies between the CTAs of a cluster, the tcgen05
+// tensor-core path (TMEM allocation, MMA issue, commit, TMEM loads/stores)
+// and the shared-memory matrix descriptors the MMA reads its operands through.
 #pragma once
 
 #include <cuda.h>
@@ -146,22 +146,6 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
 }
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
-
-// 16 bytes into another CTA's shared memory; the bytes are credited to that
-// CTA's mbarrier (complete_tx) when they land, so no fence is needed.
-__device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, float c, float d,
-                                            uint32_t remote_bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::
-          "r"(addr),
-      "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
-      : "memory");
-}
 
 // 16 bytes global -> shared through L2 (bypassing L1); src_bytes = 0 fills zeros.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
@@ -183,21 +167,6 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t
       "r"(src), "r"(bytes), "r"(remote_bar)
       : "memory");
 }
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-// Wait until the sources of all committed bulk copies have been read.
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
-__device__ __forceinline__ void st_async_v4_b32(uint32_t addr, uint4 v, uint32_t remote_bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::
-          "r"(addr),
-      "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(remote_bar)
-      : "memory");
-}
 
 // ------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
@@ -206,24 +175,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(map), "r"(bar), "r"(x), "r"(y)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int x, int y, int z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(map), "r"(bar), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-// Four rows (y0..y3) of a 2D tensor, columns [x, x + box width), landing as
-// four consecutive rows of the destination (box height 1 in the map).
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int x, int y0, int y1, int y2, int y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-      "l"(map), "r"(bar), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
       : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {

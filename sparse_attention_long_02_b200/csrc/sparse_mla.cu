@@ -18,16 +18,19 @@
 // selected byte crosses HBM once. Per tile of 64 selected keys:
 //   1. six gather warps copy the CTA's dims of the 64 rows with coalesced
 //      cp.async (through the block table for the paged cache), up to three
-//      tiles ahead, and stage the tile's slots in shared memory;
+//      tiles ahead;
 //   2. warp 1 issues S_c = Q_c K_c^T (M=128 heads, N=64 keys, K=288) into
 //      one of two TMEM logit buffers;
-//   3. warps 4-7 (one thread per head) read their partial logits, push them
-//      to the peer CTA's shared memory, add the peer's partials (fp32 adds
-//      commute, so both CTAs see identical logits), mask unselected slots,
-//      run the online softmax in the exp2 domain and store P (bf16) into one
-//      of two TMEM P buffers; the running maximum is re-based only when it
-//      grows by more than 8 (log2 units), and only then is the output in
-//      TMEM rescaled;
+//   3. eight softmax warps, two per TMEM lane quarter (thread = head, each
+//      warp of a pair taking 32 of the 64 keys), scale their partial logits
+//      into the log2 domain and stage them as fp16 in shared memory; the
+//      exchange warp sends the whole 16 KB tile to the peer CTA with one bulk
+//      copy (the TMA engine, off the load/store path the gather uses). The
+//      softmax warps add the peer's partials, mask unselected slots, agree on
+//      the tile maximum through shared memory, run the online softmax in the
+//      exp2 domain and store P (bf16) into one of two TMEM P buffers; the
+//      running maximum is re-based only when it grows by more than 8 (log2
+//      units), and only then is the output in TMEM rescaled;
 //   4. warp 1 issues O_c += P V_c with P read from TMEM (M=128, N=256 dims,
 //      K=64 keys) and V from the same gathered tile (MN-major view).
 // The final output is O / l in bf16 and lse = (m + log2 l) * ln 2.
@@ -38,7 +41,7 @@
 namespace dsa {
 namespace {
 
-constexpr int kMlaThreads = 384;
+constexpr int kMlaThreads = 512;
 constexpr int kTileKeys = 64;
 constexpr int kStages = 3;
 constexpr int kAtoms = 4;                        // 128-B swizzled atoms of 64 dims
@@ -46,19 +49,26 @@ constexpr int kAtomBytesQ = 128 * 128;           // 128 heads x 64 dims bf16
 constexpr int kRopeBytesQ = 128 * 64;            // 128 heads x 32 dims bf16 (64-B swizzle)
 constexpr int kAtomBytesKV = kTileKeys * 128;    // 64 keys x 64 dims bf16
 constexpr int kRopeBytesKV = kTileKeys * 64;     // 64 keys x 32 dims bf16
-constexpr int kGatherWarps = 6;                 // warps 0, 2, 3, 8, 9, 10
+constexpr int kGatherWarps = 6;                  // warps 0, 2, 3, 12, 13, 14
+constexpr int kSoftmaxWarps = 8;                 // warps 4-11
+constexpr int kExchangeWarp = 15;
+constexpr uint32_t kXBytes = 128 * kTileKeys * 2;   // one tile of fp16 partial logits
 constexpr uint32_t kColO = 0;                    // TMEM columns [0,256): output
 constexpr uint32_t kColS = 256;                  // [256,384): two logit buffers
 constexpr uint32_t kColP = 384;                  // [384,448): two P buffers (bf16 pairs)
 constexpr float kRebase = 8.0f;                  // lazy rescale threshold (log2 units)
 
+// Rows of 64 fp16 partials (128 B, one per head); the 16-B chunk c of row h
+// sits at chunk c ^ (h & 7), so eight consecutive heads hit distinct banks.
 struct MlaSmem {
   uint8_t q[kAtoms][kAtomBytesQ];
   uint8_t q_rope[kRopeBytesQ];
   uint8_t kv[kStages][kAtoms][kAtomBytesKV];
   uint8_t kv_rope[kStages][kRopeBytesKV];
-  uint4 x[128 * 8];                              // peer's partial logits, fp16 (swizzled rows)
-  int sidx[kStages][kTileKeys];                  // the tile's slots, -1 where skipped
+  uint4 x[128 * 8];                              // the peer's partials of the current tile
+  uint4 stage[128 * 8];                          // this CTA's partials, the bulk copy's source
+  float pair_max[2][2][128];                     // [tile parity][key half][head]
+  unsigned valid[kStages][2];                    // selected-slot bits of each half tile
   unsigned long long q_full;
   unsigned long long kv_full[kStages];
   unsigned long long kv_empty[kStages];
@@ -66,9 +76,12 @@ struct MlaSmem {
   unsigned long long s_empty[2];
   unsigned long long p_full[2];
   unsigned long long p_empty[2];
-  unsigned long long x_full;                     // the peer's partial logits have landed in x
+  unsigned long long stage_full;                 // the eight softmax warps have staged the tile
+  unsigned long long stage_free;                 // the peer has received this CTA's last tile
+  unsigned long long x_full;                     // the peer's partials have landed in x
   unsigned long long x_free;                     // the peer has read what this CTA sent it
-  unsigned long long x_read;                     // the four softmax warps have read x
+  unsigned long long x_read;                     // the softmax warps have read x
+  unsigned long long pair;                       // the softmax warps have posted their maxima
   unsigned long long o_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -92,7 +105,6 @@ __device__ __forceinline__ int kv_row(const MlaArgs& A, int v, int seq, int limi
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaThreads, 1)
 sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
-                  const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_kvr,
                   const MlaArgs A) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   MlaSmem& sm = *reinterpret_cast<MlaSmem*>(
@@ -123,13 +135,16 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.s_full[i]), 1);
-      mbar_init(smem_u32(&sm.s_empty[i]), 128);
-      mbar_init(smem_u32(&sm.p_full[i]), 128);
+      mbar_init(smem_u32(&sm.s_empty[i]), kSoftmaxWarps);
+      mbar_init(smem_u32(&sm.p_full[i]), kSoftmaxWarps);
       mbar_init(smem_u32(&sm.p_empty[i]), 1);
     }
-    mbar_init(smem_u32(&sm.x_full), 1);          // own expect_tx + the peer's st.async bytes
-    mbar_init(smem_u32(&sm.x_free), 1);          // one release from the peer per tile
-    mbar_init(smem_u32(&sm.x_read), 4);
+    mbar_init(smem_u32(&sm.stage_full), kSoftmaxWarps);
+    mbar_init(smem_u32(&sm.stage_free), 1);      // one arrival from the peer per tile
+    mbar_init(smem_u32(&sm.x_full), 1);          // own expect_tx + the peer's copied bytes
+    mbar_init(smem_u32(&sm.x_free), 1);          // one arrival from the peer per tile
+    mbar_init(smem_u32(&sm.x_read), kSoftmaxWarps);
+    mbar_init(smem_u32(&sm.pair), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.o_done), 1);
     sm.abort_flag = aborted ? 1 : 0;
     fence_barrier_init();
@@ -144,12 +159,13 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
 
-  const int gw = warp == 0 ? 0 : (warp == 2 || warp == 3) ? warp - 1 : warp - 5;   // 0..5
-  if ((warp == 0 || warp == 2 || warp == 3 || (warp >= 8 && warp <= 10)) && !aborted) {
+  const bool gather = warp == 0 || warp == 2 || warp == 3 || (warp >= 12 && warp <= 14);
+  if (gather && !aborted) {
     // ------------------------------------------------------- gather warps
     // Each warp copies whole rows: one cp.async per lane covers the 512-B latent
     // slice of a row (coalesced), lanes 0-3 add its 64-B rope slice; rows land
     // in the 128-B (latent) and 64-B (rope) swizzled layouts the MMA reads.
+    const int gw = warp == 0 ? 0 : warp <= 3 ? warp - 1 : warp - 9;   // 0..5
     if (warp == 0 && lane == 0) {
       const uint32_t qf = smem_u32(&sm.q_full);
       mbar_expect_tx(qf, kAtoms * kAtomBytesQ + kRopeBytesQ);
@@ -173,10 +189,13 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         break;
       const uint32_t full = smem_u32(&sm.kv_full[st]);
       if (gw == 0) {
-        sm.sidx[st][lane] = r0 >= 0 ? c0 : -1;
-        sm.sidx[st][32 + lane] = r1 >= 0 ? c1 : -1;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(full);
+        const unsigned b0 = __ballot_sync(0xffffffffu, r0 >= 0);
+        const unsigned b1 = __ballot_sync(0xffffffffu, r1 >= 0);
+        if (lane == 0) {
+          sm.valid[st][0] = b0;
+          sm.valid[st][1] = b1;
+          mbar_arrive(full);
+        }
       }
       const uint32_t kv0 = smem_u32(sm.kv[st][lane >> 3]);
       const uint32_t rope = smem_u32(sm.kv_rope[st]);
@@ -192,15 +211,35 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     if (warp == 0 && lane == 0) mbar_drain(smem_u32(&sm.q_full), 0);
-  } else if (warp == 11 && !aborted) {
-    // ------------------------------------------ release x back to the peer
-    // This warp issues no remote stores, so its cluster-scope release does
-    // not wait behind the softmax warps' outgoing partials.
-    if (lane == 0)
+  } else if (warp == kExchangeWarp && !aborted) {
+    // ---------------------------------------------------- exchange warp
+    // Per tile: send the staged partials to the peer's x in one bulk copy once
+    // the peer has read its previous tile, then tell the peer when its own
+    // copy has landed here (its stage may be rewritten) and when x has been
+    // read (it may send the next tile). Cluster-scope releases come from this
+    // warp only, so they never queue behind the softmax warps' work.
+    if (lane == 0) {
+      const uint32_t peer_x = mapa(smem_u32(sm.x), peer);
+      const uint32_t peer_x_full = mapa(smem_u32(&sm.x_full), peer);
+      const uint32_t peer_stage_free = mapa(smem_u32(&sm.stage_free), peer);
+      const uint32_t peer_x_free = mapa(smem_u32(&sm.x_free), peer);
+      int sent = 0;
       for (int i = 0; i < ntiles; ++i) {
+        mbar_expect_tx(smem_u32(&sm.x_full), kXBytes);        // the peer's tile i
+        if (!mbar_wait(smem_u32(&sm.stage_full), i & 1, abort_flag, err)) break;
+        if (i > 0 && !mbar_wait<true>(smem_u32(&sm.x_free), (i - 1) & 1, abort_flag, err)) break;
+        bulk_copy_to_peer(peer_x, smem_u32(sm.stage), kXBytes, peer_x_full);
+        sent = i + 1;
+        if (!mbar_wait<true>(smem_u32(&sm.x_full), i & 1, abort_flag, err)) break;
+        mbar_arrive_remote(peer_stage_free);
         if (!mbar_wait(smem_u32(&sm.x_read), i & 1, abort_flag, err)) break;
-        mbar_arrive_remote(mapa(smem_u32(&sm.x_free), peer));
+        mbar_arrive_remote(peer_x_free);
       }
+      // The copy reads this CTA's stage until it lands: wait for the peer's
+      // word on the last one before this CTA may leave.
+      if (sent > 0 && !mbar_wait<true>(smem_u32(&sm.stage_free), (sent - 1) & 1, abort_flag, err))
+        mbar_drain(smem_u32(&sm.stage_free), (sent - 1) & 1);
+    }
   } else if (warp == 1 && !aborted) {
     // ------------------------------------------------------- MMA thread
     if (lane == 0) {
@@ -252,36 +291,34 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       mma_commit(smem_u32(&sm.o_done));
       mbar_drain(smem_u32(&sm.o_done), 0);
     }
-  } else if (warp >= 4 && !aborted) {
-    // ------------------------------------------------- softmax warpgroup
+  } else if (warp >= 4 && warp < 4 + kSoftmaxWarps && !aborted) {
+    // ------------------------------------------------- softmax warps
+    const int g = (warp - 4) >> 2;                      // key half of the tile
     const int h = 32 * (warp & 3) + lane;               // head = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    const uint32_t peer_x = mapa(smem_u32(sm.x), peer) + h * 128;
-    const uint32_t peer_x_full = mapa(smem_u32(&sm.x_full), peer);
     const uint4* my_x = sm.x + h * 8;
+    uint4* my_stage = sm.stage + h * 8;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int i = 0; ok && i < ntiles; ++i) {
       const int b = i & 1, st = i % kStages;
-      float s[64];
+      float s[32];
       if (!(ok = warp_wait(smem_u32(&sm.s_full[b]), (i >> 1) & 1, abort_flag, err))) break;
       tc_fence_after();
-      tmem_ld32(tmem + lane_base + kColS + b * kTileKeys, *reinterpret_cast<float(*)[32]>(s));
-      tmem_ld32(tmem + lane_base + kColS + b * kTileKeys + 32,
-                *reinterpret_cast<float(*)[32]>(s + 32));
+      tmem_ld32(tmem + lane_base + kColS + b * kTileKeys + 32 * g, s);
       tc_fence_before();
-      mbar_arrive(smem_u32(&sm.s_empty[b]));
-      // exchange partial logits with the peer CTA: this CTA's x receives the
-      // peer's 128 x 64 partials for tile i as fp16 (16 KB, credited to x_full);
-      // the shared-memory network between SMs is the scarce resource here, and
-      // fp16 keeps 11 bits of each partial (relative error 2^-11, below the
-      // bf16 rounding P gets before the PV product)
-      if (h == 0) mbar_expect_tx(smem_u32(&sm.x_full), 128 * 64 * 2);
-      if (i > 0 && !(ok = warp_wait<true>(smem_u32(&sm.x_free), (i - 1) & 1, abort_flag, err)))
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[b]));
+#pragma unroll
+      for (int j = 0; j < 32; ++j) s[j] *= A.sm_scale_log2;
+      // Stage this half tile for the peer as fp16 once the previous tile's copy
+      // has landed. fp16 keeps 11 bits of each partial (relative error 2^-11,
+      // below the bf16 rounding P gets before the PV product) and halves the
+      // bytes crossing the network between the two SMs, the scarce resource.
+      if (i > 0 && !(ok = warp_wait<true>(smem_u32(&sm.stage_free), (i - 1) & 1, abort_flag, err)))
         break;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int pc = c ^ (h & 7);
+      for (int c = 0; c < 4; ++c) {
         uint4 v;
         __half2 h0 = __floats2half2_rn(s[8 * c], s[8 * c + 1]);
         __half2 h1 = __floats2half2_rn(s[8 * c + 2], s[8 * c + 3]);
@@ -291,23 +328,19 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         v.y = *reinterpret_cast<uint32_t*>(&h1);
         v.z = *reinterpret_cast<uint32_t*>(&h2);
         v.w = *reinterpret_cast<uint32_t*>(&h3);
-        st_async_v4_b32(peer_x + pc * 16, v, peer_x_full);
+        my_stage[(4 * g + c) ^ (h & 7)] = v;
       }
-      // which slots of the tile are selected (staged by the gather warp)
+      fence_proxy_async_smem();           // generic writes -> the bulk copy's reads
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.stage_full));
+      // which slots of this half tile are selected (staged by the gather warp)
       if (!(ok = warp_wait(smem_u32(&sm.kv_full[st]), (i / kStages) & 1, abort_flag, err))) break;
-      unsigned long long valid = 0;
-#pragma unroll
-      for (int c = 0; c < kTileKeys / 4; ++c) {
-        const int4 v = *reinterpret_cast<const int4*>(&sm.sidx[st][4 * c]);
-        valid |= static_cast<unsigned long long>((v.x >= 0) | ((v.y >= 0) << 1) |
-                                                 ((v.z >= 0) << 2) | ((v.w >= 0) << 3))
-                 << (4 * c);
-      }
+      const unsigned valid = sm.valid[st][g];
+      // add the peer's partials, then hand x back
       if (!(ok = warp_wait<true>(smem_u32(&sm.x_full), i & 1, abort_flag, err))) break;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int pc = c ^ (h & 7);
-        const uint4 v = my_x[pc];
+      for (int c = 0; c < 4; ++c) {
+        const uint4 v = my_x[(4 * g + c) ^ (h & 7)];
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -316,20 +349,23 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           s[8 * c + 2 * e + 1] += f.y;
         }
       }
-      // warp 11 hands x back to the peer once all four warps have read it
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.x_read));
-      // mask unselected slots, scale into the log2 domain, tile maximum
-      float pm[8];
+      if (valid != 0xffffffffu) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) pm[e] = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < kTileKeys; ++j) {
-        s[j] = ((valid >> j) & 1ull) ? s[j] * A.sm_scale_log2 : -INFINITY;
-        pm[j & 7] = fmaxf(pm[j & 7], s[j]);
+        for (int j = 0; j < 32; ++j)
+          if (!((valid >> j) & 1u)) s[j] = -INFINITY;
       }
-      const float mt = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int j = 0; j < 32; ++j) pm[j & 3] = fmaxf(pm[j & 3], s[j]);
+      const float my_max = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
+      // the tile maximum of this head: both halves post theirs
+      sm.pair_max[i & 1][g][h] = my_max;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.pair));
+      if (!(ok = warp_wait(smem_u32(&sm.pair), i & 1, abort_flag, err))) break;
+      const float mt = fmaxf(my_max, sm.pair_max[i & 1][g ^ 1][h]);
       float alpha = 1.f;
       bool rescale = false;
       if (mt > m_ref + kRebase) {        // also the first tile with a selected key
@@ -344,72 +380,79 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           !(ok = warp_wait(smem_u32(&sm.p_empty[b]), ((i - 2) >> 1) & 1, abort_flag, err)))
         break;
       tc_fence_after();
-      float ps[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ps[e] = 0.f;
-      const bool live = m_ref > -INFINITY;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {     // 32 keys -> 16 packed columns at a time
+      {
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};
+        const bool live = m_ref > -INFINITY;
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const int j = 32 * half + 2 * c;
-          const float p0 = live ? fast_exp2(s[j] - m_ref) : 0.f;
-          const float p1 = live ? fast_exp2(s[j + 1] - m_ref) : 0.f;
-          ps[c & 7] += p0 + p1;
+          const float p0 = live ? fast_exp2(s[2 * c] - m_ref) : 0.f;
+          const float p1 = live ? fast_exp2(s[2 * c + 1] - m_ref) : 0.f;
+          ps[c & 3] += p0 + p1;
           const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
           pk[c] = *reinterpret_cast<const uint32_t*>(&pb);
         }
-        tmem_st16(tmem + lane_base + kColP + 32 * b + 16 * half, pk);
+        tmem_st16(tmem + lane_base + kColP + 32 * b + 16 * g, pk);
+        l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
       }
-      l = l * alpha + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])));
-      // a new reference maximum: rescale the output once PV(i-1) has finished
-      // (PV(i) cannot start before this warpgroup arrives on p_full below)
+      // a new reference maximum: rescale this warp's half of the output once
+      // PV(i-1) has finished (PV(i) cannot start before p_full below)
       if (rescale && i > 0) {
         if (!(ok = warp_wait(smem_u32(&sm.p_empty[(i - 1) & 1]), ((i - 1) >> 1) & 1, abort_flag,
                              err)))
           break;
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           float o[32];
-          tmem_ld32(tmem + lane_base + kColO + 32 * c, o);
+          const uint32_t col = tmem + lane_base + kColO + 128 * g + 32 * c;
+          tmem_ld32(col, o);
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          tmem_st32(tmem + lane_base + kColO + 32 * c, o);
+          tmem_st32(col, o);
         }
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&sm.p_full[b]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[b]));
     }
     // ------------------------------------------------------- epilogue
+    // The row sum is the sum over both key halves; each warp of a pair then
+    // writes its 128 of this CTA's 256 output dims.
     if (ok && ntiles > 0 &&
         warp_wait(smem_u32(&sm.p_empty[(ntiles - 1) & 1]), ((ntiles - 1) >> 1) & 1, abort_flag,
                   err)) {
-      tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      const bool head_ok = h < A.H;
-      __nv_bfloat16* orow = A.out + (static_cast<long long>(r) * A.H + h) * 512 + dim0;
+      sm.pair_max[ntiles & 1][g][h] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.pair));
+      if (warp_wait(smem_u32(&sm.pair), ntiles & 1, abort_flag, err)) {
+        const float lt = l + sm.pair_max[ntiles & 1][g ^ 1][h];
+        tc_fence_after();
+        const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
+        const bool head_ok = h < A.H;
+        __nv_bfloat16* orow = A.out + (static_cast<long long>(r) * A.H + h) * 512 + dim0 + 128 * g;
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        float o[32];
-        tmem_ld32(tmem + lane_base + kColO + 32 * c, o);
-        if (head_ok) {
-          uint32_t pk[16];
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          tmem_ld32(tmem + lane_base + kColO + 128 * g + 32 * c, o);
+          if (head_ok) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const __nv_bfloat162 v = __floats2bfloat162_rn(o[2 * e] * inv_l, o[2 * e + 1] * inv_l);
-            pk[e] = *reinterpret_cast<const uint32_t*>(&v);
+            for (int e = 0; e < 16; ++e) {
+              const __nv_bfloat162 v =
+                  __floats2bfloat162_rn(o[2 * e] * inv_l, o[2 * e + 1] * inv_l);
+              pk[e] = *reinterpret_cast<const uint32_t*>(&v);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
           }
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         }
+        if (rank == 0 && g == 0 && head_ok && A.lse)
+          A.lse[static_cast<long long>(r) * A.H + h] =
+              lt > 0.f ? (m_ref + log2f(lt)) * 0.69314718055994531f : -INFINITY;
       }
-      if (rank == 0 && head_ok && A.lse)
-        A.lse[static_cast<long long>(r) * A.H + h] =
-            l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }
   tc_fence_before();
@@ -428,23 +471,19 @@ cudaError_t launch_sparse_mla(const MlaArgs& a_in, const void* q, const void* kv
   MlaArgs a = a_in;
   a.kv_rows = static_cast<int>(kv_rows);
   a.kv = static_cast<const __nv_bfloat16*>(kv);
-  CUtensorMap tq, tqr, tkv, tkvr;
+  CUtensorMap tq, tqr;
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   cudaError_t e =
       make_tmap_2d(&tq, q, bf, 576, q_rows, 576 * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e == cudaSuccess)
     e = make_tmap_2d(&tqr, q, bf, 576, q_rows, 576 * 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
-  if (e == cudaSuccess)
-    e = make_tmap_2d(&tkv, kv, bf, 576, kv_rows, 576 * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (e == cudaSuccess)
-    e = make_tmap_2d(&tkvr, kv, bf, 576, kv_rows, 576 * 2, 32, 1, CU_TENSOR_MAP_SWIZZLE_64B);
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(MlaSmem) + 1024;
   e = cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(2 * a.T);      // x has no 65535 limit; cluster pairs are consecutive x
-  sparse_mla_kernel<<<grid, kMlaThreads, smem, st>>>(tq, tqr, tkv, tkvr, a);
+  sparse_mla_kernel<<<grid, kMlaThreads, smem, st>>>(tq, tqr, a);
   return cudaGetLastError();
 }
 
