@@ -206,6 +206,13 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const long long s = static_cast<long long>(tile0 + i) * kKeyTile + row;   // logical key
       const bool key_ok = s < key_limit;
       const uint32_t taddr = tmem + lane_base + g * ncol;
+      // hand the buffer back to the MMA as soon as its last columns are in
+      // registers, so the next MMA into it overlaps the tail of this epilogue
+      auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.t_empty[g]));
+      };
       auto emit = [&](int qq, float acc) {
         if (qq >= nqb || !key_ok) return;
         const long long t = q0 + qq;
@@ -221,6 +228,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int c = 0; c < ncol / 64; ++c) {
           float v[64];
           tmem_ld64(taddr + c * 64, v);
+          if (c == ncol / 64 - 1) release();
           const float2* wp = reinterpret_cast<const float2*>(sm.w + c * 64);
 #pragma unroll
           for (int sub = 0; sub < 2; ++sub) {
@@ -245,6 +253,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int c = 0; c < ncol / 32; ++c) {
           float v[32];
           tmem_ld32(taddr + c * 32, v);
+          if (c == ncol / 32 - 1) release();
           const float* wp = sm.w + c * 32;
 #pragma unroll
           for (int qq = 0; qq < 32 / HI; ++qq) {
@@ -256,9 +265,6 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.t_empty[g]));
     }
   }
   tc_fence_before();
