@@ -17,10 +17,11 @@
 // CTAs do the same work, each gathers only the dims it uses, and every
 // selected byte crosses HBM once. Per tile of 64 selected keys:
 //   1. six gather warps copy the CTA's dims of the 64 rows with coalesced
-//      cp.async (through the block table for the paged cache), up to three
+//      cp.async (through the block table for the paged cache), up to five
 //      tiles ahead;
-//   2. warp 1 issues S_c = Q_c K_c^T (M=128 heads, N=64 keys, K=288) into
-//      one of two TMEM logit buffers;
+//   2. warp 1 issues S_c = Q_c K_c^T (M=128 heads, N=64 keys, K=288) with
+//      Q_c read from TMEM, where it was placed once per query, and K_c from
+//      the gathered tile, into the TMEM logit buffer;
 //   3. eight softmax warps, two per TMEM lane quarter (thread = head, each
 //      warp of a pair taking 32 of the 64 keys), scale their partial logits
 //      into the log2 domain and stage them as fp16 in shared memory; the
@@ -28,7 +29,7 @@
 //      copy (the TMA engine, off the load/store path the gather uses). The
 //      softmax warps add the peer's partials, mask unselected slots, agree on
 //      the tile maximum through shared memory, run the online softmax in the
-//      exp2 domain and store P (bf16) into one of two TMEM P buffers; the
+//      exp2 domain and store P (bf16) into the TMEM P buffer; the
 //      running maximum is re-based only when it grows by more than 8 (log2
 //      units), and only then is the output in TMEM rescaled;
 //   4. warp 1 issues O_c += P V_c with P read from TMEM (M=128, N=256 dims,
@@ -43,7 +44,7 @@ namespace {
 
 constexpr int kMlaThreads = 512;
 constexpr int kTileKeys = 64;
-constexpr int kStages = 3;
+constexpr int kStages = 5;
 constexpr int kAtoms = 4;                        // 128-B swizzled atoms of 64 dims
 constexpr int kAtomBytesQ = 128 * 128;           // 128 heads x 64 dims bf16
 constexpr int kRopeBytesQ = 128 * 64;            // 128 heads x 32 dims bf16 (64-B swizzle)
@@ -54,28 +55,31 @@ constexpr int kSoftmaxWarps = 8;                 // warps 4-11
 constexpr int kExchangeWarp = 15;
 constexpr uint32_t kXBytes = 128 * kTileKeys * 2;   // one tile of fp16 partial logits
 constexpr uint32_t kColO = 0;                    // TMEM columns [0,256): output
-constexpr uint32_t kColS = 256;                  // [256,384): two logit buffers
-constexpr uint32_t kColP = 384;                  // [384,448): two P buffers (bf16 pairs)
+constexpr uint32_t kColQ = 256;                  // [256,400): Q_c, bf16 pairs (256 + 32 dims)
+constexpr uint32_t kColP = 416;                  // [416,448): P, bf16 pairs
+constexpr uint32_t kColS = 448;                  // [448,512): logits
+// Q arrives by TMA in ring stages 3-4 (72 KB) and is moved into TMEM before
+// the gather first reaches stage 3.
+constexpr int kQStage = 3;
 constexpr float kRebase = 8.0f;                  // lazy rescale threshold (log2 units)
 
 // Rows of 64 fp16 partials (128 B, one per head); the 16-B chunk c of row h
 // sits at chunk c ^ (h & 7), so eight consecutive heads hit distinct banks.
 struct MlaSmem {
-  uint8_t q[kAtoms][kAtomBytesQ];
-  uint8_t q_rope[kRopeBytesQ];
   uint8_t kv[kStages][kAtoms][kAtomBytesKV];
   uint8_t kv_rope[kStages][kRopeBytesKV];
   uint4 x[128 * 8];                              // the peer's partials of the current tile
   uint4 stage[128 * 8];                          // this CTA's partials, the bulk copy's source
   float pair_max[2][2][128];                     // [tile parity][key half][head]
   unsigned valid[kStages][2];                    // selected-slot bits of each half tile
-  unsigned long long q_full;
+  unsigned long long q_full;                     // Q has landed in its staging slots
+  unsigned long long q_ready;                    // Q is in TMEM (stages 3-4 are free)
   unsigned long long kv_full[kStages];
   unsigned long long kv_empty[kStages];
-  unsigned long long s_full[2];
-  unsigned long long s_empty[2];
-  unsigned long long p_full[2];
-  unsigned long long p_empty[2];
+  unsigned long long s_full;
+  unsigned long long s_empty;
+  unsigned long long p_full;
+  unsigned long long p_empty;
   unsigned long long stage_full;                 // the eight softmax warps have staged the tile
   unsigned long long stage_free;                 // the peer has received this CTA's last tile
   unsigned long long x_full;                     // the peer's partials have landed in x
@@ -86,6 +90,10 @@ struct MlaSmem {
   uint32_t tmem_base;
   int abort_flag;
 };
+
+static_assert(2 * kAtoms * kAtomBytesKV == kAtoms * kAtomBytesQ, "Q latent staging = 2 stages");
+static_assert(2 * kRopeBytesKV == kRopeBytesQ, "Q rope staging = 2 stages");
+static_assert(kQStage + 2 <= kStages, "Q staging inside the ring");
 
 // Physical row of slot value `v` (a logical position), or -1 if skipped.
 __device__ __forceinline__ int kv_row(const MlaArgs& A, int v, int seq, int limit) {
@@ -128,17 +136,16 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&sm.q_full), 1);
+    mbar_init(smem_u32(&sm.q_ready), 4);         // the four warps that move Q into TMEM
     for (int i = 0; i < kStages; ++i) {
       // one cp.async-completion arrival per gathering thread + the slot writer
       mbar_init(smem_u32(&sm.kv_full[i]), 32 * kGatherWarps + 1);
       mbar_init(smem_u32(&sm.kv_empty[i]), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&sm.s_full[i]), 1);
-      mbar_init(smem_u32(&sm.s_empty[i]), kSoftmaxWarps);
-      mbar_init(smem_u32(&sm.p_full[i]), kSoftmaxWarps);
-      mbar_init(smem_u32(&sm.p_empty[i]), 1);
-    }
+    mbar_init(smem_u32(&sm.s_full), 1);
+    mbar_init(smem_u32(&sm.s_empty), kSoftmaxWarps);
+    mbar_init(smem_u32(&sm.p_full), kSoftmaxWarps);
+    mbar_init(smem_u32(&sm.p_empty), 1);
     mbar_init(smem_u32(&sm.stage_full), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.stage_free), 1);      // one arrival from the peer per tile
     mbar_init(smem_u32(&sm.x_full), 1);          // own expect_tx + the peer's copied bytes
@@ -169,9 +176,10 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (warp == 0 && lane == 0) {
       const uint32_t qf = smem_u32(&sm.q_full);
       mbar_expect_tx(qf, kAtoms * kAtomBytesQ + kRopeBytesQ);
+      const uint32_t qs = smem_u32(sm.kv[kQStage][0]);
       for (int a = 0; a < kAtoms; ++a)
-        tma_load_2d(smem_u32(sm.q[a]), &tm_q, qf, dim0 + 64 * a, r * A.H);
-      tma_load_2d(smem_u32(sm.q_rope), &tm_qr, qf, rope0, r * A.H);
+        tma_load_2d(qs + a * kAtomBytesQ, &tm_q, qf, dim0 + 64 * a, r * A.H);
+      tma_load_2d(smem_u32(sm.kv_rope[kQStage]), &tm_qr, qf, rope0, r * A.H);
     }
     int v0 = lane < A.k ? __ldg(sel + lane) : -1;
     int v1 = lane + 32 < A.k ? __ldg(sel + lane + 32) : -1;
@@ -184,6 +192,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         v1 = j0 + 32 < A.k ? __ldg(sel + j0 + 32) : -1;
       }
       const int r0 = kv_row(A, c0, seq, limit), r1 = kv_row(A, c1, seq, limit);
+      if (i == kQStage && !warp_wait(smem_u32(&sm.q_ready), 0, abort_flag, err)) break;
       if (i >= kStages &&
           !warp_wait(smem_u32(&sm.kv_empty[st]), ((i / kStages) + 1) & 1, abort_flag, err))
         break;
@@ -245,43 +254,42 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16(128, kTileKeys, false);
       const uint32_t id_pv = idesc_bf16(128, 256, true);
-      bool ok = mbar_wait(smem_u32(&sm.q_full), 0, abort_flag, err);
+      bool ok = mbar_wait(smem_u32(&sm.q_ready), 0, abort_flag, err);
       auto issue_pv = [&](int i) -> bool {
-        const int st = i % kStages, b = i & 1;
-        if (!mbar_wait(smem_u32(&sm.p_full[b]), (i >> 1) & 1, abort_flag, err)) return false;
+        const int st = i % kStages;
+        if (!mbar_wait(smem_u32(&sm.p_full), i & 1, abort_flag, err)) return false;
         tc_fence_after();
         const uint64_t vdesc = sdesc_sw128(smem_u32(sm.kv[st][0]), kAtomBytesKV, 1024);
 #pragma unroll
         for (int kk = 0; kk < kTileKeys / 16; ++kk)   // 16 keys: 8 P columns, 2 V row groups
-          mma_bf16_ts(tmem + kColO, tmem + kColP + 32 * b + 8 * kk, vdesc + (kk * 2048 >> 4),
-                      id_pv, (i > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(smem_u32(&sm.p_empty[b]));
+          mma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk, vdesc + (kk * 2048 >> 4), id_pv,
+                      (i > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(smem_u32(&sm.p_empty));
         mma_commit(smem_u32(&sm.kv_empty[st]));
         return true;
       };
       int done_pv = 0;
       for (int i = 0; ok && i < ntiles; ++i) {
-        const int st = i % kStages, b = i & 1;
+        const int st = i % kStages;
         if (!mbar_wait(smem_u32(&sm.kv_full[st]), (i / kStages) & 1, abort_flag, err)) break;
-        if (i >= 2 && !mbar_wait(smem_u32(&sm.s_empty[b]), ((i >> 1) + 1) & 1, abort_flag, err))
-          break;
+        // the softmax warps have read the previous tile's logits
+        if (i >= 1 && !mbar_wait(smem_u32(&sm.s_empty), (i - 1) & 1, abort_flag, err)) break;
         fence_proxy_async_smem();         // cp.async (generic) writes -> tensor-core reads
         tc_fence_after();
-        const uint32_t d = tmem + kColS + b * kTileKeys;
+        const uint32_t d = tmem + kColS;
         for (int a = 0; a < kAtoms; ++a) {
-          const uint64_t qd = sdesc_sw128(smem_u32(sm.q[a]), 0, 1024);
           const uint64_t kd = sdesc_sw128(smem_u32(sm.kv[st][a]), 0, 1024);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)          // 4 x K=16 dims (32 bytes)
-            mma_bf16(d, qd + 2 * kk, kd + 2 * kk, id_qk, (a > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk)          // 4 x K=16 dims (8 TMEM columns of Q)
+            mma_bf16_ts(d, tmem + kColQ + 32 * a + 8 * kk, kd + 2 * kk, id_qk,
+                        (a > 0 || kk > 0) ? 1u : 0u);
         }
         {
-          const uint64_t qd = sdesc_sw64(smem_u32(sm.q_rope), 512);
           const uint64_t kd = sdesc_sw64(smem_u32(sm.kv_rope[st]), 512);
-          mma_bf16(d, qd, kd, id_qk, 1u);
-          mma_bf16(d, qd + 2, kd + 2, id_qk, 1u);
+          mma_bf16_ts(d, tmem + kColQ + 128, kd, id_qk, 1u);
+          mma_bf16_ts(d, tmem + kColQ + 136, kd + 2, id_qk, 1u);
         }
-        mma_commit(smem_u32(&sm.s_full[b]));
+        mma_commit(smem_u32(&sm.s_full));
         if (i > 0) {
           if (!issue_pv(i - 1)) break;
           done_pv = i;
@@ -300,15 +308,56 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint4* my_stage = sm.stage + h * 8;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
+    if (g == 0) {
+      // Move this head's row of Q_c from its staging slots into TMEM (bf16
+      // pairs, lane = head): 256 latent dims from the 128-B swizzled atoms,
+      // then the 32 rope dims from the 64-B swizzled block.
+      if ((ok = warp_wait(smem_u32(&sm.q_full), 0, abort_flag, err))) {
+        const uint8_t* qs = sm.kv[kQStage][0];
+#pragma unroll 1
+        for (int a = 0; a < kAtoms; ++a) {
+          const uint4* row = reinterpret_cast<const uint4*>(qs + a * kAtomBytesQ + h * 128);
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint4 v = row[(4 * half + c) ^ (h & 7)];
+              pk[4 * c] = v.x;
+              pk[4 * c + 1] = v.y;
+              pk[4 * c + 2] = v.z;
+              pk[4 * c + 3] = v.w;
+            }
+            tmem_st16(tmem + lane_base + kColQ + 32 * a + 16 * half, pk);
+          }
+        }
+        {
+          const uint4* row = reinterpret_cast<const uint4*>(sm.kv_rope[kQStage] + h * 64);
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 v = row[c ^ ((h >> 1) & 3)];
+            pk[4 * c] = v.x;
+            pk[4 * c + 1] = v.y;
+            pk[4 * c + 2] = v.z;
+            pk[4 * c + 3] = v.w;
+          }
+          tmem_st16(tmem + lane_base + kColQ + 128, pk);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.q_ready));
+      }
+    }
     for (int i = 0; ok && i < ntiles; ++i) {
-      const int b = i & 1, st = i % kStages;
+      const int st = i % kStages;
       float s[32];
-      if (!(ok = warp_wait(smem_u32(&sm.s_full[b]), (i >> 1) & 1, abort_flag, err))) break;
+      if (!(ok = warp_wait(smem_u32(&sm.s_full), i & 1, abort_flag, err))) break;
       tc_fence_after();
-      tmem_ld32(tmem + lane_base + kColS + b * kTileKeys + 32 * g, s);
+      tmem_ld32(tmem + lane_base + kColS + 32 * g, s);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[b]));
+      if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty));
 #pragma unroll
       for (int j = 0; j < 32; ++j) s[j] *= A.sm_scale_log2;
       // Stage this half tile for the peer as fp16 once the previous tile's copy
@@ -375,10 +424,9 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         m_ref = mt;
       }
-      // P buffer b is free once PV(i-2) has finished
-      if (i >= 2 &&
-          !(ok = warp_wait(smem_u32(&sm.p_empty[b]), ((i - 2) >> 1) & 1, abort_flag, err)))
-        break;
+      // P (and the output, if it is rescaled below) is free once PV(i-1) has
+      // finished; PV(i) cannot start before p_full at the end of this tile
+      if (i >= 1 && !(ok = warp_wait(smem_u32(&sm.p_empty), (i - 1) & 1, abort_flag, err))) break;
       tc_fence_after();
       {
         float ps[4] = {0.f, 0.f, 0.f, 0.f};
@@ -392,16 +440,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
           pk[c] = *reinterpret_cast<const uint32_t*>(&pb);
         }
-        tmem_st16(tmem + lane_base + kColP + 32 * b + 16 * g, pk);
+        tmem_st16(tmem + lane_base + kColP + 16 * g, pk);
         l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
       }
-      // a new reference maximum: rescale this warp's half of the output once
-      // PV(i-1) has finished (PV(i) cannot start before p_full below)
-      if (rescale && i > 0) {
-        if (!(ok = warp_wait(smem_u32(&sm.p_empty[(i - 1) & 1]), ((i - 1) >> 1) & 1, abort_flag,
-                             err)))
-          break;
-        tc_fence_after();
+      // a new reference maximum: rescale this warp's half of the output
+      if (rescale) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           float o[32];
@@ -414,14 +457,13 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[b]));
+      if (lane == 0) mbar_arrive(smem_u32(&sm.p_full));
     }
     // ------------------------------------------------------- epilogue
     // The row sum is the sum over both key halves; each warp of a pair then
     // writes its 128 of this CTA's 256 output dims.
     if (ok && ntiles > 0 &&
-        warp_wait(smem_u32(&sm.p_empty[(ntiles - 1) & 1]), ((ntiles - 1) >> 1) & 1, abort_flag,
-                  err)) {
+        warp_wait(smem_u32(&sm.p_empty), (ntiles - 1) & 1, abort_flag, err)) {
       sm.pair_max[ntiles & 1][g][h] = l;
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.pair));
