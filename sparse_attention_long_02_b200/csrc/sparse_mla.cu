@@ -17,7 +17,7 @@
 // CTAs do the same work, each gathers only the dims it uses, and every
 // selected byte crosses HBM once. Per tile of 64 selected keys:
 //   1. six gather warps copy the CTA's dims of the 64 rows with coalesced
-//      cp.async (through the block table for the paged cache), up to five
+//      cp.async (through the block table for the paged cache), up to four
 //      tiles ahead;
 //   2. warp 1 issues S_c = Q_c K_c^T (M=128 heads, N=64 keys, K=288) with
 //      Q_c read from TMEM, where it was placed once per query, and K_c from
@@ -26,8 +26,10 @@
 //      warp of a pair taking 32 of the 64 keys), scale their partial logits
 //      into the log2 domain and stage them as fp16 in shared memory; the
 //      exchange warp sends the whole 16 KB tile to the peer CTA with one bulk
-//      copy (the TMA engine, off the load/store path the gather uses). The
-//      softmax warps add the peer's partials, mask unselected slots, agree on
+//      copy (the TMA engine, off the load/store path the gather uses). Tile
+//      i+1 is staged and sent while tile i is finished, so the transfer runs
+//      under the softmax arithmetic. Both CTAs add the same two fp16 partials,
+//      so they see identical logits; they mask unselected slots, agree on
 //      the tile maximum through shared memory, run the online softmax in the
 //      exp2 domain and store P (bf16) into the TMEM P buffer; the
 //      running maximum is re-based only when it grows by more than 8 (log2
@@ -44,7 +46,7 @@ namespace {
 
 constexpr int kMlaThreads = 512;
 constexpr int kTileKeys = 64;
-constexpr int kStages = 5;
+constexpr int kStages = 4;
 constexpr int kAtoms = 4;                        // 128-B swizzled atoms of 64 dims
 constexpr int kAtomBytesQ = 128 * 128;           // 128 heads x 64 dims bf16
 constexpr int kRopeBytesQ = 128 * 64;            // 128 heads x 32 dims bf16 (64-B swizzle)
@@ -58,9 +60,9 @@ constexpr uint32_t kColO = 0;                    // TMEM columns [0,256): output
 constexpr uint32_t kColQ = 256;                  // [256,400): Q_c, bf16 pairs (256 + 32 dims)
 constexpr uint32_t kColP = 416;                  // [416,448): P, bf16 pairs
 constexpr uint32_t kColS = 448;                  // [448,512): logits
-// Q arrives by TMA in ring stages 3-4 (72 KB) and is moved into TMEM before
-// the gather first reaches stage 3.
-constexpr int kQStage = 3;
+// Q arrives by TMA in ring stages 2-3 (72 KB) and is moved into TMEM before
+// the gather first reaches stage 2.
+constexpr int kQStage = 2;
 constexpr float kRebase = 8.0f;                  // lazy rescale threshold (log2 units)
 
 // Rows of 64 fp16 partials (128 B, one per head); the 16-B chunk c of row h
@@ -68,23 +70,24 @@ constexpr float kRebase = 8.0f;                  // lazy rescale threshold (log2
 struct MlaSmem {
   uint8_t kv[kStages][kAtoms][kAtomBytesKV];
   uint8_t kv_rope[kStages][kRopeBytesKV];
-  uint4 x[128 * 8];                              // the peer's partials of the current tile
-  uint4 stage[128 * 8];                          // this CTA's partials, the bulk copy's source
+  uint4 x[2][128 * 8];                           // the peer's partials, by tile parity
+  uint4 stage[2][128 * 8];                       // this CTA's partials (bulk copy source)
   float pair_max[2][2][128];                     // [tile parity][key half][head]
   unsigned valid[kStages][2];                    // selected-slot bits of each half tile
   unsigned long long q_full;                     // Q has landed in its staging slots
-  unsigned long long q_ready;                    // Q is in TMEM (stages 3-4 are free)
+  unsigned long long q_ready;                    // Q is in TMEM (stages 2-3 are free)
   unsigned long long kv_full[kStages];
   unsigned long long kv_empty[kStages];
   unsigned long long s_full;
   unsigned long long s_empty;
   unsigned long long p_full;
   unsigned long long p_empty;
-  unsigned long long stage_full;                 // the eight softmax warps have staged the tile
-  unsigned long long stage_free;                 // the peer has received this CTA's last tile
-  unsigned long long x_full;                     // the peer's partials have landed in x
-  unsigned long long x_free;                     // the peer has read what this CTA sent it
-  unsigned long long x_read;                     // the softmax warps have read x
+  // per buffer (tile parity):
+  unsigned long long stage_full[2];              // the eight softmax warps have staged a tile
+  unsigned long long stage_free[2];              // the peer has received the tile staged here
+  unsigned long long x_full[2];                  // the peer's partials have landed in x
+  unsigned long long x_free[2];                  // the peer has read what this CTA sent it
+  unsigned long long x_read[2];                  // the softmax warps have read x
   unsigned long long pair;                       // the softmax warps have posted their maxima
   unsigned long long o_done;
   uint32_t tmem_base;
@@ -146,11 +149,13 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mbar_init(smem_u32(&sm.s_empty), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.p_full), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.p_empty), 1);
-    mbar_init(smem_u32(&sm.stage_full), kSoftmaxWarps);
-    mbar_init(smem_u32(&sm.stage_free), 1);      // one arrival from the peer per tile
-    mbar_init(smem_u32(&sm.x_full), 1);          // own expect_tx + the peer's copied bytes
-    mbar_init(smem_u32(&sm.x_free), 1);          // one arrival from the peer per tile
-    mbar_init(smem_u32(&sm.x_read), kSoftmaxWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&sm.stage_full[b]), kSoftmaxWarps);
+      mbar_init(smem_u32(&sm.stage_free[b]), 1);  // one arrival from the peer per use
+      mbar_init(smem_u32(&sm.x_full[b]), 1);      // own expect_tx + the peer's copied bytes
+      mbar_init(smem_u32(&sm.x_free[b]), 1);      // one arrival from the peer per use
+      mbar_init(smem_u32(&sm.x_read[b]), kSoftmaxWarps);
+    }
     mbar_init(smem_u32(&sm.pair), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.o_done), 1);
     sm.abort_flag = aborted ? 1 : 0;
@@ -222,32 +227,42 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (warp == 0 && lane == 0) mbar_drain(smem_u32(&sm.q_full), 0);
   } else if (warp == kExchangeWarp && !aborted) {
     // ---------------------------------------------------- exchange warp
-    // Per tile: send the staged partials to the peer's x in one bulk copy once
-    // the peer has read its previous tile, then tell the peer when its own
-    // copy has landed here (its stage may be rewritten) and when x has been
-    // read (it may send the next tile). Cluster-scope releases come from this
-    // warp only, so they never queue behind the softmax warps' work.
+    // Tile j's partials travel from stage[j & 1] to the peer's x[j & 1] in
+    // one bulk copy, once they are staged and the peer has read tile j-2 out
+    // of that buffer. This warp also tells the peer when its copy of tile i
+    // has landed here (its stage buffer may be refilled) and when x has been
+    // read (it may send into that buffer again). Cluster-scope releases come
+    // from this warp only, so they never queue behind the softmax warps.
     if (lane == 0) {
-      const uint32_t peer_x = mapa(smem_u32(sm.x), peer);
-      const uint32_t peer_x_full = mapa(smem_u32(&sm.x_full), peer);
-      const uint32_t peer_stage_free = mapa(smem_u32(&sm.stage_free), peer);
-      const uint32_t peer_x_free = mapa(smem_u32(&sm.x_free), peer);
       int sent = 0;
-      for (int i = 0; i < ntiles; ++i) {
-        mbar_expect_tx(smem_u32(&sm.x_full), kXBytes);        // the peer's tile i
-        if (!mbar_wait(smem_u32(&sm.stage_full), i & 1, abort_flag, err)) break;
-        if (i > 0 && !mbar_wait<true>(smem_u32(&sm.x_free), (i - 1) & 1, abort_flag, err)) break;
-        bulk_copy_to_peer(peer_x, smem_u32(sm.stage), kXBytes, peer_x_full);
-        sent = i + 1;
-        if (!mbar_wait<true>(smem_u32(&sm.x_full), i & 1, abort_flag, err)) break;
-        mbar_arrive_remote(peer_stage_free);
-        if (!mbar_wait(smem_u32(&sm.x_read), i & 1, abort_flag, err)) break;
-        mbar_arrive_remote(peer_x_free);
+      auto send = [&](int j) -> bool {
+        const int b = j & 1;
+        if (!mbar_wait(smem_u32(&sm.stage_full[b]), (j >> 1) & 1, abort_flag, err)) return false;
+        if (j >= 2 && !mbar_wait<true>(smem_u32(&sm.x_free[b]), ((j - 2) >> 1) & 1, abort_flag, err))
+          return false;
+        bulk_copy_to_peer(mapa(smem_u32(sm.x[b]), peer), smem_u32(sm.stage[b]), kXBytes,
+                          mapa(smem_u32(&sm.x_full[b]), peer));
+        sent = j + 1;
+        return true;
+      };
+      for (int j = 0; j < 2 && j < ntiles; ++j)                 // the peer's tiles 0 and 1
+        mbar_expect_tx(smem_u32(&sm.x_full[j]), kXBytes);
+      bool ok = send(0);
+      for (int i = 0; ok && i < ntiles; ++i) {
+        const int b = i & 1;
+        if (i + 1 < ntiles && !(ok = send(i + 1))) break;
+        if (!(ok = mbar_wait<true>(smem_u32(&sm.x_full[b]), (i >> 1) & 1, abort_flag, err))) break;
+        mbar_arrive_remote(mapa(smem_u32(&sm.stage_free[b]), peer));
+        if (i + 2 < ntiles) mbar_expect_tx(smem_u32(&sm.x_full[b]), kXBytes);   // tile i+2
+        if (!(ok = mbar_wait(smem_u32(&sm.x_read[b]), (i >> 1) & 1, abort_flag, err))) break;
+        mbar_arrive_remote(mapa(smem_u32(&sm.x_free[b]), peer));
       }
-      // The copy reads this CTA's stage until it lands: wait for the peer's
-      // word on the last one before this CTA may leave.
-      if (sent > 0 && !mbar_wait<true>(smem_u32(&sm.stage_free), (sent - 1) & 1, abort_flag, err))
-        mbar_drain(smem_u32(&sm.stage_free), (sent - 1) & 1);
+      // A copy reads this CTA's stage buffer until it lands: wait for the
+      // peer's word on the last two before this CTA may leave.
+      for (int j = sent > 2 ? sent - 2 : 0; j < sent; ++j) {
+        const uint32_t bar = smem_u32(&sm.stage_free[j & 1]);
+        if (!mbar_wait<true>(bar, (j >> 1) & 1, abort_flag, err)) mbar_drain(bar, (j >> 1) & 1);
+      }
     }
   } else if (warp == 1 && !aborted) {
     // ------------------------------------------------------- MMA thread
@@ -268,7 +283,9 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mma_commit(smem_u32(&sm.kv_empty[st]));
         return true;
       };
-      int done_pv = 0;
+      // QK runs two tiles ahead of PV: the softmax reads tile i+1's logits
+      // while it finishes tile i
+      int next_pv = 0;
       for (int i = 0; ok && i < ntiles; ++i) {
         const int st = i % kStages;
         if (!mbar_wait(smem_u32(&sm.kv_full[st]), (i / kStages) & 1, abort_flag, err)) break;
@@ -290,12 +307,12 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           mma_bf16_ts(d, tmem + kColQ + 136, kd + 2, id_qk, 1u);
         }
         mma_commit(smem_u32(&sm.s_full));
-        if (i > 0) {
-          if (!issue_pv(i - 1)) break;
-          done_pv = i;
+        if (i >= 2) {
+          if (!(ok = issue_pv(i - 2))) break;
+          next_pv = i - 1;
         }
       }
-      if (ok && done_pv == ntiles - 1 && !*abort_flag) issue_pv(ntiles - 1);
+      while (ok && next_pv < ntiles && !*abort_flag && issue_pv(next_pv)) ++next_pv;
       mma_commit(smem_u32(&sm.o_done));
       mbar_drain(smem_u32(&sm.o_done), 0);
     }
@@ -304,8 +321,6 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int g = (warp - 4) >> 2;                      // key half of the tile
     const int h = 32 * (warp & 3) + lane;               // head = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    const uint4* my_x = sm.x + h * 8;
-    uint4* my_stage = sm.stage + h * 8;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     if (g == 0) {
@@ -349,57 +364,72 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (lane == 0) mbar_arrive(smem_u32(&sm.q_ready));
       }
     }
-    for (int i = 0; ok && i < ntiles; ++i) {
-      const int st = i % kStages;
-      float s[32];
-      if (!(ok = warp_wait(smem_u32(&sm.s_full), i & 1, abort_flag, err))) break;
+    // This warp's half of tile j's partial logits, scaled into log2 units
+    // and rounded to fp16: staged for the peer and kept here, so that both
+    // CTAs add the same two fp16 values. fp16 keeps 11 bits of each partial
+    // (relative error 2^-11, below the bf16 rounding P gets before the PV
+    // product) and halves the bytes crossing the network between the two
+    // SMs, the scarce resource.
+    uint32_t own[16];
+    auto stage_tile = [&](int j, uint32_t (&keep)[16]) -> bool {
+      const int b = j & 1;
+      float v32[32];
+      if (!warp_wait(smem_u32(&sm.s_full), j & 1, abort_flag, err)) return false;
       tc_fence_after();
-      tmem_ld32(tmem + lane_base + kColS + 32 * g, s);
+      tmem_ld32(tmem + lane_base + kColS + 32 * g, v32);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty));
-#pragma unroll
-      for (int j = 0; j < 32; ++j) s[j] *= A.sm_scale_log2;
-      // Stage this half tile for the peer as fp16 once the previous tile's copy
-      // has landed. fp16 keeps 11 bits of each partial (relative error 2^-11,
-      // below the bf16 rounding P gets before the PV product) and halves the
-      // bytes crossing the network between the two SMs, the scarce resource.
-      if (i > 0 && !(ok = warp_wait<true>(smem_u32(&sm.stage_free), (i - 1) & 1, abort_flag, err)))
-        break;
+      // the buffer held tile j-2: its copy must have landed at the peer
+      if (j >= 2 &&
+          !warp_wait<true>(smem_u32(&sm.stage_free[b]), ((j - 2) >> 1) & 1, abort_flag, err))
+        return false;
+      uint4* dst = sm.stage[b] + h * 8;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint4 v;
-        __half2 h0 = __floats2half2_rn(s[8 * c], s[8 * c + 1]);
-        __half2 h1 = __floats2half2_rn(s[8 * c + 2], s[8 * c + 3]);
-        __half2 h2 = __floats2half2_rn(s[8 * c + 4], s[8 * c + 5]);
-        __half2 h3 = __floats2half2_rn(s[8 * c + 6], s[8 * c + 7]);
-        v.x = *reinterpret_cast<uint32_t*>(&h0);
-        v.y = *reinterpret_cast<uint32_t*>(&h1);
-        v.z = *reinterpret_cast<uint32_t*>(&h2);
-        v.w = *reinterpret_cast<uint32_t*>(&h3);
-        my_stage[(4 * g + c) ^ (h & 7)] = v;
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          __half2 hv = __floats2half2_rn(v32[8 * c + 2 * e] * A.sm_scale_log2,
+                                         v32[8 * c + 2 * e + 1] * A.sm_scale_log2);
+          w[e] = *reinterpret_cast<uint32_t*>(&hv);
+          keep[4 * c + e] = w[e];
+        }
+        dst[(4 * g + c) ^ (h & 7)] = make_uint4(w[0], w[1], w[2], w[3]);
       }
       fence_proxy_async_smem();           // generic writes -> the bulk copy's reads
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.stage_full));
+      if (lane == 0) mbar_arrive(smem_u32(&sm.stage_full[b]));
+      return true;
+    };
+    if (ok && ntiles > 0) ok = stage_tile(0, own);
+    for (int i = 0; ok && i < ntiles; ++i) {
+      const int st = i % kStages, b = i & 1;
       // which slots of this half tile are selected (staged by the gather warp)
       if (!(ok = warp_wait(smem_u32(&sm.kv_full[st]), (i / kStages) & 1, abort_flag, err))) break;
       const unsigned valid = sm.valid[st][g];
-      // add the peer's partials, then hand x back
-      if (!(ok = warp_wait<true>(smem_u32(&sm.x_full), i & 1, abort_flag, err))) break;
+      // own + peer partials, then hand x back
+      if (!(ok = warp_wait<true>(smem_u32(&sm.x_full[b]), (i >> 1) & 1, abort_flag, err))) break;
+      float s[32];
+      {
+        const uint4* xp = sm.x[b] + h * 8;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint4 v = my_x[(4 * g + c) ^ (h & 7)];
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        for (int c = 0; c < 4; ++c) {
+          const uint4 v = xp[(4 * g + c) ^ (h & 7)];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[e]));
-          s[8 * c + 2 * e] += f.x;
-          s[8 * c + 2 * e + 1] += f.y;
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t we = e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w;
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&we));
+            const float2 o = __half22float2(*reinterpret_cast<const __half2*>(&own[4 * c + e]));
+            s[8 * c + 2 * e] = o.x + f.x;
+            s[8 * c + 2 * e + 1] = o.y + f.y;
+          }
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.x_read));
+      if (lane == 0) mbar_arrive(smem_u32(&sm.x_read[b]));
+      // the next tile's partials go out while this one is finished
+      if (i + 1 < ntiles && !(ok = stage_tile(i + 1, own))) break;
       if (valid != 0xffffffffu) {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
