@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--next", action="store_true",
+                    help="also time dense causal and sliding-window attention beside DSA at 16K")
     return ap.parse_args()
 
 
@@ -342,6 +344,51 @@ def time_decode(dsa, steps, warmup):
     return res, work, B * nq
 
 
+def time_next(dsa, steps=3, warmup=2):
+    """Dense causal and sliding-window attention on the same sparse MLA
+    kernel (index sets from dsa_window_indices) beside the whole DSA path,
+    on the 16K prefill workload."""
+    cfg = W.CONFIGS[2]
+    inp = W.make_prefill(cfg, device="cuda")
+    L, H, k, sm = inp["T"], inp["H"], inp["k"], inp["sm_scale"]
+    q, kv = inp["q"], inp["kv"]
+    out = torch.empty(L, H, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(L, H, dtype=torch.float32, device="cuda")
+    pf = Prefill(dsa, cfg, inp)
+    swa_idx = dsa.window_indices(L, L, k, k)
+    chunk = 2048        # dense rows in chunks; a chunk's rows see keys up to its last row
+    dense_idx = [dsa.window_indices(chunk, L, c0 + chunk, c0 + chunk, q_pos0=c0)
+                 for c0 in range(0, L, chunk)]
+
+    def swa():
+        dsa.sparse_mla(q, kv, swa_idx, sm, out=out, lse=lse)
+
+    def dense():
+        for c, c0 in enumerate(range(0, L, chunk)):
+            dsa.sparse_mla(q[c0:c0 + chunk], kv, dense_idx[c], sm, out=out[c0:c0 + chunk],
+                           lse=lse[c0:c0 + chunk])
+
+    res = {"workload": f"prefill L={L} (config 2), MLA {H} heads over the 512+64 latent; "
+                       f"dsa = indexer + top-{k} + sparse MLA; swa = window {k}; "
+                       f"dense_causal = every causal key, rows in chunks of {chunk} "
+                       f"(1/9 of the slots are masked, past the diagonal)"}
+    for name, fn in (("dsa", pf.step), ("swa", swa), ("dense_causal", dense)):
+        for _ in range(warmup):
+            fn()
+        e0, e1 = _ev(), _ev()
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        e1.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        res[name] = {"ms": ms, "tokens_per_s": L / (ms * 1e-3)}
+    st = dsa.get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the window runs: {dsa.STATUS.get(st, st)}")
+    return res
+
+
 # ------------------------------------------------------------ CPU oracle
 
 def oracle_sample(inp, n_rows=32, threads=None):
@@ -472,6 +519,8 @@ def main():
             "sparse_mla": {"ms": dres["sparse_mla"], "bound": "hbm", "achieved": mla_gbs,
                            "peak": pk["hbm"], "unit": "GB/s", "frac": mla_gbs / pk["hbm"]},
             "indexer_topk_ms": dres["total"] - dres["sparse_mla"]}
+    if args.next:
+        line["next"] = time_next(dsa)
     if not args.no_e2e:
         e_ms, h2d, d2h = e2e_prefill(pf, max(1, min(args.steps, 3)))
         line["e2e"] = {"value": tokens / (ranks.max(e_ms) / 1e3), "unit": "tokens/s",

@@ -141,6 +141,26 @@ int dsa_sparse_mla_fwd(const void *q, const void *kv, const int32_t *idx,
                        float *lse, dsa_stream_t stream);
 
 /*
+ * Index sets for sliding-window and dense causal attention, to run through
+ * dsa_sparse_mla_fwd in place of the top-k selection. Sliding-window
+ * attention keeps a fixed number of the keys just before each token (page 1,
+ * section "秘密武器"; page 4, section "Sparse Attention"), and DSA generalises
+ * it; a window covering the whole causal prefix is dense causal attention,
+ * the full interface page 2 (section "六、实测表现与取舍") keeps beside DSA.
+ *
+ *   row t (position p = min(q_pos0 + t, S - 1)) gets the keys
+ *   max(0, p - window + 1) .. p in increasing order, then -1 up to k.
+ *
+ *   window  1 .. k; keys per row, the query's own position included
+ *   k       row length of idx, multiple of 4
+ *   idx     [T][k] int32 out, 16-byte aligned, caller-owned
+ * Returns DSA_ERR_INVALID_ARG (nothing launched) for window > k or other bad
+ * arguments.
+ */
+int dsa_window_indices(int T, int S, int q_pos0, int window, int k, int32_t *idx,
+                       dsa_stream_t stream);
+
+/*
  * Whole prefill path: indexer -> top-k -> sparse MLA for T query rows at
  * positions q_pos0 .. q_pos0 + T - 1 against S cached keys (S >= q_pos0 + T
  * for a self-contained prefill). Query rows are scored in chunks of `chunk`

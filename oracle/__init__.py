@@ -66,6 +66,8 @@ def lib():
                                              I64, ctypes.c_double, P, I64, P, P]
             L.dsa_oracle_topk.restype = ctypes.c_int
             L.dsa_oracle_topk.argtypes = [P, I64, I64, P, ctypes.c_int, P]
+            L.dsa_oracle_window.restype = ctypes.c_int
+            L.dsa_oracle_window.argtypes = [I64, I64, I64, ctypes.c_int, ctypes.c_int, P]
             L.dsa_oracle_sparse_mla.restype = ctypes.c_int
             L.dsa_oracle_sparse_mla.argtypes = [P, P, P, I64, I64, ctypes.c_int,
                                                 ctypes.c_int, ctypes.c_double, P, I64, P, P]
@@ -141,6 +143,15 @@ def topk(I, row_len, k):
     rc = lib().dsa_oracle_topk(_ptr(I), I.shape[0], I.shape[1], _ptr(n), int(k), _ptr(out))
     if rc != 0:
         raise ValueError(f"oracle topk failed ({rc})")
+    return out
+
+
+def window(nrows, S, window, k, q_pos0=0):
+    """Sliding-window key positions [nrows][k] (increasing, -1 padded)."""
+    out = np.empty((nrows, k), np.int32)
+    rc = lib().dsa_oracle_window(int(nrows), int(S), int(q_pos0), int(window), int(k), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle window failed ({rc})")
     return out
 
 

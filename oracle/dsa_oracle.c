@@ -165,6 +165,32 @@ int dsa_oracle_topk(const float *I, int64_t nrows, int64_t ld,
 }
 
 /*
+ * Sliding-window selection, the fixed-distance rule DSA generalises
+ * ("m.gxzdkb.com/media/457.html", section "秘密武器": a token attends only to
+ * a fixed number of the keys before it; "oilbeater.com ... deepseek-sparse-
+ * attention", section "Sparse Attention"). With a window covering the whole
+ * prefix it is dense causal attention's index set.
+ *
+ *   Row r sits at position p = min(q_pos0 + r, S - 1) and takes every key s
+ *   with p - window < s <= p and s >= 0, in increasing order; the rest of
+ *   the row is -1. Requires 1 <= window <= k.
+ */
+int dsa_oracle_window(int64_t nrows, int64_t S, int64_t q_pos0, int window, int k,
+                      int32_t *idx) {
+    if (window < 1 || k < window || S < 1) return -3;
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t p = q_pos0 + r;
+        if (p > S - 1) p = S - 1;
+        int32_t *out = idx + r * k;
+        int j = 0;
+        for (int64_t s = p - window + 1; s <= p; ++s)
+            if (s >= 0) out[j++] = (int32_t)s;
+        while (j < k) out[j++] = -1;
+    }
+    return 0;
+}
+
+/*
  * Sparse MLA forward for a subset of query rows (step 4 of the workflow).
  *
  *   q    [T][H][576] bf16 bits; kv [S][576] bf16 bits (512 latent + 64 rope)

@@ -41,6 +41,7 @@ _sig("dsa_get_device_error", I32, P)
 _sig("dsa_indexer_scores", I32, P, P, P, P, P, I32, I32, I32, I32, F32, P, I64, P)
 _sig("dsa_topk", I32, P, I32, I32, I64, I32, I32, P, P)
 _sig("dsa_sparse_mla_fwd", I32, P, P, P, I32, I32, I32, I32, F32, P, P, P)
+_sig("dsa_window_indices", I32, I32, I32, I32, I32, I32, P, P)
 _sig("dsa_forward_workspace_size", SZ, I32, I32, I32, I32, I32, I32)
 _sig("dsa_forward", I32, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, F32, F32,
      P, P, P, P, SZ, P)
@@ -138,6 +139,16 @@ def indexer_scores(q8, q_scale, k8, k_scale, w, scale, q_pos0=0, scores=None, st
                                    float(scale), _p(_dev(scores, torch.float32)),
                                    scores.shape[1], _stream(stream)), "dsa_indexer_scores")
     return scores
+
+
+def window_indices(T, S, window, k, q_pos0=0, idx=None, device="cuda", stream=None):
+    """Sliding-window (or, with window >= the prefix, dense causal) index sets
+    -> int32 [T][k]: row t takes keys max(0, p - window + 1) .. p, p = q_pos0 + t."""
+    if idx is None:
+        idx = torch.empty(T, k, dtype=torch.int32, device=device)
+    _check(_lib.dsa_window_indices(T, S, q_pos0, window, k, _p(_dev(idx, torch.int32)),
+                                   _stream(stream)), "dsa_window_indices")
+    return idx
 
 
 def topk(scores, S, k, q_pos0=0, idx=None, stream=None):

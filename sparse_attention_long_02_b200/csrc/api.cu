@@ -215,6 +215,16 @@ int dsa_topk(const float* scores, int T, int S, int64_t ld, int q_pos0, int k, i
   return run_topk(scores, T, S, ld, q_pos0, nullptr, 1, k, idx, static_cast<cudaStream_t>(stream));
 }
 
+int dsa_window_indices(int T, int S, int q_pos0, int window, int k, int32_t* idx,
+                       dsa_stream_t stream) {
+  if (!idx || T < 0 || S <= 0 || q_pos0 < 0 || window < 1 || k <= 0 || (k & 3) || window > k ||
+      !aligned16(idx))
+    return DSA_ERR_INVALID_ARG;
+  if (T == 0) return DSA_OK;
+  return status_of(dsa::launch_window(T, S, q_pos0, window, k, idx,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
 static int mla_common(const void* q, const void* kv, const int32_t* idx, int T, int S, int H, int k,
                       float sm_scale, void* out, float* lse, const int32_t* block_table,
                       const int32_t* seq_len, int max_blocks, int nblk, int nq,

@@ -61,6 +61,7 @@ cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType
 cudaError_t launch_indexer(const IndexerArgs& a, const void* q8, const void* k8, long long k_rows,
                            cudaStream_t st);
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st);
+cudaError_t launch_window(int T, int S, int q_pos0, int window, int k, int* idx, cudaStream_t st);
 cudaError_t launch_sparse_mla(const MlaArgs& a, const void* q, const void* kv, long long kv_rows,
                               long long q_rows, cudaStream_t st);
 

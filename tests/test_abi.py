@@ -64,6 +64,11 @@ def test_host_validation_rejects_before_launch(dsa):
     # forward: workspace missing / too small
     assert L.dsa_forward(fake, None, fake, None, fake, fake, fake, 8, 8, 4, 8, 0, 4, 0, 1.0, 0.1,
                          None, fake, None, None, 0, None) == -3
+    # window indices: window above k, non-positive window, k not a multiple of 4
+    assert L.dsa_window_indices(4, 16, 0, 9, 8, fake, None) == -1
+    assert L.dsa_window_indices(4, 16, 0, 0, 8, fake, None) == -1
+    assert L.dsa_window_indices(4, 16, 0, 4, 6, fake, None) == -1
+    assert L.dsa_window_indices(4, 16, 0, 4, 8, None, None) == -1
     # empty problems are a no-op
     assert L.dsa_topk(fake, 0, 4, 4, 0, 4, fake, None) == 0
 

@@ -285,3 +285,32 @@ def test_topk_fast_and_general_paths(dsa, kind, n, k):
     exp = np.sort(np.where(ref < 0, np.iinfo(np.int32).max, ref), axis=1)
     exp = np.where(exp == np.iinfo(np.int32).max, -1, exp)
     assert np.array_equal(idx.cpu().numpy(), exp)
+
+
+# ------------------------------------------- sliding window / dense causal
+
+@pytest.mark.parametrize("T,S,q_pos0,window,k", [(37, 37, 0, 1, 4), (300, 300, 0, 64, 64),
+                                                 (50, 400, 333, 128, 132), (20, 100, 90, 16, 16),
+                                                 (129, 129, 0, 129, 132)])
+def test_window_indices_bit_exact(dsa, T, S, q_pos0, window, k):
+    got = dsa.window_indices(T, S, window, k, q_pos0=q_pos0)
+    no_device_error(dsa)
+    ref = oracle.window(T, S, window, k, q_pos0=q_pos0)
+    assert torch.equal(got.cpu(), torch.from_numpy(ref))
+
+
+@pytest.mark.parametrize("window,k", [(96, 96), (300, 300)])
+def test_sliding_window_and_dense_causal_mla(dsa, window, k):
+    """The sparse MLA over window index sets: sliding-window attention (a
+    window shorter than the rows) and dense causal attention (a window
+    covering every prefix), against the oracle on sampled rows."""
+    rng = np.random.default_rng(7)
+    T, H = 300, 128
+    q = torch.from_numpy(rng.normal(size=(T, H, 576))).to(torch.bfloat16)
+    kv = torch.from_numpy(rng.normal(size=(T, 576))).to(torch.bfloat16)
+    idx = dsa.window_indices(T, T, window, k)
+    out, lse = dsa.sparse_mla(q.cuda(), kv.cuda(), idx, 1 / 24)
+    no_device_error(dsa)
+    rows = [0, 1, 63, 64, 95, 96, 97, 150, 255, 299]
+    ref, ref_lse = oracle.sparse_mla(q, kv, oracle.window(T, T, window, k), 1 / 24, rows=rows)
+    assert_mla_close(out[rows], ref, lse[rows], ref_lse)

@@ -348,3 +348,50 @@ def test_decode_invariant_under_physical_block_permutation():
     d2 = oracle.decode(inp2)
     assert np.array_equal(d2["idx"], d["idx"])
     assert np.array_equal(d2["out"], d["out"])
+
+
+# ------------------------------------------- sliding window / dense causal
+
+def band_mask(T, window):
+    """Library band: key s visible from row t iff t - window < s <= t."""
+    return torch.ones(T, T, dtype=torch.bool).tril().triu(-(window - 1))
+
+
+@pytest.mark.parametrize("window,q_pos0,S", [(1, 0, 40), (7, 0, 40), (16, 5, 40), (40, 0, 40),
+                                             (9, 30, 34)])
+def test_window_is_the_band_of_a_library_mask(window, q_pos0, S):
+    nrows, k = 12, 40
+    sel = oracle.window(nrows, S, window, k, q_pos0=q_pos0)
+    band = band_mask(S, window)
+    for r in range(nrows):
+        p = min(q_pos0 + r, S - 1)                # rows past the cache clamp to its end
+        want = torch.nonzero(band[p]).flatten().numpy()
+        got = sel[r][sel[r] >= 0]
+        np.testing.assert_array_equal(got, want)
+        assert (sel[r][len(got):] == -1).all()
+
+
+def test_sliding_window_attention_is_banded_sdpa():
+    rng = np.random.default_rng(21)
+    T, H, window, k = 30, 3, 6, 8
+    q, kv = _bf16(rng, (T, H, 576)), _bf16(rng, (T, 576))
+    out, lse = oracle.sparse_mla(q, kv, oracle.window(T, T, window, k), 1 / 24)
+    qd = q.double().permute(1, 0, 2)
+    kd = kv.double().unsqueeze(0).expand(H, -1, -1)
+    vd = kv[:, :512].double().unsqueeze(0).expand(H, -1, -1)
+    mask = band_mask(T, window)
+    ref = torch.nn.functional.scaled_dot_product_attention(qd, kd, vd, attn_mask=mask,
+                                                           scale=1 / 24)
+    ref_lse = torch.logsumexp(((qd @ kd.transpose(1, 2)) / 24).masked_fill(~mask, -np.inf), -1)
+    np.testing.assert_allclose(out, ref.permute(1, 0, 2).numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse.T.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_window_covering_the_prefix_is_dense_causal_attention():
+    rng = np.random.default_rng(22)
+    T, H = 20, 2
+    q, kv = _bf16(rng, (T, H, 576)), _bf16(rng, (T, 576))
+    out, lse = oracle.sparse_mla(q, kv, oracle.window(T, T, T, 20), 1 / 24)
+    ref, ref_lse = dense_causal_sdpa(q, kv, 1 / 24)
+    np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=1e-12, atol=1e-12)
