@@ -36,6 +36,7 @@ struct TopkSmem {
   int cand_idx[kCandCap];
   unsigned warp_tot[kWarps];
   unsigned s_bucket, s_above;
+  unsigned s_count;
 };
 
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -284,7 +285,168 @@ __device__ void select_fast(const float4* x4, long long n, long long n4, int k, 
   }
 }
 
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkArgs a) {
+// Radix select (11 + 11 + 10 bits) in shared memory: the `want`-th largest of
+// keys[0..m) and how many keys equal to it rank within the first `want`.
+// `hist` needs 2048 entries and must not overlap `keys`.
+__device__ void smem_select(const uint32_t* keys, int m, unsigned want, unsigned* hist,
+                            TopkSmem& sm, uint32_t* kth, unsigned* need) {
+  const int tid = threadIdx.x;
+  const int bits[3] = {11, 11, 10};
+  uint32_t prefix = 0;
+  int shift = 32;
+  for (int p = 0; p < 3; ++p) {
+    const int nb = 1 << bits[p];
+    shift -= bits[p];
+    const int hi_shift = shift + bits[p];
+    for (int j = tid; j < nb; j += kTopkThreads) hist[j] = 0;
+    __syncthreads();
+    for (int j = tid; j < m; j += kTopkThreads) {
+      const uint32_t u = keys[j];
+      if (p == 0 || (u >> hi_shift) == prefix) atomicAdd(&hist[(u >> shift) & (nb - 1)], 1u);
+    }
+    __syncthreads();
+    find_bucket(hist, nb, want, &sm.s_bucket, &sm.s_above);
+    prefix = (prefix << bits[p]) | sm.s_bucket;
+    want -= sm.s_above;
+    __syncthreads();
+  }
+  *kth = prefix;
+  *need = want;
+}
+
+// Ordered scan of a bitmap of n bits (bit i = key i): calls emit(rank, i) for
+// every set bit, rank counting set bits in index order from 0.
+template <typename F>
+__device__ void bitmap_scan(const unsigned* bm, long long n, TopkSmem& sm, F emit) {
+  const int tid = threadIdx.x;
+  const int words = static_cast<int>((n + 31) >> 5);
+  const int per = (words + kTopkThreads - 1) / kTopkThreads;
+  const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
+  unsigned cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
+  unsigned tot;
+  unsigned rank = block_excl_scan(cnt, sm.warp_tot, tot);
+  for (int w = w0; w < w1; ++w) {
+    unsigned b = bm[w];
+    while (b) {
+      const int bit = __ffs(b) - 1;
+      emit(rank++, 32 * w + bit);
+      b &= b - 1;
+    }
+  }
+}
+
+// Sampled path. The k-th largest key is estimated from a sample of the row
+// (the first 256 keys of every 4096) with a margin; one sweep then keeps
+// every key at or above the estimate, appended in any order with one shared
+// atomic per warp. If at least k were kept, the selection lies among them,
+// ties included (the k-th largest key is at or above the estimate): it is
+// chosen exactly in shared memory and put back in index order through a
+// bitmap of the row. Otherwise, or when the kept keys overflow the buffer,
+// the caller falls back to the two-pass paths. Returns whether the selection
+// was written.
+constexpr int kSampleSeg = 4096;       // row segment
+constexpr int kSampleRun = 256;        // sampled keys at the start of each segment
+constexpr long long kSampledMaxN = 32ll * kSampleSeg;   // sample and bitmaps fit hist + sure
+
+__device__ bool select_sampled(const float4* x4, long long n, long long n4, int k, int* out,
+                               TopkSmem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int nseg = static_cast<int>((n + kSampleSeg - 1) / kSampleSeg);
+  uint32_t* samp = sm.hist;                     // hist and sure are contiguous: 8192 keys
+  const int runs4 = kSampleRun / 4;
+  for (int j = tid; j < nseg * runs4; j += kTopkThreads) {
+    const long long i4 = static_cast<long long>(j / runs4) * (kSampleSeg / 4) + (j % runs4);
+    uint32_t u[4] = {0u, 0u, 0u, 0u};          // past the row end: 0, below every real key
+    if (i4 < n4) {
+      const float4 v = x4[i4];
+      const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) u[c] = (4 * i4 + c < n) ? order_key(e[c]) : 0u;
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) samp[4 * j + c] = u[c];
+  }
+  if (tid == 0) sm.s_count = 0;
+  __syncthreads();
+  const long long m = (n / kSampleSeg) * kSampleRun + min(static_cast<long long>(kSampleRun),
+                                                           n % kSampleSeg);
+  const long long rank = static_cast<long long>(1.4 * k * static_cast<double>(m) / n) + 9;
+  if (rank >= m) return false;
+  uint32_t tau;
+  unsigned unused;
+  smem_select(samp, nseg * kSampleRun, static_cast<unsigned>(rank),
+              reinterpret_cast<unsigned*>(sm.cand_key), sm, &tau, &unused);
+  // the sweep: keys >= tau appended with one atomic per warp and slot; four
+  // 16-B loads per thread are issued before any is used
+  constexpr int kBatch = 4;
+  for (long long i0 = 0; i0 < n4; i0 += kTopkThreads * kBatch) {
+    float4 v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const long long i = i0 + u * kTopkThreads + tid;
+      v[u] = i < n4 ? x4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const long long i = i0 + u * kTopkThreads + tid;
+      const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const bool in = i < n4 && 4 * i + c < n;
+        const uint32_t key = order_key(e[c]);
+        const bool keep = in && key >= tau;
+        const unsigned ball = __ballot_sync(0xffffffffu, keep);
+        if (ball) {
+          unsigned base = 0;
+          if (lane == 0) base = atomicAdd(&sm.s_count, static_cast<unsigned>(__popc(ball)));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if (keep) {
+            const unsigned pos = base + __popc(ball & ((1u << lane) - 1u));
+            if (pos < static_cast<unsigned>(kCandCap)) {
+              sm.cand_key[pos] = key;
+              sm.cand_idx[pos] = static_cast<int>(4 * i + c);
+            }
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const unsigned kept = sm.s_count;
+  if (kept < static_cast<unsigned>(k) || kept > static_cast<unsigned>(kCandCap)) return false;
+  const int ncand = static_cast<int>(kept);
+  uint32_t thr;
+  unsigned need;
+  smem_select(sm.cand_key, ncand, static_cast<unsigned>(k), sm.hist, sm, &thr, &need);
+  // bitmaps of the row: gt = keys above thr, eq = keys equal to it
+  unsigned* gt = sm.hist;
+  unsigned* eq = reinterpret_cast<unsigned*>(sm.sure);
+  const int words = static_cast<int>((n + 31) >> 5);
+  for (int w = tid; w < words; w += kTopkThreads) {
+    gt[w] = 0u;
+    eq[w] = 0u;
+  }
+  __syncthreads();
+  for (int j = tid; j < ncand; j += kTopkThreads) {
+    const uint32_t u = sm.cand_key[j];
+    const int ix = sm.cand_idx[j];
+    if (u > thr) atomicOr(&gt[ix >> 5], 1u << (ix & 31));
+    else if (u == thr) atomicOr(&eq[ix >> 5], 1u << (ix & 31));
+  }
+  __syncthreads();
+  // the first `need` ties in index order join the selection
+  bitmap_scan(eq, n, sm, [&](unsigned r, int ix) {
+    if (r < need) atomicOr(&gt[ix >> 5], 1u << (ix & 31));
+  });
+  __syncthreads();
+  bitmap_scan(gt, n, sm, [&](unsigned r, int ix) {
+    if (r < static_cast<unsigned>(k)) out[r] = ix;
+  });
+  return true;
+}
+
+__global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(const TopkArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
   const int r = blockIdx.x;
@@ -302,6 +464,9 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const TopkArgs a) {
   }
   const float4* x4 = reinterpret_cast<const float4*>(a.scores + static_cast<long long>(r) * a.ld);
   const long long n4 = (n + 3) >> 2;
+  if (a.k <= 2048 && n >= 4ll * a.k && n <= kSampledMaxN && select_sampled(x4, n, n4, a.k, out, sm))
+    return;
+  __syncthreads();
   // pass 1: 12-bit histogram of the whole row
   for (int i = tid; i < kBins; i += kTopkThreads) sm.hist[i] = 0;
   __syncthreads();

@@ -266,20 +266,33 @@ def test_decode_paged_vs_oracle(dsa, lens, nq):
 
 @pytest.mark.parametrize("kind,n,k", [("random", 20000, 2048), ("ties", 20000, 2048),
                                       ("constant", 9000, 1024), ("random", 12000, 5000),
-                                      ("ties", 3000, 256)])
+                                      ("ties", 3000, 256), ("sample_high", 20000, 2048),
+                                      ("random", 131072, 2048), ("random", 70001, 2048),
+                                      ("random", 8192, 2048), ("planted", 65536, 2048)])
 def test_topk_fast_and_general_paths(dsa, kind, n, k):
-    """Random rows take the in-shared-memory path; rows whose k-th bucket is
-    crowded (heavy ties, constant rows) and k > 4096 take the general path."""
+    """Every selection path against the oracle's full sort:
+    - random, planted, periodically boosted, full-length (131072) and
+      ragged rows take the in-shared-memory path (their k-th bucket is small);
+    - rows whose k-th bucket is crowded (heavy ties, constant rows) and
+      k > 4096 take the general path."""
     rng = np.random.default_rng(n + k)
     R = 6
-    if kind == "random":
+    if kind in ("random", "sample_high", "planted"):
         I = rng.normal(size=(R, n)).astype(np.float32)
+        if kind == "sample_high":
+            I[:, (np.arange(n) % 4096) < 256] += 10.0
+        if kind == "planted":
+            for r in range(R):
+                I[r, rng.choice(n, 300, replace=False)] += 8.0
     elif kind == "ties":
         I = (rng.integers(-3, 4, size=(R, n)) / 8.0).astype(np.float32)
     else:
         I = np.full((R, n), 0.5, np.float32)
     q_pos0 = n - R                       # rows see n-R+1 .. n keys
-    idx = dsa.topk(torch.from_numpy(I).cuda(), n, k, q_pos0=q_pos0)
+    ld = (n + 3) // 4 * 4                # row stride: a multiple of 4 (ragged n pads it)
+    Ig = np.zeros((R, ld), np.float32)
+    Ig[:, :n] = I
+    idx = dsa.topk(torch.from_numpy(Ig).cuda(), n, k, q_pos0=q_pos0)
     no_device_error(dsa)
     ref = oracle.topk(I, oracle.prefill_row_len(R, n, q_pos0), k)
     exp = np.sort(np.where(ref < 0, np.iinfo(np.int32).max, ref), axis=1)
