@@ -81,30 +81,30 @@ __device__ __forceinline__ unsigned block_excl_scan(unsigned v, unsigned* warp_t
 }
 
 // With hist[0..nb) filled, find (from the top) the bucket where the count
-// reaches `want`; writes the bucket and the count strictly above it.
+// reaches `want`; writes the bucket and the count strictly above it. Thread t
+// sums bins [nb - (t+1)·per, nb - t·per); a block scan over those sums, taken
+// from the top, tells which thread's range holds the bucket.
 __device__ __forceinline__ void find_bucket(const unsigned* hist, int nb, unsigned want,
                                             unsigned* s_bucket, unsigned* s_above) {
-  if ((threadIdx.x >> 5) == 0) {
-    const int lane = threadIdx.x & 31;
-    const int per = nb / 32;
-    const int top = nb - 1 - lane * per;
-    unsigned local = 0;
+  __shared__ unsigned scan_tot[kWarps];
+  const int tid = threadIdx.x;
+  const int per = nb / kTopkThreads > 0 ? nb / kTopkThreads : 1;
+  const int top = nb - 1 - tid * per;            // this thread's highest bin
+  unsigned local = 0;
+  if (top >= 0)
     for (int j = 0; j < per; ++j) local += hist[top - j];
-    const unsigned incl = warp_incl_scan(local);
-    const unsigned excl = incl - local;
-    const unsigned hit = __ballot_sync(0xffffffffu, incl >= want);
-    const int first = __ffs(hit) - 1;
-    if (lane == first) {
-      unsigned cum = excl;
-      for (int j = 0; j < per; ++j) {
-        const unsigned c = hist[top - j];
-        if (cum + c >= want) {
-          *s_bucket = top - j;
-          *s_above = cum;
-          break;
-        }
-        cum += c;
+  unsigned tot;
+  const unsigned excl = block_excl_scan(local, scan_tot, tot);
+  if (top >= 0 && excl < want && excl + local >= want) {
+    unsigned cum = excl;
+    for (int j = 0; j < per; ++j) {
+      const unsigned c = hist[top - j];
+      if (cum + c >= want) {
+        *s_bucket = top - j;
+        *s_above = cum;
+        break;
       }
+      cum += c;
     }
   }
   __syncthreads();
@@ -161,6 +161,7 @@ __device__ void select_general(const float4* x4, long long n, long long n4, int 
   unsigned want = static_cast<unsigned>(k);
   const int bits[3] = {11, 11, 10};
   int shift = 32;
+#pragma unroll
   for (int p = 0; p < 3; ++p) {
     const int nb = 1 << bits[p];
     shift -= bits[p];
@@ -294,6 +295,7 @@ __device__ void smem_select(const uint32_t* keys, int m, unsigned want, unsigned
   const int bits[3] = {11, 11, 10};
   uint32_t prefix = 0;
   int shift = 32;
+#pragma unroll
   for (int p = 0; p < 3; ++p) {
     const int nb = 1 << bits[p];
     shift -= bits[p];
@@ -354,18 +356,26 @@ __device__ bool select_sampled(const float4* x4, long long n, long long n4, int 
   const int tid = threadIdx.x, lane = tid & 31;
   const int nseg = static_cast<int>((n + kSampleSeg - 1) / kSampleSeg);
   uint32_t* samp = sm.hist;                     // hist and sure are contiguous: 8192 keys
+  // all of a thread's sample loads are issued before any is used
   const int runs4 = kSampleRun / 4;
-  for (int j = tid; j < nseg * runs4; j += kTopkThreads) {
+  constexpr int kIters = (static_cast<int>(kSampledMaxN / kSampleSeg) * kSampleRun / 4) /
+                         kTopkThreads;
+  float4 sv[kIters];
+#pragma unroll
+  for (int it = 0; it < kIters; ++it) {
+    const int j = tid + it * kTopkThreads;
     const long long i4 = static_cast<long long>(j / runs4) * (kSampleSeg / 4) + (j % runs4);
-    uint32_t u[4] = {0u, 0u, 0u, 0u};          // past the row end: 0, below every real key
-    if (i4 < n4) {
-      const float4 v = x4[i4];
-      const float e[4] = {v.x, v.y, v.z, v.w};
+    sv[it] = (j < nseg * runs4 && i4 < n4) ? x4[i4] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 #pragma unroll
-      for (int c = 0; c < 4; ++c) u[c] = (4 * i4 + c < n) ? order_key(e[c]) : 0u;
-    }
+  for (int it = 0; it < kIters; ++it) {
+    const int j = tid + it * kTopkThreads;
+    if (j >= nseg * runs4) break;
+    const long long i4 = static_cast<long long>(j / runs4) * (kSampleSeg / 4) + (j % runs4);
+    const float e[4] = {sv[it].x, sv[it].y, sv[it].z, sv[it].w};
 #pragma unroll
-    for (int c = 0; c < 4; ++c) samp[4 * j + c] = u[c];
+    for (int c = 0; c < 4; ++c)           // past the row end: 0, below every real key
+      samp[4 * j + c] = (4 * i4 + c < n) ? order_key(e[c]) : 0u;
   }
   if (tid == 0) sm.s_count = 0;
   __syncthreads();
