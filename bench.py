@@ -174,6 +174,12 @@ def decode_work(lens, nq, Hi, H, k):
                 mla_flops=mla_flops, sel=sel)
 
 
+# DRAM bytes (read + write) per launch of the current kernels at the full 128K prefill, from
+# one-pass ncu captures (dram__bytes_read.sum + dram__bytes_write.sum): the sparse MLA's one
+# launch, and the mean of the indexer's 32 chunk launches. Reset to None when a kernel changes.
+NCU_TRAFFIC = {"sparse_mla": 62.05e9 + 17.24e9, "indexer": 0.2993e9 + 1.0210e9}
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -495,7 +501,8 @@ def main():
     launches_per_step = {"indexer": math.ceil(L / pf.chunk), "sparse_mla": 1}[dom]
     roof = {"kernel": dom, "bound": "tensor", "achieved": stages[dom]["achieved"],
             "peak": stages[dom]["peak"], "unit": "TFLOP/s", "frac": stages[dom]["frac"],
-            "traffic": None, "launches_per_step": launches_per_step,
+            "traffic": NCU_TRAFFIC.get(dom), "traffic_unit": "bytes per launch",
+            "launches_per_step": launches_per_step,
             "peak_src": f"{pk['src']} sustained bf16" + (" x2 (FP8/BF16 nominal ratio)"
                                                          if dom == "indexer" else "")}
     t_roof = max(work["idx_flops"] / (fp8_sus * 1e12), work["idx_bytes"] / (pk["hbm"] * 1e9)) + \
