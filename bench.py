@@ -59,19 +59,28 @@ def parse():
 # ------------------------------------------------------------------ ranks
 
 class Ranks:
-    def __init__(self, gpus):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE). The only
+    collectives are the timing barrier and the max of the per-rank times; the
+    problems themselves are independent. `backend` "gloo" keeps everything on
+    the CPU (tests without GPUs)."""
+
+    def __init__(self, gpus, backend="nccl"):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.dev = "cuda" if backend == "nccl" else "cpu"
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                    device_id=torch.device("cuda", self.local))
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+                dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                        device_id=torch.device("cuda", self.local))
+            else:
+                dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
             self.pg = dist
-        elif torch.cuda.is_available():
+        elif backend == "nccl" and torch.cuda.is_available():
             torch.cuda.set_device(0)
         self.gpus = gpus
 
@@ -82,7 +91,7 @@ class Ranks:
     def max(self, x: float) -> float:
         if not self.pg:
             return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        t = torch.tensor([x], dtype=torch.float64, device=self.dev)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
