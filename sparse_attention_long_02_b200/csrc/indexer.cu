@@ -311,7 +311,10 @@ int indexer_queries_per_cta(int Hi) {
   return qb < 64 ? qb : 64;
 }
 
-static int indexer_tiles_per_cta() { return 64; }
+// Key tiles per CTA: prefill rows are long, so units of 128 tiles (16384 keys)
+// amortise each CTA's setup; decode keeps 64 so that B = 64 sequences still
+// spread over every SM.
+static int indexer_tiles_per_cta(bool paged) { return paged ? 64 : 128; }
 
 cudaError_t launch_indexer(const IndexerArgs& a_in, const void* q8, const void* k8,
                            long long k_rows, cudaStream_t st) {
@@ -324,7 +327,7 @@ cudaError_t launch_indexer(const IndexerArgs& a_in, const void* q8, const void* 
   a.n_mma = n;
   a.q_box_rows = n;
   a.tmem_cols = 2 * n <= 32 ? 32 : 2 * n <= 64 ? 64 : 2 * n <= 128 ? 128 : 2 * n <= 256 ? 256 : 512;
-  a.tiles_per_cta = indexer_tiles_per_cta();
+  a.tiles_per_cta = indexer_tiles_per_cta(paged);
 
   CUtensorMap tq, tk;
   const long long q_rows = paged ? static_cast<long long>(a.B) * a.nq * a.Hi

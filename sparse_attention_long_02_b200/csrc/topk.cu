@@ -286,17 +286,21 @@ __device__ void select_fast(const float4* x4, long long n, long long n4, int k, 
   }
 }
 
-// Radix select (11 + 11 + 10 bits) in shared memory: the `want`-th largest of
-// keys[0..m) and how many keys equal to it rank within the first `want`.
-// `hist` needs 2048 entries and must not overlap `keys`.
+// Radix select in shared memory over keys[0..m). With kPasses = 3 (11 + 11 +
+// 10 bits) it returns the `want`-th largest key and how many keys equal to it
+// rank within the first `want`. With kPasses = 2 (12 + 10 bits) it returns
+// the lower edge of the 22-bit bucket that holds the `want`-th largest key: a
+// threshold at or below it, at least `want` keys at or above it. `hist` needs
+// 2048 (3 passes) or 4096 (2 passes) entries and must not overlap `keys`.
+template <int kPasses>
 __device__ void smem_select(const uint32_t* keys, int m, unsigned want, unsigned* hist,
                             TopkSmem& sm, uint32_t* kth, unsigned* need) {
   const int tid = threadIdx.x;
-  const int bits[3] = {11, 11, 10};
+  const int bits[3] = {kPasses == 3 ? 11 : 12, kPasses == 3 ? 11 : 10, 10};
   uint32_t prefix = 0;
   int shift = 32;
 #pragma unroll
-  for (int p = 0; p < 3; ++p) {
+  for (int p = 0; p < kPasses; ++p) {
     const int nb = 1 << bits[p];
     shift -= bits[p];
     const int hi_shift = shift + bits[p];
@@ -312,7 +316,7 @@ __device__ void smem_select(const uint32_t* keys, int m, unsigned want, unsigned
     want -= sm.s_above;
     __syncthreads();
   }
-  *kth = prefix;
+  *kth = prefix << shift;
   *need = want;
 }
 
@@ -385,8 +389,8 @@ __device__ bool select_sampled(const float4* x4, long long n, long long n4, int 
   if (rank >= m) return false;
   uint32_t tau;
   unsigned unused;
-  smem_select(samp, nseg * kSampleRun, static_cast<unsigned>(rank),
-              reinterpret_cast<unsigned*>(sm.cand_key), sm, &tau, &unused);
+  smem_select<2>(samp, nseg * kSampleRun, static_cast<unsigned>(rank),
+                 reinterpret_cast<unsigned*>(sm.cand_key), sm, &tau, &unused);
   // the sweep: keys >= tau appended with one atomic per warp and slot; four
   // 16-B loads per thread are issued before any is used
   constexpr int kBatch = 4;
@@ -428,7 +432,7 @@ __device__ bool select_sampled(const float4* x4, long long n, long long n4, int 
   const int ncand = static_cast<int>(kept);
   uint32_t thr;
   unsigned need;
-  smem_select(sm.cand_key, ncand, static_cast<unsigned>(k), sm.hist, sm, &thr, &need);
+  smem_select<3>(sm.cand_key, ncand, static_cast<unsigned>(k), sm.hist, sm, &thr, &need);
   // bitmaps of the row: gt = keys above thr, eq = keys equal to it
   unsigned* gt = sm.hist;
   unsigned* eq = reinterpret_cast<unsigned*>(sm.sure);
