@@ -401,7 +401,39 @@ def time_next(dsa, steps=3, warmup=2):
     st = dsa.get_device_error()
     if st != 0:
         raise RuntimeError(f"device error in the window runs: {dsa.STATUS.get(st, st)}")
+    res["projection"] = time_projection(dsa, steps, warmup)
     return res
+
+
+def time_projection(dsa, steps, warmup, T=4096, d=4096, Hi=64):
+    """Step 1 of the workflow (hidden states -> FP8 indexer inputs) for one 4096-token
+    chunk; the width d is not given by the pages."""
+    inp = W.make_projection(T, d, Hi, seed=5, device="cuda")
+    ws = torch.empty(dsa.lib().dsa_project_workspace_size(T, Hi), dtype=torch.uint8,
+                     device="cuda")
+
+    def run():
+        dsa.project_indexer_inputs(inp["h"], inp["wt"], inp["rope"], Hi, workspace=ws)
+
+    for _ in range(warmup):
+        run()
+    e0, e1 = _ev(), _ev()
+    e0.record()
+    for _ in range(steps):
+        run()
+    e1.record()
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    st = dsa.get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the projection: {dsa.STATUS.get(st, st)}")
+    flops = 2.0 * T * d * (Hi * 128 + 128 + Hi)
+    tf = flops / (ms * 1e-3) / 1e12
+    pk = peaks()
+    return {"workload": f"T={T} tokens, d={d}, Hi={Hi}: GEMM to {Hi * 128 + 128 + Hi} outputs, "
+                        "rotary on q and k, per-token FP8", "ms": ms,
+            "tokens_per_s": T / (ms * 1e-3), "achieved": tf, "unit": "TFLOP/s",
+            "peak": pk["bf16_sus"], "frac": tf / pk["bf16_sus"]}
 
 
 # ------------------------------------------------------------ CPU oracle

@@ -141,6 +141,36 @@ int dsa_sparse_mla_fwd(const void *q, const void *kv, const int32_t *idx,
                        float *lse, dsa_stream_t stream);
 
 /*
+ * Step 1 of the workflow (page 3, section 4 "步骤一：查询与键的投影"; page 5,
+ * section "第一步"): the hidden states are projected to the indexer's queries
+ * and keys, rotary position encoding is applied to both, and each indexer
+ * head gets a weight a_h, a linear map of the same hidden state. The outputs
+ * are the FP8 inputs dsa_indexer_scores takes.
+ *
+ *   h       [T][d] bf16 hidden states, d a multiple of 8
+ *   wt      [Hi*128 + 128 + Hi][d] bf16: the rows of W_Q (Hi heads x 128),
+ *           then W_K (128), then W_a (Hi), each row one output's weights
+ *   rope    [T][64][2] fp32 (cos, sin) of each token's position for the 64
+ *           dimension pairs (2i, 2i+1) of a 128-wide head; pair i of q (every
+ *           head) and of k becomes (y0 cos - y1 sin, y0 sin + y1 cos)
+ *   q8      [T][Hi][128] e4m3 out, q_scale [T] fp32 out
+ *   k8      [T][128] e4m3 out, k_scale [T] fp32 out
+ *   a       [T][Hi] fp32 out (a_h, not scaled)
+ *   Scales are per token, over all of its q (or k) values: scale = amax / 448
+ *   (1 when amax = 0); codes are e4m3(y / scale), rounded to nearest even and
+ *   saturated at +-448.
+ *   workspace  >= dsa_project_workspace_size(T, Hi) bytes, 16-byte aligned,
+ *              caller-owned (fp32 rotated q and k, per-token maxima)
+ * Hi in {1, 2, 4, ..., 64}; the library has no counterpart for the widths,
+ * which the pages leave open.
+ */
+size_t dsa_project_workspace_size(int T, int Hi);
+int dsa_project_indexer_inputs(const void *h, const void *wt, const float *rope, int T,
+                               int d, int Hi, void *q8, float *q_scale, void *k8,
+                               float *k_scale, float *a, void *workspace, size_t ws_bytes,
+                               dsa_stream_t stream);
+
+/*
  * Index sets for sliding-window and dense causal attention, to run through
  * dsa_sparse_mla_fwd in place of the top-k selection. Sliding-window
  * attention keeps a fixed number of the keys just before each token (page 1,

@@ -67,6 +67,8 @@ def lib():
             L.dsa_oracle_topk.restype = ctypes.c_int
             L.dsa_oracle_topk.argtypes = [P, I64, I64, P, ctypes.c_int, P]
             L.dsa_oracle_window.restype = ctypes.c_int
+            L.dsa_oracle_project.restype = ctypes.c_int
+            L.dsa_oracle_project.argtypes = [P, P, P, I64, I64, ctypes.c_int, P, I64, P]
             L.dsa_oracle_window.argtypes = [I64, I64, I64, ctypes.c_int, ctypes.c_int, P]
             L.dsa_oracle_sparse_mla.restype = ctypes.c_int
             L.dsa_oracle_sparse_mla.argtypes = [P, P, P, I64, I64, ctypes.c_int,
@@ -143,6 +145,24 @@ def topk(I, row_len, k):
     rc = lib().dsa_oracle_topk(_ptr(I), I.shape[0], I.shape[1], _ptr(n), int(k), _ptr(out))
     if rc != 0:
         raise ValueError(f"oracle topk failed ({rc})")
+    return out
+
+
+def project(h, wt, rope, Hi, rows=None):
+    """Projection of hidden states h [T][d] (bf16) through wt [N][d] (bf16) with
+    the rotation table rope [T][64][2] -> float64 [nrows][N]: rotated q heads,
+    rotated k, then a_h (before any FP8 encoding)."""
+    hb = _np(h, np.uint16)
+    wb = _np(wt, np.uint16)
+    rp = np.ascontiguousarray(_np(rope, np.float32))
+    T, d = hb.shape
+    r = _rows(rows, T)
+    N = Hi * 128 + 128 + Hi
+    out = np.empty((len(r), N), np.float64)
+    rc = lib().dsa_oracle_project(_ptr(hb), _ptr(wb), _ptr(rp), T, d, int(Hi), _ptr(r), len(r),
+                                  _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle project failed ({rc})")
     return out
 
 

@@ -165,6 +165,46 @@ int dsa_oracle_topk(const float *I, int64_t nrows, int64_t ld,
 }
 
 /*
+ * Projection to the indexer inputs (step 1 of the workflow: "DeepSeek-V3.2-
+ * Exp 模型优势与 DSA 工作原理", section 4 "步骤一：查询与键的投影"): queries
+ * Q = H W_Q and keys K = H W_K with rotary position encoding, and per-head
+ * weights a_h, a linear map of H.
+ *
+ *   h    [T][d] bf16 bits, wt [N][d] bf16 bits with N = Hi*128 + 128 + Hi:
+ *        the rows of W_Q (Hi heads x 128), then W_K (128), then W_a (Hi)
+ *   rope [T][64][2] (cos, sin) per token and dimension pair
+ *   For each selected row t: y[n] = sum_j h[t][j] * wt[n][j] in double; then
+ *   every (2i, 2i+1) pair of a q head and of k becomes
+ *   (y0 cos_i - y1 sin_i, y0 sin_i + y1 cos_i) with token t's table entry i.
+ *   out [nrows][N] double.
+ */
+int dsa_oracle_project(const uint16_t *h, const uint16_t *wt, const float *rope, int64_t T,
+                       int64_t d, int Hi, const int64_t *rows, int64_t nrows, double *out) {
+    if (Hi < 1 || d < 1) return -3;
+    const int64_t N = (int64_t)Hi * 128 + 128 + Hi;
+    const int64_t nqk = (int64_t)Hi * 128 + 128;
+    for (int64_t r = 0; r < nrows; ++r) {
+        const int64_t t = rows[r];
+        if (t < 0 || t >= T) return -2;
+        double *y = out + r * N;
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < d; ++j)
+                acc += dsa_oracle_bf16(h[t * d + j]) * dsa_oracle_bf16(wt[n * d + j]);
+            y[n] = acc;
+        }
+        for (int64_t n = 0; n < nqk; n += 2) {
+            const int64_t i = (n % 128) / 2;
+            const double c = rope[(t * 64 + i) * 2], sn = rope[(t * 64 + i) * 2 + 1];
+            const double y0 = y[n], y1 = y[n + 1];
+            y[n] = y0 * c - y1 * sn;
+            y[n + 1] = y0 * sn + y1 * c;
+        }
+    }
+    return 0;
+}
+
+/*
  * Sliding-window selection, the fixed-distance rule DSA generalises
  * ("m.gxzdkb.com/media/457.html", section "秘密武器": a token attends only to
  * a fixed number of the keys before it; "oilbeater.com ... deepseek-sparse-

@@ -42,6 +42,8 @@ _sig("dsa_indexer_scores", I32, P, P, P, P, P, I32, I32, I32, I32, F32, P, I64, 
 _sig("dsa_topk", I32, P, I32, I32, I64, I32, I32, P, P)
 _sig("dsa_sparse_mla_fwd", I32, P, P, P, I32, I32, I32, I32, F32, P, P, P)
 _sig("dsa_window_indices", I32, I32, I32, I32, I32, I32, P, P)
+_sig("dsa_project_workspace_size", SZ, I32, I32)
+_sig("dsa_project_indexer_inputs", I32, P, P, P, I32, I32, I32, P, P, P, P, P, P, SZ, P)
 _sig("dsa_forward_workspace_size", SZ, I32, I32, I32, I32, I32, I32)
 _sig("dsa_forward", I32, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, F32, F32,
      P, P, P, P, SZ, P)
@@ -139,6 +141,31 @@ def indexer_scores(q8, q_scale, k8, k_scale, w, scale, q_pos0=0, scores=None, st
                                    float(scale), _p(_dev(scores, torch.float32)),
                                    scores.shape[1], _stream(stream)), "dsa_indexer_scores")
     return scores
+
+
+def project_indexer_inputs(h, wt, rope, Hi, workspace=None, stream=None):
+    """Hidden states -> FP8 indexer inputs: (q8 u8 [T][Hi][128], q_scale [T],
+    k8 u8 [T][128], k_scale [T], a f32 [T][Hi]); ``wt`` holds the rows of W_Q,
+    W_K and W_a ([Hi*128 + 128 + Hi][d] bf16), ``rope`` the (cos, sin) table
+    [T][64][2]."""
+    h = _dev(h, torch.bfloat16)
+    wt = _dev(wt, torch.bfloat16)
+    rope = _dev(rope, torch.float32)
+    T, d = h.shape
+    dev = h.device
+    q8 = torch.empty(T, Hi, 128, dtype=torch.uint8, device=dev)
+    k8 = torch.empty(T, 128, dtype=torch.uint8, device=dev)
+    q_scale = torch.empty(T, dtype=torch.float32, device=dev)
+    k_scale = torch.empty(T, dtype=torch.float32, device=dev)
+    a = torch.empty(T, Hi, dtype=torch.float32, device=dev)
+    need = _lib.dsa_project_workspace_size(T, Hi)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check(_lib.dsa_project_indexer_inputs(_p(h), _p(wt), _p(rope), T, d, Hi, _p(q8), _p(q_scale),
+                                           _p(k8), _p(k_scale), _p(a), _p(workspace),
+                                           workspace.numel(), _stream(stream)),
+           "dsa_project_indexer_inputs")
+    return q8, q_scale, k8, k_scale, a
 
 
 def window_indices(T, S, window, k, q_pos0=0, idx=None, device="cuda", stream=None):

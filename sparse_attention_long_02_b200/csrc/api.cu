@@ -215,6 +215,46 @@ int dsa_topk(const float* scores, int T, int S, int64_t ld, int q_pos0, int k, i
   return run_topk(scores, T, S, ld, q_pos0, nullptr, 1, k, idx, static_cast<cudaStream_t>(stream));
 }
 
+size_t dsa_project_workspace_size(int T, int Hi) {
+  if (T <= 0 || !valid_hi(Hi)) return 0;
+  return round_up(static_cast<size_t>(T) * (Hi * 128 + 128) * 4, 256) +
+         2 * round_up(static_cast<size_t>(T) * 4, 256);
+}
+
+int dsa_project_indexer_inputs(const void* h, const void* wt, const float* rope, int T, int d,
+                               int Hi, void* q8, float* q_scale, void* k8, float* k_scale, float* a,
+                               void* workspace, size_t ws_bytes, dsa_stream_t stream) {
+  if (!h || !wt || !rope || !q8 || !q_scale || !k8 || !k_scale || !a || T < 0 || d < 8 ||
+      (d & 7) || !aligned16(h) || !aligned16(wt) || !aligned16(rope) || !aligned16(q8) ||
+      !aligned16(k8) || !aligned16(a))
+    return DSA_ERR_INVALID_ARG;
+  if (!valid_hi(Hi)) return DSA_ERR_UNSUPPORTED;
+  if (T == 0) return DSA_OK;
+  const size_t need = dsa_project_workspace_size(T, Hi);
+  if (!workspace || !aligned16(workspace) || ws_bytes < need) return DSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProjArgs P;
+  P.T = T;
+  P.d = d;
+  P.Hi = Hi;
+  P.N = Hi * 128 + 128 + Hi;
+  P.rope = rope;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  P.y = reinterpret_cast<float*>(ws);
+  const size_t ybytes = round_up(static_cast<size_t>(T) * (Hi * 128 + 128) * 4, 256);
+  P.amax_q = reinterpret_cast<unsigned*>(ws + ybytes);
+  P.amax_k = reinterpret_cast<unsigned*>(ws + ybytes + round_up(static_cast<size_t>(T) * 4, 256));
+  P.a = a;
+  P.q8 = static_cast<uint8_t*>(q8);
+  P.k8 = static_cast<uint8_t*>(k8);
+  P.q_scale = q_scale;
+  P.k_scale = k_scale;
+  P.err = device_error_word();
+  cudaError_t e = cudaMemsetAsync(ws + ybytes, 0, 2 * round_up(static_cast<size_t>(T) * 4, 256), st);
+  if (e == cudaSuccess) e = launch_project(P, h, wt, st);
+  return status_of(e);
+}
+
 int dsa_window_indices(int T, int S, int q_pos0, int window, int k, int32_t* idx,
                        dsa_stream_t stream) {
   if (!idx || T < 0 || S <= 0 || q_pos0 < 0 || window < 1 || k <= 0 || (k & 3) || window > k ||

@@ -39,6 +39,20 @@ struct TopkArgs {
   unsigned* err = nullptr;
 };
 
+struct ProjArgs {
+  int T = 0, d = 0, Hi = 0, N = 0;        // tokens, hidden width, indexer heads, outputs
+  const float* rope = nullptr;            // [T][64] (cos, sin) pairs
+  float* y = nullptr;                     // workspace [T][Hi*128 + 128] fp32, rotated q | k
+  unsigned* amax_q = nullptr;             // workspace [T], |y| maximum as float bits
+  unsigned* amax_k = nullptr;
+  float* a = nullptr;                     // [T][Hi] per-head weights out
+  uint8_t* q8 = nullptr;                  // [T][Hi][128] e4m3 out
+  uint8_t* k8 = nullptr;                  // [T][128] e4m3 out
+  float* q_scale = nullptr;               // [T] out
+  float* k_scale = nullptr;               // [T] out
+  unsigned* err = nullptr;
+};
+
 struct MlaArgs {
   int T = 0, S = 0, H = 0, k = 0;         // query rows, keys (contiguous), heads, slots per row
   float sm_scale_log2 = 0.f;              // sm_scale * log2(e)
@@ -62,6 +76,7 @@ cudaError_t launch_indexer(const IndexerArgs& a, const void* q8, const void* k8,
                            cudaStream_t st);
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st);
 cudaError_t launch_window(int T, int S, int q_pos0, int window, int k, int* idx, cudaStream_t st);
+cudaError_t launch_project(const ProjArgs& a, const void* h, const void* wt, cudaStream_t st);
 cudaError_t launch_sparse_mla(const MlaArgs& a, const void* q, const void* kv, long long kv_rows,
                               long long q_rows, cudaStream_t st);
 

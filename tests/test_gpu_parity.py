@@ -327,3 +327,29 @@ def test_sliding_window_and_dense_causal_mla(dsa, window, k):
     rows = [0, 1, 63, 64, 95, 96, 97, 150, 255, 299]
     ref, ref_lse = oracle.sparse_mla(q, kv, oracle.window(T, T, window, k), 1 / 24, rows=rows)
     assert_mla_close(out[rows], ref, lse[rows], ref_lse)
+
+
+# ------------------------------------------------ projection (workflow step 1)
+
+@pytest.mark.parametrize("T,d,Hi", [(300, 200, 64), (129, 64, 4), (5, 8, 1)])
+def test_projection_vs_oracle(dsa, T, d, Hi):
+    """The GEMM + rotation against the float64 oracle; the FP8 encoding of the
+    kernel's own fp32 values against torch's e4m3 cast (same precision, so the
+    codes and scales must be identical)."""
+    inp = W.make_projection(T, d, Hi, seed=T + d + Hi)
+    need = dsa.lib().dsa_project_workspace_size(T, Hi)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    q8, q_scale, k8, k_scale, a = dsa.project_indexer_inputs(
+        inp["h"].cuda(), inp["wt"].cuda(), inp["rope"].cuda(), Hi, workspace=ws)
+    no_device_error(dsa)
+    nq, nqk = Hi * 128, Hi * 128 + 128
+    y = ws[: T * nqk * 4].view(torch.float32).view(T, nqk).cpu()      # rotated q | k, fp32
+    ref = oracle.project(inp["h"], inp["wt"], inp["rope"], Hi)
+    np.testing.assert_allclose(y.double().numpy(), ref[:, :nqk], rtol=1e-4, atol=1e-4)
+    np.testing.assert_allclose(a.cpu().double().numpy(), ref[:, nqk:], rtol=1e-4, atol=1e-4)
+    for part, codes, scale in ((y[:, :nq], q8.view(T, nq), q_scale), (y[:, nq:], k8, k_scale)):
+        amax = part.abs().amax(dim=1)
+        s = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+        assert torch.equal(scale.cpu(), s)
+        want = (part / s.unsqueeze(1)).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+        assert torch.equal(codes.cpu(), want)

@@ -395,3 +395,35 @@ def test_window_covering_the_prefix_is_dense_causal_attention():
     ref, ref_lse = dense_causal_sdpa(q, kv, 1 / 24)
     np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(lse, ref_lse, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------ projection (workflow step 1)
+
+def test_projection_with_identity_rotation_is_a_matmul():
+    inp = W.make_projection(20, 48, 2, seed=31)
+    ident = torch.zeros(20, 64, 2)
+    ident[..., 0] = 1.0
+    y = oracle.project(inp["h"], inp["wt"], ident, 2)
+    ref = (inp["h"].double() @ inp["wt"].double().T).numpy()
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_projection_rotation_is_complex_multiplication():
+    """Pair (2i, 2i+1) of every q head and of k is multiplied, as a complex
+    number, by cos + i sin of the table entry i; a_h is not rotated."""
+    Hi, T = 3, 9
+    inp = W.make_projection(T, 40, Hi, seed=32)
+    rng = np.random.default_rng(33)
+    ang = rng.uniform(-np.pi, np.pi, size=(T, 64))
+    table = torch.from_numpy(np.stack([np.cos(ang), np.sin(ang)], -1)).float()
+    rows = [8, 0, 5]
+    y = oracle.project(inp["h"], inp["wt"], table, Hi, rows=rows)
+    plain = (inp["h"].double() @ inp["wt"].double().T).numpy()[rows]
+    nqk = Hi * 128 + 128
+    z = plain[:, :nqk:2] + 1j * plain[:, 1:nqk:2]                # [rows][pairs]
+    tab = table.double().numpy()[rows]
+    rot = np.tile(tab[..., 0] + 1j * tab[..., 1], (1, nqk // 128))
+    zr = z * rot
+    np.testing.assert_allclose(y[:, :nqk:2], zr.real, rtol=1e-9, atol=1e-9)
+    np.testing.assert_allclose(y[:, 1:nqk:2], zr.imag, rtol=1e-9, atol=1e-9)
+    np.testing.assert_allclose(y[:, nqk:], plain[:, nqk:], rtol=1e-12, atol=1e-12)

@@ -217,3 +217,24 @@ def make_decode(cfg: Config, device="cpu", B: int | None = None,
                 block_table=table.to(device), seq_len=lens.to(device),
                 scale=cfg.scale, sm_scale=cfg.sm_scale, k=cfg.k, nq=nq, B=B,
                 max_blocks=max_blocks, nblk=nblk, Hi=Hi, H=H)
+
+
+def rope_table(T: int, q_pos0: int = 0, base: float = 10000.0, device="cpu") -> torch.Tensor:
+    """(cos, sin) of the rotary angles for positions q_pos0 .. q_pos0 + T - 1 and the
+    64 dimension pairs of a 128-wide head: [T][64][2] float32, angle (p * base^(-i/64)
+    for pair i), evaluated in float64. The projection kernel and the oracle both
+    take it as input data."""
+    pos = torch.arange(q_pos0, q_pos0 + T, dtype=torch.float64).unsqueeze(1)
+    inv = base ** (-torch.arange(64, dtype=torch.float64) / 64.0)
+    ang = pos * inv.unsqueeze(0)
+    return torch.stack([ang.cos(), ang.sin()], dim=-1).float().contiguous().to(device)
+
+
+def make_projection(T: int, d: int, Hi: int, seed: int, device="cpu"):
+    """Hidden states h ~ N(0, 1) [T][d] and weights [Hi*128 + 128 + Hi][d] ~ N(0, 1/d),
+    both bf16 (so each output is about N(0, 1)), plus the rotary table of positions 0..T-1."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    N = Hi * D_INDEX + D_INDEX + Hi
+    h = _normal((T, d), g, device, torch.bfloat16)
+    wt = (torch.randn(N, d, generator=g, device=device) / math.sqrt(d)).to(torch.bfloat16)
+    return dict(h=h, wt=wt, rope=rope_table(T, device=device), T=T, d=d, Hi=Hi)
