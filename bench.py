@@ -402,6 +402,53 @@ def time_next(dsa, steps=3, warmup=2):
     if st != 0:
         raise RuntimeError(f"device error in the window runs: {dsa.STATUS.get(st, st)}")
     res["projection"] = time_projection(dsa, steps, warmup)
+    res["warmup_objective"] = time_warmup(dsa, steps, warmup)
+    return res
+
+
+def time_warmup(dsa, steps, warmup, L=2048):
+    """The indexer's warm-up objective on one L-token prefill: the
+    head-mean dense attention target (lse from the sparse MLA over dense index sets),
+    the KL with its gradient on the indexer scores, and the backward to q, k, w."""
+    cfg = W.Config(93, "warmup", "prefill", k=L, Hi=64, H=128, seed=6, L=L)
+    inp = W.make_prefill(cfg, device="cuda")
+    idx = dsa.window_indices(L, L, L, L)
+    out = torch.empty(L, inp["H"], 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(L, inp["H"], dtype=torch.float32, device="cuda")
+    ws = torch.empty(dsa.lib().dsa_attention_probs_workspace_size(L, L, inp["H"]),
+                     dtype=torch.uint8, device="cuda")
+    state = {}
+
+    def target():
+        dsa.sparse_mla(inp["q"], inp["kv"], idx, inp["sm_scale"], out=out, lse=lse)
+        state["p"] = dsa.attention_probs_mean(inp["q"], inp["kv"], lse, inp["sm_scale"],
+                                              workspace=ws)
+
+    def kl():
+        I = dsa.indexer_scores(inp["q8"], inp["q_scale"], inp["k8"], inp["k_scale"], inp["w"],
+                               inp["scale"])
+        state["loss"], state["grad"] = dsa.indexer_kl(I, state["p"], L)
+
+    def backward():
+        dsa.indexer_backward(inp["q8"], inp["q_scale"], inp["k8"], inp["k_scale"], inp["w"],
+                             inp["scale"], state["grad"])
+
+    res = {"workload": f"prefill L={L}, 128 MLA heads, 64 indexer heads: target (dense MLA "
+                       "for lse + head-mean weights), KL + gradient, backward to q, k, w"}
+    for name, fn in (("target", target), ("kl", kl), ("backward", backward)):
+        for _ in range(warmup):
+            fn()
+        e0, e1 = _ev(), _ev()
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        e1.synchronize()
+        res[name] = {"ms": e0.elapsed_time(e1) / steps}
+    st = dsa.get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the warm-up objective: {dsa.STATUS.get(st, st)}")
+    res["loss_mean"] = float(state["loss"].mean())
     return res
 
 

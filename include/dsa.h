@@ -171,6 +171,46 @@ int dsa_project_indexer_inputs(const void *h, const void *wt, const float *rope,
                                dsa_stream_t stream);
 
 /*
+ * The indexer's warm-up objective (page 2, section "四、训练的两步走冷启动"):
+ * dense attention is run, the weight distribution each token receives is the
+ * target, and the indexer alone is trained to fit it with a KL divergence.
+ * The target of query t is read as the dense causal attention distribution
+ * averaged over heads; the indexer's distribution is softmax(I[t, s]) over
+ * the same keys. Row t sits at position q_pos0 + t and sees keys 0 .. that
+ * position (clamped to S - 1). fp32 throughout.
+ *
+ * dsa_attention_probs_mean:
+ *   p[t][s] = (1/H) sum_h exp(sm_scale q[t,h] . kv[s] - lse[t][h]), 0 past the
+ *   row's keys; q [T][H][576] bf16, kv [S][576] bf16, lse [T][H] the natural
+ *   log normaliser of each head, as dsa_sparse_mla_fwd returns it over index
+ *   sets covering every causal key (dsa_window_indices with window >= S);
+ *   p [T][ldp] fp32 out. The logits q . kv go through a tensor-core GEMM into
+ *   the caller's workspace of dsa_attention_probs_workspace_size(T, S, H)
+ *   bytes (T * H rows of S fp32, S rounded up to 4).
+ * dsa_indexer_kl:
+ *   loss[t] = sum_s p[t][s] (log p[t][s] - log r[t][s]), r = softmax(I[t, :]);
+ *   grad[t][s] = r[t][s] - p[t][s] (dloss/dI), 0 past the row's keys.
+ *   I [T][ldi], p [T][ldp], grad [T][ldg] fp32; loss [T] fp32.
+ * dsa_indexer_backward:
+ *   through I = sum_h w * ReLU(scale * qf . kf) with qf = q8 * q_scale and
+ *   kf = k8 * k_scale (the FP8 inputs dsa_indexer_scores takes), given
+ *   grad = dloss/dI [T][ldg]: dq [T][Hi][128] (w.r.t. qf), dk [S][128]
+ *   (w.r.t. kf), dw [T][Hi], all fp32, caller-owned.
+ * Each returns DSA_ERR_INVALID_ARG (nothing launched) on bad arguments and
+ * DSA_ERR_UNSUPPORTED for an indexer head count outside {1, 2, 4, ..., 64}.
+ */
+size_t dsa_attention_probs_workspace_size(int T, int S, int H);
+int dsa_attention_probs_mean(const void *q, const void *kv, const float *lse, int T, int S,
+                             int H, int q_pos0, float sm_scale, float *p, int64_t ldp,
+                             void *workspace, size_t ws_bytes, dsa_stream_t stream);
+int dsa_indexer_kl(const float *I, int64_t ldi, const float *p, int64_t ldp, int T, int S,
+                   int q_pos0, float *loss, float *grad, int64_t ldg, dsa_stream_t stream);
+int dsa_indexer_backward(const void *q8, const float *q_scale, const void *k8,
+                         const float *k_scale, const float *w, int T, int S, int Hi,
+                         int q_pos0, float scale, const float *grad, int64_t ldg, float *dq,
+                         float *dk, float *dw, dsa_stream_t stream);
+
+/*
  * Index sets for sliding-window and dense causal attention, to run through
  * dsa_sparse_mla_fwd in place of the top-k selection. Sliding-window
  * attention keeps a fixed number of the keys just before each token (page 1,

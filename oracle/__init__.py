@@ -68,6 +68,14 @@ def lib():
             L.dsa_oracle_topk.argtypes = [P, I64, I64, P, ctypes.c_int, P]
             L.dsa_oracle_window.restype = ctypes.c_int
             L.dsa_oracle_project.restype = ctypes.c_int
+            L.dsa_oracle_attn_probs.restype = ctypes.c_int
+            L.dsa_oracle_attn_probs.argtypes = [P, P, I64, I64, ctypes.c_int, I64, ctypes.c_double,
+                                                P, I64, P]
+            L.dsa_oracle_indexer_kl.restype = ctypes.c_int
+            L.dsa_oracle_indexer_kl.argtypes = [P, P, I64, I64, P, P, P]
+            L.dsa_oracle_indexer_backward.restype = ctypes.c_int
+            L.dsa_oracle_indexer_backward.argtypes = [P, P, P, P, P, I64, I64, ctypes.c_int, I64,
+                                                      ctypes.c_double, P, P, P, P]
             L.dsa_oracle_project.argtypes = [P, P, P, I64, I64, ctypes.c_int, P, I64, P]
             L.dsa_oracle_window.argtypes = [I64, I64, I64, ctypes.c_int, ctypes.c_int, P]
             L.dsa_oracle_sparse_mla.restype = ctypes.c_int
@@ -164,6 +172,59 @@ def project(h, wt, rope, Hi, rows=None):
     if rc != 0:
         raise ValueError(f"oracle project failed ({rc})")
     return out
+
+
+def attention_probs(q, kv, sm_scale, q_pos0=0, rows=None):
+    """Warm-up target: head-mean dense causal attention weights -> float64 [nrows][S]."""
+    qb = _np(q, np.uint16)
+    kvb = _np(kv, np.uint16)
+    T, H = qb.shape[0], qb.shape[1]
+    S = kvb.shape[0]
+    r = _rows(rows, T)
+    out = np.empty((len(r), S), np.float64)
+    rc = lib().dsa_oracle_attn_probs(_ptr(qb), _ptr(kvb), T, S, H, int(q_pos0), float(sm_scale),
+                                     _ptr(r), len(r), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle attn_probs failed ({rc})")
+    return out
+
+
+def indexer_kl(I, p, row_len):
+    """KL(p || softmax(I)) per row and its gradient r - p (float64)."""
+    Id = np.ascontiguousarray(I, np.float64)
+    pd = np.ascontiguousarray(p, np.float64)
+    n = np.ascontiguousarray(row_len, np.int64)
+    loss = np.empty(Id.shape[0], np.float64)
+    grad = np.empty_like(Id)
+    rc = lib().dsa_oracle_indexer_kl(_ptr(Id), _ptr(pd), Id.shape[0], Id.shape[1], _ptr(n),
+                                     _ptr(loss), _ptr(grad))
+    if rc != 0:
+        raise ValueError(f"oracle indexer_kl failed ({rc})")
+    return loss, grad
+
+
+def indexer_backward(q8, q_scale, k8, k_scale, w, scale, grad, q_pos0=0):
+    """(dq [T][Hi][128], dk [S][128], dw [T][Hi]) float64: gradients of the warm-up
+    loss w.r.t. the dequantised indexer inputs, given grad = dloss/dI [T][S]."""
+    q8 = _np(q8, np.uint8)
+    k8 = _np(k8, np.uint8)
+    qs = None if q_scale is None else np.ascontiguousarray(_np(q_scale, np.float32))
+    ks = None if k_scale is None else np.ascontiguousarray(_np(k_scale, np.float32))
+    w = np.ascontiguousarray(_np(w, np.float32))
+    T, Hi = q8.shape[0], q8.shape[1]
+    S = k8.shape[0]
+    g = np.ascontiguousarray(grad, np.float64)[:, :S]
+    g = np.ascontiguousarray(g)
+    dq = np.empty((T, Hi, 128), np.float64)
+    dk = np.empty((S, 128), np.float64)
+    dw = np.empty((T, Hi), np.float64)
+    rc = lib().dsa_oracle_indexer_backward(_ptr(q8), None if qs is None else _ptr(qs), _ptr(k8),
+                                           None if ks is None else _ptr(ks), _ptr(w), T, S, Hi,
+                                           int(q_pos0), float(scale), _ptr(g), _ptr(dq),
+                                           _ptr(dk), _ptr(dw))
+    if rc != 0:
+        raise ValueError(f"oracle indexer_backward failed ({rc})")
+    return dq, dk, dw
 
 
 def window(nrows, S, window, k, q_pos0=0):

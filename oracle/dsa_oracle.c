@@ -205,6 +205,129 @@ int dsa_oracle_project(const uint16_t *h, const uint16_t *wt, const float *rope,
 }
 
 /*
+ * The indexer's warm-up objective ("ele-yufo.com/posts/deepseek-v3-2-exp",
+ * section "四、训练的两步走冷启动"): dense attention gives each token's weight
+ * distribution as the target, and the indexer is fitted to it by a KL
+ * divergence. Row t sits at position q_pos0 + t and sees keys 0 .. min(that,
+ * S - 1).
+ *
+ * dsa_oracle_attn_probs: out[r][s] = (1/H) sum_h softmax_s(sm_scale q[t,h].kv[s])
+ *   over the row's keys, 0 past them. q [T][H][576], kv [S][576] bf16 bits;
+ *   out [nrows][S] double.
+ */
+int dsa_oracle_attn_probs(const uint16_t *q, const uint16_t *kv, int64_t T, int64_t S, int H,
+                          int64_t q_pos0, double sm_scale, const int64_t *rows, int64_t nrows,
+                          double *out) {
+    if (S < 1 || H < 1) return -3;
+    double *z = (double *)malloc(sizeof(double) * (size_t)S);
+    if (!z) return -1;
+    for (int64_t r = 0; r < nrows; ++r) {
+        const int64_t t = rows[r];
+        if (t < 0 || t >= T) { free(z); return -2; }
+        int64_t pos = q_pos0 + t;
+        if (pos > S - 1) pos = S - 1;
+        double *o = out + r * S;
+        for (int64_t s = 0; s < S; ++s) o[s] = 0.0;
+        for (int h = 0; h < H; ++h) {
+            const uint16_t *qr = q + ((int64_t)t * H + h) * 576;
+            double m = -INFINITY;
+            for (int64_t s = 0; s <= pos; ++s) {
+                double acc = 0.0;
+                for (int d = 0; d < 576; ++d)
+                    acc += dsa_oracle_bf16(qr[d]) * dsa_oracle_bf16(kv[s * 576 + d]);
+                z[s] = sm_scale * acc;
+                if (z[s] > m) m = z[s];
+            }
+            double sum = 0.0;
+            for (int64_t s = 0; s <= pos; ++s) sum += exp(z[s] - m);
+            for (int64_t s = 0; s <= pos; ++s) o[s] += exp(z[s] - m) / sum / H;
+        }
+    }
+    free(z);
+    return 0;
+}
+
+/*
+ * dsa_oracle_indexer_kl: for each row (n = row_len[r] keys), r_s = softmax(I)_s,
+ *   loss[r] = sum_{s: p_s > 0} p_s (log p_s - log r_s), grad[r][s] = r_s - p_s
+ *   (0 for s >= n). I, p, grad [nrows][ld] double.
+ */
+int dsa_oracle_indexer_kl(const double *I, const double *p, int64_t nrows, int64_t ld,
+                          const int64_t *row_len, double *loss, double *grad) {
+    for (int64_t r = 0; r < nrows; ++r) {
+        const int64_t n = row_len[r];
+        if (n < 1 || n > ld) return -2;
+        const double *ir = I + r * ld, *pr = p + r * ld;
+        double m = -INFINITY;
+        for (int64_t s = 0; s < n; ++s) if (ir[s] > m) m = ir[s];
+        double z = 0.0;
+        for (int64_t s = 0; s < n; ++s) z += exp(ir[s] - m);
+        const double logz = m + log(z);
+        double kl = 0.0;
+        for (int64_t s = 0; s < ld; ++s) {
+            double g = 0.0;
+            if (s < n) {
+                const double lr = ir[s] - logz;
+                if (pr[s] > 0.0) kl += pr[s] * (log(pr[s]) - lr);
+                g = exp(lr) - pr[s];
+            }
+            grad[r * ld + s] = g;
+        }
+        loss[r] = kl;
+    }
+    return 0;
+}
+
+/*
+ * dsa_oracle_indexer_backward: gradients through I[t,s] = sum_h w[t,h] *
+ * ReLU(scale * x[t,h,s]), x = qf[t,h] . kf[s], qf = e4m3(q8) * q_scale[t],
+ * kf = e4m3(k8) * k_scale[s], given grad[t][s] = dloss/dI over each row's keys
+ * (the ReLU's decision [x > 0] is taken on the exact raw product e4m3(q8) .
+ * e4m3(k8), which has the sign of x since the scales are positive):
+ *   dq[t][h][:] = sum_s grad * w[t,h] * scale * [x > 0] * kf[s][:]
+ *   dk[s][:]    = sum_{t,h} grad * w[t,h] * scale * [x > 0] * qf[t][h][:]
+ *   dw[t][h]    = sum_s grad * ReLU(scale * x)
+ * grad [T][S] double; dq [T][Hi][128], dk [S][128], dw [T][Hi] double out.
+ */
+int dsa_oracle_indexer_backward(const uint8_t *q8, const float *q_scale, const uint8_t *k8,
+                                const float *k_scale, const float *w, int64_t T, int64_t S,
+                                int Hi, int64_t q_pos0, double scale, const double *grad,
+                                double *dq, double *dk, double *dw) {
+    for (int64_t i = 0; i < T * Hi * 128; ++i) dq[i] = 0.0;
+    for (int64_t i = 0; i < S * 128; ++i) dk[i] = 0.0;
+    for (int64_t i = 0; i < T * Hi; ++i) dw[i] = 0.0;
+    double qf[128], kf[128];
+    for (int64_t t = 0; t < T; ++t) {
+        int64_t pos = q_pos0 + t;
+        if (pos > S - 1) pos = S - 1;
+        const double qs = q_scale ? q_scale[t] : 1.0;
+        for (int h = 0; h < Hi; ++h) {
+            for (int d = 0; d < 128; ++d)
+                qf[d] = dsa_oracle_e4m3(q8[(t * Hi + h) * 128 + d]) * qs;
+            for (int64_t s = 0; s <= pos; ++s) {
+                const double ks = k_scale ? k_scale[s] : 1.0;
+                double xr = 0.0;               /* raw e4m3 dot product: exact in double */
+                for (int d = 0; d < 128; ++d) {
+                    kf[d] = dsa_oracle_e4m3(k8[s * 128 + d]) * ks;
+                    xr += dsa_oracle_e4m3(q8[(t * Hi + h) * 128 + d]) * dsa_oracle_e4m3(k8[s * 128 + d]);
+                }
+                const double x = qs * ks * xr;
+                const double g = grad[t * S + s];
+                if (xr > 0.0) {
+                    const double c = g * w[t * Hi + h] * scale;
+                    for (int d = 0; d < 128; ++d) {
+                        dq[(t * Hi + h) * 128 + d] += c * kf[d];
+                        dk[s * 128 + d] += c * qf[d];
+                    }
+                    dw[t * Hi + h] += g * scale * x;
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+/*
  * Sliding-window selection, the fixed-distance rule DSA generalises
  * ("m.gxzdkb.com/media/457.html", section "秘密武器": a token attends only to
  * a fixed number of the keys before it; "oilbeater.com ... deepseek-sparse-

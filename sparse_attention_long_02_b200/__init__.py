@@ -43,6 +43,10 @@ _sig("dsa_topk", I32, P, I32, I32, I64, I32, I32, P, P)
 _sig("dsa_sparse_mla_fwd", I32, P, P, P, I32, I32, I32, I32, F32, P, P, P)
 _sig("dsa_window_indices", I32, I32, I32, I32, I32, I32, P, P)
 _sig("dsa_project_workspace_size", SZ, I32, I32)
+_sig("dsa_attention_probs_workspace_size", SZ, I32, I32, I32)
+_sig("dsa_attention_probs_mean", I32, P, P, P, I32, I32, I32, I32, F32, P, I64, P, SZ, P)
+_sig("dsa_indexer_kl", I32, P, I64, P, I64, I32, I32, I32, P, P, I64, P)
+_sig("dsa_indexer_backward", I32, P, P, P, P, P, I32, I32, I32, I32, F32, P, I64, P, P, P, P)
 _sig("dsa_project_indexer_inputs", I32, P, P, P, I32, I32, I32, P, P, P, P, P, P, SZ, P)
 _sig("dsa_forward_workspace_size", SZ, I32, I32, I32, I32, I32, I32)
 _sig("dsa_forward", I32, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, F32, F32,
@@ -166,6 +170,52 @@ def project_indexer_inputs(h, wt, rope, Hi, workspace=None, stream=None):
                                            workspace.numel(), _stream(stream)),
            "dsa_project_indexer_inputs")
     return q8, q_scale, k8, k_scale, a
+
+
+def attention_probs_mean(q, kv, lse, sm_scale, q_pos0=0, workspace=None, stream=None):
+    """Head-mean dense causal attention weights -> float32 [T][S] (the warm-up target)."""
+    q, kv = _dev(q, torch.bfloat16), _dev(kv, torch.bfloat16)
+    lse = _dev(lse, torch.float32)
+    T, H = q.shape[0], q.shape[1]
+    S = kv.shape[0]
+    p = torch.empty(T, S, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        need = _lib.dsa_attention_probs_workspace_size(T, S, H)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(_lib.dsa_attention_probs_mean(_p(q), _p(kv), _p(lse), T, S, H, q_pos0,
+                                         float(sm_scale), _p(p), S, _p(workspace),
+                                         workspace.numel(), _stream(stream)),
+           "dsa_attention_probs_mean")
+    return p
+
+
+def indexer_kl(I, p, S, q_pos0=0, stream=None):
+    """KL(p || softmax(I)) per row -> (loss [T], grad [T][ld] = dloss/dI)."""
+    I, p = _dev(I, torch.float32), _dev(p, torch.float32)
+    T = I.shape[0]
+    loss = torch.empty(T, dtype=torch.float32, device=I.device)
+    grad = torch.empty(T, I.shape[1], dtype=torch.float32, device=I.device)
+    _check(_lib.dsa_indexer_kl(_p(I), I.shape[1], _p(p), p.shape[1], T, S, q_pos0, _p(loss),
+                               _p(grad), grad.shape[1], _stream(stream)), "dsa_indexer_kl")
+    return loss, grad
+
+
+def indexer_backward(q8, q_scale, k8, k_scale, w, scale, grad, q_pos0=0, stream=None):
+    """Gradients of the warm-up loss w.r.t. the dequantised indexer inputs ->
+    (dq [T][Hi][128], dk [S][128], dw [T][Hi]) in float32."""
+    q8, k8 = _u8(q8), _u8(k8)
+    w, grad = _dev(w, torch.float32), _dev(grad, torch.float32)
+    T, Hi = q8.shape[0], q8.shape[1]
+    S = k8.shape[0]
+    dev = q8.device
+    dq = torch.empty(T, Hi, 128, dtype=torch.float32, device=dev)
+    dk = torch.empty(S, 128, dtype=torch.float32, device=dev)
+    dw = torch.empty(T, Hi, dtype=torch.float32, device=dev)
+    _check(_lib.dsa_indexer_backward(_p(q8), _p(_dev(q_scale, torch.float32)), _p(k8),
+                                     _p(_dev(k_scale, torch.float32)), _p(w), T, S, Hi, q_pos0,
+                                     float(scale), _p(grad), grad.shape[1], _p(dq), _p(dk),
+                                     _p(dw), _stream(stream)), "dsa_indexer_backward")
+    return dq, dk, dw
 
 
 def window_indices(T, S, window, k, q_pos0=0, idx=None, device="cuda", stream=None):

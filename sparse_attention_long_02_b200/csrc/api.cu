@@ -255,6 +255,65 @@ int dsa_project_indexer_inputs(const void* h, const void* wt, const float* rope,
   return status_of(e);
 }
 
+size_t dsa_attention_probs_workspace_size(int T, int S, int H) {
+  if (T <= 0 || S <= 0 || H < 1) return 0;
+  return static_cast<size_t>(T) * H * round_up(static_cast<size_t>(S), 4) * 4;
+}
+
+int dsa_attention_probs_mean(const void* q, const void* kv, const float* lse, int T, int S,
+                             int H, int q_pos0, float sm_scale, float* p, int64_t ldp,
+                             void* workspace, size_t ws_bytes, dsa_stream_t stream) {
+  if (!q || !kv || !lse || !p || T < 0 || S <= 0 || q_pos0 < 0 || H < 1 || H > 128 ||
+      ldp < S || !(sm_scale > 0.f) || !aligned16(q) || !aligned16(kv) ||
+      static_cast<long long>(T) * H > (1ll << 30))
+    return DSA_ERR_INVALID_ARG;
+  if (T == 0) return DSA_OK;
+  const size_t need = dsa_attention_probs_workspace_size(T, S, H);
+  if (!workspace || !aligned16(workspace) || ws_bytes < need) return DSA_ERR_WORKSPACE;
+  return status_of(launch_attention_probs(q, kv, lse, T, S, H, q_pos0, sm_scale, p, ldp,
+                                          static_cast<float*>(workspace),
+                                          static_cast<long long>(round_up(S, 4)),
+                                          device_error_word(), static_cast<cudaStream_t>(stream)));
+}
+
+int dsa_indexer_kl(const float* I, int64_t ldi, const float* p, int64_t ldp, int T, int S,
+                   int q_pos0, float* loss, float* grad, int64_t ldg, dsa_stream_t stream) {
+  if (!I || !p || !loss || !grad || T < 0 || S <= 0 || q_pos0 < 0 || ldi < S || ldp < S ||
+      ldg < S)
+    return DSA_ERR_INVALID_ARG;
+  if (T == 0) return DSA_OK;
+  return status_of(launch_indexer_kl(I, ldi, p, ldp, T, S, q_pos0, loss, grad, ldg,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+int dsa_indexer_backward(const void* q8, const float* q_scale, const void* k8, const float* k_scale,
+                         const float* w, int T, int S, int Hi, int q_pos0, float scale,
+                         const float* grad, int64_t ldg, float* dq, float* dk, float* dw,
+                         dsa_stream_t stream) {
+  if (!q8 || !k8 || !w || !grad || !dq || !dk || !dw || T < 0 || S <= 0 || q_pos0 < 0 ||
+      ldg < S || !(scale > 0.f))
+    return DSA_ERR_INVALID_ARG;
+  if (!valid_hi(Hi)) return DSA_ERR_UNSUPPORTED;
+  if (T == 0) return DSA_OK;
+  IndexerBwdArgs a;
+  a.T = T;
+  a.S = S;
+  a.Hi = Hi;
+  a.q_pos0 = q_pos0;
+  a.scale = scale;
+  a.q8 = static_cast<const uint8_t*>(q8);
+  a.q_scale = q_scale;
+  a.k8 = static_cast<const uint8_t*>(k8);
+  a.k_scale = k_scale;
+  a.w = w;
+  a.grad = grad;
+  a.ldg = ldg;
+  a.dq = dq;
+  a.dk = dk;
+  a.dw = dw;
+  return status_of(launch_indexer_backward(a, static_cast<cudaStream_t>(stream)));
+}
+
 int dsa_window_indices(int T, int S, int q_pos0, int window, int k, int32_t* idx,
                        dsa_stream_t stream) {
   if (!idx || T < 0 || S <= 0 || q_pos0 < 0 || window < 1 || k <= 0 || (k & 3) || window > k ||

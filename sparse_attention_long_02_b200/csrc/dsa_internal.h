@@ -43,6 +43,7 @@ struct ProjArgs {
   int T = 0, d = 0, Hi = 0, N = 0;        // tokens, hidden width, indexer heads, outputs
   const float* rope = nullptr;            // [T][64] (cos, sin) pairs
   float* y = nullptr;                     // workspace [T][Hi*128 + 128] fp32, rotated q | k
+  long long ldy = 0;                      // row stride of y in the plain GEMM
   unsigned* amax_q = nullptr;             // workspace [T], |y| maximum as float bits
   unsigned* amax_k = nullptr;
   float* a = nullptr;                     // [T][Hi] per-head weights out
@@ -51,6 +52,21 @@ struct ProjArgs {
   float* q_scale = nullptr;               // [T] out
   float* k_scale = nullptr;               // [T] out
   unsigned* err = nullptr;
+};
+
+struct IndexerBwdArgs {
+  int T = 0, S = 0, Hi = 0, q_pos0 = 0;
+  float scale = 1.f;
+  const uint8_t* q8 = nullptr;            // [T][Hi][128] e4m3
+  const float* q_scale = nullptr;         // [T] or null
+  const uint8_t* k8 = nullptr;            // [S][128] e4m3
+  const float* k_scale = nullptr;         // [S] or null
+  const float* w = nullptr;               // [T][Hi]
+  const float* grad = nullptr;            // [T][ldg] dL/dI
+  long long ldg = 0;
+  float* dq = nullptr;                    // [T][Hi][128] out
+  float* dk = nullptr;                    // [S][128] out
+  float* dw = nullptr;                    // [T][Hi] out
 };
 
 struct MlaArgs {
@@ -77,6 +93,16 @@ cudaError_t launch_indexer(const IndexerArgs& a, const void* q8, const void* k8,
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st);
 cudaError_t launch_window(int T, int S, int q_pos0, int window, int k, int* idx, cudaStream_t st);
 cudaError_t launch_project(const ProjArgs& a, const void* h, const void* wt, cudaStream_t st);
+// C [M][ldc] fp32 = A [M][K] x B [N][K]^T, bf16 operands, K a multiple of 8.
+cudaError_t launch_gemm_f32(const void* a, const void* b, float* c, int M, int N, int K,
+                            long long ldc, unsigned* err, cudaStream_t st);
+cudaError_t launch_attention_probs(const void* q, const void* kv, const float* lse, int T, int S,
+                                   int H, int q_pos0, float sm_scale, float* p, long long ldp,
+                                   float* z, long long ldz, unsigned* err, cudaStream_t st);
+cudaError_t launch_indexer_kl(const float* I, long long ldi, const float* p, long long ldp, int T,
+                              int S, int q_pos0, float* loss, float* grad, long long ldg,
+                              cudaStream_t st);
+cudaError_t launch_indexer_backward(const IndexerBwdArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_mla(const MlaArgs& a, const void* q, const void* kv, long long kv_rows,
                               long long q_rows, cudaStream_t st);
 

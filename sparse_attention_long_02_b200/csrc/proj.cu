@@ -15,6 +15,9 @@
 // token's |y| maximum (one atomic per tile and part), and writes a_h.
 // Kernel 2 quantises q and k per token: scale = amax / 448 (1 if amax = 0),
 // code = e4m3(y / scale), rounded to nearest even and saturated at +-448.
+//
+// The same GEMM with a plain epilogue (every output written in fp32) serves
+// the attention logits of the indexer's warm-up target.
 #include "common.cuh"
 #include "dsa_internal.h"
 #include <cuda_fp8.h>
@@ -37,6 +40,7 @@ struct ProjSmem {
   int abort_flag;
 };
 
+template <bool kPlain>
 __global__ void __launch_bounds__(kProjThreads, 1)
 proj_gemm_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w,
                  const ProjArgs P) {
@@ -118,6 +122,13 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant
         float y[32];
         tmem_ld32(tmem + lane_base + 32 * c, y);
         if (t >= P.T || col0 >= P.N) continue;
+        if constexpr (kPlain) {
+          float* dst = P.y + t * P.ldy + col0;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (col0 + j < P.N) dst[j] = y[j];
+          continue;
+        }
         if (col0 < nqk) {
           // q or k columns: rotate the 16 pairs of this chunk by the token's table
           const float2* cs = reinterpret_cast<const float2*>(P.rope) + t * 64 + (col0 % 128) / 2;
@@ -144,8 +155,8 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant
         }
       }
       // bit patterns of non-negative floats order like the floats
-      if (t < P.T && amax_q > 0.f) atomicMax(P.amax_q + t, __float_as_uint(amax_q));
-      if (t < P.T && amax_k > 0.f) atomicMax(P.amax_k + t, __float_as_uint(amax_k));
+      if (!kPlain && t < P.T && amax_q > 0.f) atomicMax(P.amax_q + t, __float_as_uint(amax_q));
+      if (!kPlain && t < P.T && amax_k > 0.f) atomicMax(P.amax_k + t, __float_as_uint(amax_k));
     }
   }
   tc_fence_before();
@@ -190,7 +201,8 @@ __global__ void __launch_bounds__(256) proj_quant_kernel(const ProjArgs P) {
 
 }  // namespace
 
-cudaError_t launch_project(const ProjArgs& a, const void* h, const void* wt, cudaStream_t st) {
+template <bool kPlain>
+cudaError_t launch_gemm(const ProjArgs& a, const void* h, const void* wt, cudaStream_t st) {
   CUtensorMap th, tw;
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   cudaError_t e = make_tmap_2d(&th, h, bf, a.d, a.T, static_cast<uint64_t>(a.d) * 2, kBK, kBM,
@@ -200,15 +212,31 @@ cudaError_t launch_project(const ProjArgs& a, const void* h, const void* wt, cud
                      CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(ProjSmem) + 1024;
-  e = cudaFuncSetAttribute(proj_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(proj_gemm_kernel<kPlain>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   dim3 grid((a.N + kBN - 1) / kBN, (a.T + kBM - 1) / kBM);
-  proj_gemm_kernel<<<grid, kProjThreads, smem, st>>>(th, tw, a);
-  e = cudaGetLastError();
+  proj_gemm_kernel<kPlain><<<grid, kProjThreads, smem, st>>>(th, tw, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_project(const ProjArgs& a, const void* h, const void* wt, cudaStream_t st) {
+  cudaError_t e = launch_gemm<false>(a, h, wt, st);
   if (e != cudaSuccess) return e;
   proj_quant_kernel<<<a.T, 256, 0, st>>>(a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_f32(const void* a, const void* b, float* c, int M, int N, int K,
+                            long long ldc, unsigned* err, cudaStream_t st) {
+  ProjArgs P;
+  P.T = M;
+  P.N = N;
+  P.d = K;
+  P.y = c;
+  P.ldy = ldc;
+  P.err = err;
+  return launch_gemm<true>(P, a, b, st);
 }
 
 }  // namespace dsa

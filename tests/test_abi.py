@@ -69,6 +69,13 @@ def test_host_validation_rejects_before_launch(dsa):
     assert L.dsa_window_indices(4, 16, 0, 0, 8, fake, None) == -1
     assert L.dsa_window_indices(4, 16, 0, 4, 6, fake, None) == -1
     assert L.dsa_window_indices(4, 16, 0, 4, 8, None, None) == -1
+    # warm-up target: logits workspace missing / too small; ldp below S
+    assert L.dsa_attention_probs_mean(fake, fake, fake, 4, 8, 2, 0, ctypes.c_float(0.1), fake, 8,
+                                      None, 0, None) == -3
+    assert L.dsa_attention_probs_mean(fake, fake, fake, 4, 8, 2, 0, ctypes.c_float(0.1), fake, 8,
+                                      fake, 4 * 2 * 8 * 4 - 1, None) == -3
+    assert L.dsa_attention_probs_mean(fake, fake, fake, 4, 8, 2, 0, ctypes.c_float(0.1), fake, 7,
+                                      fake, 1 << 20, None) == -1
     # empty problems are a no-op
     assert L.dsa_topk(fake, 0, 4, 4, 0, 4, fake, None) == 0
 
@@ -84,3 +91,6 @@ def test_workspace_sizes(dsa):
     assert L.dsa_decode_paged_workspace_size(64, 1, 512, 64, 128, 2048) == \
         64 * 512 * 64 * 4 + 64 * 2048 * 4
     assert L.dsa_forward_workspace_size(0, 8, 4, 8, 4, 0) == 0
+    # warm-up target: T * H rows of fp32 logits, S rounded up to 4
+    assert L.dsa_attention_probs_workspace_size(2048, 2048, 128) == 2048 * 128 * 2048 * 4
+    assert L.dsa_attention_probs_workspace_size(3, 10, 2) == 3 * 2 * 12 * 4

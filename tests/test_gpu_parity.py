@@ -353,3 +353,74 @@ def test_projection_vs_oracle(dsa, T, d, Hi):
         assert torch.equal(scale.cpu(), s)
         want = (part / s.unsqueeze(1)).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
         assert torch.equal(codes.cpu(), want)
+
+
+# ------------------------------------------------- indexer warm-up objective
+
+def test_warmup_target_kl_and_backward(dsa):
+    """The warm-up objective end to end on one small prefill:
+    - target: per-head lse from the sparse MLA over dense window indices, then
+      the head-mean attention weights;
+    - KL and its gradient on the indexer scores;
+    - backward to the dequantised indexer inputs.
+    Each is checked against the oracle on the GPU's own inputs."""
+    rng = np.random.default_rng(51)
+    T, H, Hi, scale = 150, 8, 4, 1 / 16
+    q = torch.from_numpy(rng.normal(size=(T, H, 576))).to(torch.bfloat16)
+    kv = torch.from_numpy(rng.normal(size=(T, 576))).to(torch.bfloat16)
+    k = (T + 3) // 4 * 4
+    idx = dsa.window_indices(T, T, T, k)
+    _, lse = dsa.sparse_mla(q.cuda(), kv.cuda(), idx, 1 / 24)
+    p = dsa.attention_probs_mean(q.cuda(), kv.cuda(), lse, 1 / 24)
+    no_device_error(dsa)
+    p_ref = oracle.attention_probs(q, kv, 1 / 24)
+    # the MLA's lse carries its fp16-exchange rounding (<= 2e-3): p inherits it relatively
+    np.testing.assert_allclose(p.cpu().numpy(), p_ref, rtol=5e-3, atol=1e-7)
+    # KL on indexer scores from FP8 inputs
+    q8 = torch.from_numpy(rng.integers(-8, 9, size=(T, Hi, 128))).float().to(
+        torch.float8_e4m3fn).view(torch.uint8)
+    k8 = torch.from_numpy(rng.integers(-8, 9, size=(T, 128))).float().to(
+        torch.float8_e4m3fn).view(torch.uint8)
+    q_scale = torch.from_numpy(rng.uniform(0.01, 0.02, T)).float()
+    k_scale = torch.from_numpy(rng.uniform(0.01, 0.02, T)).float()
+    w = torch.from_numpy(rng.normal(size=(T, Hi)) / 8).float()
+    I = dsa.indexer_scores(q8.cuda(), q_scale.cuda(), k8.cuda(), k_scale.cuda(), w.cuda(), scale)
+    p_used = p.cpu().double().numpy()
+    loss, grad = dsa.indexer_kl(I, p, T)
+    no_device_error(dsa)
+    n = np.arange(1, T + 1)
+    I_h = I.cpu().double().numpy()[:, :T]
+    I_h = np.where(np.isfinite(I_h), I_h, 0.0)
+    l_ref, g_ref = oracle.indexer_kl(I_h, p_used, n)
+    np.testing.assert_allclose(loss.cpu().numpy(), l_ref, rtol=1e-4, atol=1e-6)
+    np.testing.assert_allclose(grad.cpu().numpy()[:, :T], g_ref, rtol=1e-4, atol=1e-6)
+    # backward on the GPU's own gradient
+    dq, dk, dw = dsa.indexer_backward(q8.cuda(), q_scale.cuda(), k8.cuda(), k_scale.cuda(),
+                                      w.cuda(), scale, grad)
+    no_device_error(dsa)
+    dq_r, dk_r, dw_r = oracle.indexer_backward(q8, q_scale, k8, k_scale, w, scale,
+                                               grad.cpu().double().numpy())
+    for got, ref in ((dq, dq_r), (dk, dk_r), (dw, dw_r)):
+        mag = np.abs(ref).max()
+        np.testing.assert_allclose(got.cpu().double().numpy(), ref, rtol=0, atol=1e-4 * mag)
+
+
+@pytest.mark.parametrize("T,S,q_pos0,Hi", [(37, 300, 263, 64), (64, 64, 0, 1)])
+def test_warmup_backward_offset_rows(dsa, T, S, q_pos0, Hi):
+    """Backward for a chunk of rows at an offset (keys 0 .. q_pos0 + t) and for one head."""
+    rng = np.random.default_rng(T + S + Hi)
+    q8 = torch.from_numpy(rng.integers(-8, 9, size=(T, Hi, 128))).float().to(
+        torch.float8_e4m3fn).view(torch.uint8)
+    k8 = torch.from_numpy(rng.integers(-8, 9, size=(S, 128))).float().to(
+        torch.float8_e4m3fn).view(torch.uint8)
+    w = torch.from_numpy(rng.normal(size=(T, Hi))).float()
+    ld = (S + 3) // 4 * 4
+    g = torch.from_numpy(rng.normal(size=(T, ld))).float()
+    dq, dk, dw = dsa.indexer_backward(q8.cuda(), None, k8.cuda(), None, w.cuda(), 0.5, g.cuda(),
+                                      q_pos0=q_pos0)
+    no_device_error(dsa)
+    dq_r, dk_r, dw_r = oracle.indexer_backward(q8, None, k8, None, w, 0.5, g.double().numpy(),
+                                               q_pos0=q_pos0)
+    for got, ref in ((dq, dq_r), (dk, dk_r), (dw, dw_r)):
+        mag = np.abs(ref).max()
+        np.testing.assert_allclose(got.cpu().double().numpy(), ref, rtol=0, atol=1e-5 * mag)

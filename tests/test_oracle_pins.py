@@ -427,3 +427,96 @@ def test_projection_rotation_is_complex_multiplication():
     np.testing.assert_allclose(y[:, :nqk:2], zr.real, rtol=1e-9, atol=1e-9)
     np.testing.assert_allclose(y[:, 1:nqk:2], zr.imag, rtol=1e-9, atol=1e-9)
     np.testing.assert_allclose(y[:, nqk:], plain[:, nqk:], rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------- indexer warm-up objective
+
+def test_warmup_target_rows_sum_to_one_and_match_softmax_and_attention():
+    rng = np.random.default_rng(41)
+    T, H = 12, 3
+    q, kv = _bf16(rng, (T, H, 576)), _bf16(rng, (T, 576))
+    p = oracle.attention_probs(q, kv, 1 / 24)
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, rtol=1e-12)
+    assert (p[np.triu_indices(T, 1)] == 0).all()                 # causal
+    # one head: the library softmax of the masked logits
+    p1 = oracle.attention_probs(q[:, :1], kv, 1 / 24)
+    z = (q[:, 0].double() @ kv.double().T) / 24
+    ref = torch.softmax(z.masked_fill(~torch.ones(T, T, dtype=torch.bool).tril(), -np.inf), -1)
+    np.testing.assert_allclose(p1, ref.numpy(), rtol=1e-10, atol=1e-14)
+    # the same weights give the pinned sparse-MLA oracle's dense output
+    idx = np.full((T, T), -1, np.int32)
+    for t in range(T):
+        idx[t, : t + 1] = np.arange(t + 1)
+    out, _ = oracle.sparse_mla(q[:, :1], kv, idx, 1 / 24)
+    np.testing.assert_allclose(out[:, 0], p1 @ kv[:, :512].double().numpy(), rtol=1e-9, atol=1e-12)
+
+
+def test_warmup_kl_zero_at_the_target_and_gradient_by_finite_differences():
+    rng = np.random.default_rng(42)
+    R, n = 4, 17
+    p = rng.dirichlet(np.ones(n), size=R)
+    I = np.log(p) + rng.normal(size=(R, 1))                      # softmax(I) == p
+    loss, grad = oracle.indexer_kl(I, p, np.full(R, n))
+    np.testing.assert_allclose(loss, 0.0, atol=1e-12)
+    np.testing.assert_allclose(grad, 0.0, atol=1e-12)
+    I = rng.normal(size=(R, n)) * 2.0
+    loss, grad = oracle.indexer_kl(I, p, np.full(R, n))
+    assert (loss > 0).all()
+    eps = 1e-6
+    for s in (0, 5, 16):
+        e = np.zeros_like(I)
+        e[:, s] = eps
+        lp, _ = oracle.indexer_kl(I + e, p, np.full(R, n))
+        lm, _ = oracle.indexer_kl(I - e, p, np.full(R, n))
+        np.testing.assert_allclose((lp - lm) / (2 * eps), grad[:, s], rtol=1e-6, atol=1e-9)
+
+
+def _float_indexer(qf, kf, w, scale, q_pos0=0):
+    """I[t, s] from dequantised inputs, float64, causal (-inf past the row's keys)."""
+    x = np.einsum("thd,sd->ths", qf, kf)
+    I = np.einsum("th,ths->ts", w, np.maximum(scale * x, 0.0))
+    T, S = I.shape
+    mask = np.arange(S)[None, :] <= (q_pos0 + np.arange(T))[:, None]
+    return np.where(mask, I, -np.inf)
+
+
+def test_warmup_backward_matches_finite_differences():
+    rng = np.random.default_rng(43)
+    T, Hi, scale = 6, 2, 0.25
+    q8 = e4m3_codes(rng, (T, Hi, 128), -4, 4)
+    k8 = e4m3_codes(rng, (T, 128), -4, 4)
+    q_scale = torch.from_numpy(rng.uniform(0.5, 1.5, T)).float()
+    k_scale = torch.from_numpy(rng.uniform(0.5, 1.5, T)).float()
+    w = torch.from_numpy(rng.normal(size=(T, Hi)) / 8).float()
+    qf = lib_float(q8).numpy() * q_scale.double().numpy()[:, None, None]
+    kf = lib_float(k8).numpy() * k_scale.double().numpy()[:, None]
+    wd = w.double().numpy()
+    p = np.tril(rng.uniform(0.1, 1.0, (T, T)))
+    p /= p.sum(axis=1, keepdims=True)
+    n = np.arange(1, T + 1)
+
+    def loss_of(qf_, kf_, w_):
+        I = _float_indexer(qf_, kf_, w_, scale)
+        I = np.where(np.isfinite(I), I, 0.0)
+        return oracle.indexer_kl(I, p, n)[0].sum()
+
+    I0 = np.where(np.isfinite(_float_indexer(qf, kf, wd, scale)),
+                  _float_indexer(qf, kf, wd, scale), 0.0)
+    _, g = oracle.indexer_kl(I0, p, n)
+    dq, dk, dw = oracle.indexer_backward(q8, q_scale, k8, k_scale, w, scale, g)
+    eps = 1e-5
+    for (t, h, d) in [(5, 1, 3), (2, 0, 100), (4, 1, 64)]:
+        e = np.zeros_like(qf)
+        e[t, h, d] = eps
+        num = (loss_of(qf + e, kf, wd) - loss_of(qf - e, kf, wd)) / (2 * eps)
+        np.testing.assert_allclose(dq[t, h, d], num, rtol=1e-5, atol=1e-9)
+    for (s, d) in [(0, 7), (3, 127), (5, 50)]:
+        e = np.zeros_like(kf)
+        e[s, d] = eps
+        num = (loss_of(qf, kf + e, wd) - loss_of(qf, kf - e, wd)) / (2 * eps)
+        np.testing.assert_allclose(dk[s, d], num, rtol=1e-5, atol=1e-9)
+    for (t, h) in [(5, 0), (3, 1)]:
+        e = np.zeros_like(wd)
+        e[t, h] = eps
+        num = (loss_of(qf, kf, wd + e) - loss_of(qf, kf, wd - e)) / (2 * eps)
+        np.testing.assert_allclose(dw[t, h], num, rtol=1e-5, atol=1e-9)
