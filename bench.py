@@ -429,9 +429,12 @@ def time_warmup(dsa, steps, warmup, L=2048):
                                inp["scale"])
         state["loss"], state["grad"] = dsa.indexer_kl(I, state["p"], L)
 
+    bws = torch.empty(dsa.lib().dsa_indexer_backward_workspace_size(L, L, inp["Hi"]),
+                      dtype=torch.uint8, device="cuda")
+
     def backward():
         dsa.indexer_backward(inp["q8"], inp["q_scale"], inp["k8"], inp["k_scale"], inp["w"],
-                             inp["scale"], state["grad"])
+                             inp["scale"], state["grad"], workspace=bws)
 
     res = {"workload": f"prefill L={L}, 128 MLA heads, 64 indexer heads: target (dense MLA "
                        "for lse + head-mean weights), KL + gradient, backward to q, k, w"}

@@ -177,7 +177,7 @@ int dsa_project_indexer_inputs(const void *h, const void *wt, const float *rope,
  * The target of query t is read as the dense causal attention distribution
  * averaged over heads; the indexer's distribution is softmax(I[t, s]) over
  * the same keys. Row t sits at position q_pos0 + t and sees keys 0 .. that
- * position (clamped to S - 1). fp32 throughout.
+ * position (clamped to S - 1). fp32 results.
  *
  * dsa_attention_probs_mean:
  *   p[t][s] = (1/H) sum_h exp(sm_scale q[t,h] . kv[s] - lse[t][h]), 0 past the
@@ -195,8 +195,15 @@ int dsa_project_indexer_inputs(const void *h, const void *wt, const float *rope,
  *   through I = sum_h w * ReLU(scale * qf . kf) with qf = q8 * q_scale and
  *   kf = k8 * k_scale (the FP8 inputs dsa_indexer_scores takes), given
  *   grad = dloss/dI [T][ldg]: dq [T][Hi][128] (w.r.t. qf), dk [S][128]
- *   (w.r.t. kf), dw [T][Hi], all fp32, caller-owned.
- * Each returns DSA_ERR_INVALID_ARG (nothing launched) on bad arguments and
+ *   (w.r.t. kf), dw [T][Hi], all fp32, caller-owned, dq and dk 16-byte
+ *   aligned; dk sums over the T rows given (a caller splitting the rows into
+ *   chunks adds the chunks' dk). The products q8 . k8, dq and dk are tensor-
+ *   core GEMMs through the caller's workspace of
+ *   dsa_indexer_backward_workspace_size(T, S, Hi) bytes, about
+ *   T * Hi * S * 10 bytes (keep T * Hi * S near 2^28 or below by chunking the
+ *   rows); T * Hi and S at most 2^23.
+ * Each returns DSA_ERR_INVALID_ARG (nothing launched) on bad arguments,
+ * DSA_ERR_WORKSPACE for a missing or short workspace, and
  * DSA_ERR_UNSUPPORTED for an indexer head count outside {1, 2, 4, ..., 64}.
  */
 size_t dsa_attention_probs_workspace_size(int T, int S, int H);
@@ -205,10 +212,11 @@ int dsa_attention_probs_mean(const void *q, const void *kv, const float *lse, in
                              void *workspace, size_t ws_bytes, dsa_stream_t stream);
 int dsa_indexer_kl(const float *I, int64_t ldi, const float *p, int64_t ldp, int T, int S,
                    int q_pos0, float *loss, float *grad, int64_t ldg, dsa_stream_t stream);
+size_t dsa_indexer_backward_workspace_size(int T, int S, int Hi);
 int dsa_indexer_backward(const void *q8, const float *q_scale, const void *k8,
-                         const float *k_scale, const float *w, int T, int S, int Hi,
-                         int q_pos0, float scale, const float *grad, int64_t ldg, float *dq,
-                         float *dk, float *dw, dsa_stream_t stream);
+                         const float *k_scale, const float *w, int T, int S, int Hi, int q_pos0,
+                         float scale, const float *grad, int64_t ldg, float *dq, float *dk,
+                         float *dw, void *workspace, size_t ws_bytes, dsa_stream_t stream);
 
 /*
  * Index sets for sliding-window and dense causal attention, to run through

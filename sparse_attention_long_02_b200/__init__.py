@@ -46,7 +46,9 @@ _sig("dsa_project_workspace_size", SZ, I32, I32)
 _sig("dsa_attention_probs_workspace_size", SZ, I32, I32, I32)
 _sig("dsa_attention_probs_mean", I32, P, P, P, I32, I32, I32, I32, F32, P, I64, P, SZ, P)
 _sig("dsa_indexer_kl", I32, P, I64, P, I64, I32, I32, I32, P, P, I64, P)
-_sig("dsa_indexer_backward", I32, P, P, P, P, P, I32, I32, I32, I32, F32, P, I64, P, P, P, P)
+_sig("dsa_indexer_backward_workspace_size", SZ, I32, I32, I32)
+_sig("dsa_indexer_backward", I32, P, P, P, P, P, I32, I32, I32, I32, F32, P, I64, P, P, P, P, SZ,
+     P)
 _sig("dsa_project_indexer_inputs", I32, P, P, P, I32, I32, I32, P, P, P, P, P, P, SZ, P)
 _sig("dsa_forward_workspace_size", SZ, I32, I32, I32, I32, I32, I32)
 _sig("dsa_forward", I32, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, F32, F32,
@@ -200,7 +202,8 @@ def indexer_kl(I, p, S, q_pos0=0, stream=None):
     return loss, grad
 
 
-def indexer_backward(q8, q_scale, k8, k_scale, w, scale, grad, q_pos0=0, stream=None):
+def indexer_backward(q8, q_scale, k8, k_scale, w, scale, grad, q_pos0=0, workspace=None,
+                     stream=None):
     """Gradients of the warm-up loss w.r.t. the dequantised indexer inputs ->
     (dq [T][Hi][128], dk [S][128], dw [T][Hi]) in float32."""
     q8, k8 = _u8(q8), _u8(k8)
@@ -211,10 +214,14 @@ def indexer_backward(q8, q_scale, k8, k_scale, w, scale, grad, q_pos0=0, stream=
     dq = torch.empty(T, Hi, 128, dtype=torch.float32, device=dev)
     dk = torch.empty(S, 128, dtype=torch.float32, device=dev)
     dw = torch.empty(T, Hi, dtype=torch.float32, device=dev)
+    if workspace is None:
+        need = _lib.dsa_indexer_backward_workspace_size(T, S, Hi)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     _check(_lib.dsa_indexer_backward(_p(q8), _p(_dev(q_scale, torch.float32)), _p(k8),
                                      _p(_dev(k_scale, torch.float32)), _p(w), T, S, Hi, q_pos0,
                                      float(scale), _p(grad), grad.shape[1], _p(dq), _p(dk),
-                                     _p(dw), _stream(stream)), "dsa_indexer_backward")
+                                     _p(dw), _p(workspace), workspace.numel(), _stream(stream)),
+           "dsa_indexer_backward")
     return dq, dk, dw
 
 

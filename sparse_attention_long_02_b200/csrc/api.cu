@@ -286,15 +286,24 @@ int dsa_indexer_kl(const float* I, int64_t ldi, const float* p, int64_t ldp, int
                                      static_cast<cudaStream_t>(stream)));
 }
 
+size_t dsa_indexer_backward_workspace_size(int T, int S, int Hi) {
+  if (T <= 0 || S <= 0 || !valid_hi(Hi)) return 0;
+  return dsa::indexer_backward_workspace(T, S, Hi);
+}
+
 int dsa_indexer_backward(const void* q8, const float* q_scale, const void* k8, const float* k_scale,
                          const float* w, int T, int S, int Hi, int q_pos0, float scale,
                          const float* grad, int64_t ldg, float* dq, float* dk, float* dw,
-                         dsa_stream_t stream) {
+                         void* workspace, size_t ws_bytes, dsa_stream_t stream) {
   if (!q8 || !k8 || !w || !grad || !dq || !dk || !dw || T < 0 || S <= 0 || q_pos0 < 0 ||
-      ldg < S || !(scale > 0.f))
+      ldg < S || !(scale > 0.f) || !aligned16(dq) || !aligned16(dk) ||
+      S > (1 << 23) || static_cast<long long>(T) * Hi > (1ll << 23))
     return DSA_ERR_INVALID_ARG;
   if (!valid_hi(Hi)) return DSA_ERR_UNSUPPORTED;
   if (T == 0) return DSA_OK;
+  if (!workspace || !aligned16(workspace) ||
+      ws_bytes < dsa::indexer_backward_workspace(T, S, Hi))
+    return DSA_ERR_WORKSPACE;
   IndexerBwdArgs a;
   a.T = T;
   a.S = S;
@@ -311,7 +320,8 @@ int dsa_indexer_backward(const void* q8, const float* q_scale, const void* k8, c
   a.dq = dq;
   a.dk = dk;
   a.dw = dw;
-  return status_of(launch_indexer_backward(a, static_cast<cudaStream_t>(stream)));
+  return status_of(launch_indexer_backward(a, workspace, device_error_word(),
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 int dsa_window_indices(int T, int S, int q_pos0, int window, int k, int32_t* idx,

@@ -44,6 +44,9 @@ struct ProjArgs {
   const float* rope = nullptr;            // [T][64] (cos, sin) pairs
   float* y = nullptr;                     // workspace [T][Hi*128 + 128] fp32, rotated q | k
   long long ldy = 0;                      // row stride of y in the plain GEMM
+  long long zstride = 0;                  // plain GEMM: offset of split z's output
+  int kb = 0;                             // plain GEMM: B's K extent (0: d); B's K wraps
+  int kt_split = 0;                       // plain GEMM: 64-wide K steps per split (0: all)
   unsigned* amax_q = nullptr;             // workspace [T], |y| maximum as float bits
   unsigned* amax_k = nullptr;
   float* a = nullptr;                     // [T][Hi] per-head weights out
@@ -95,14 +98,17 @@ cudaError_t launch_window(int T, int S, int q_pos0, int window, int k, int* idx,
 cudaError_t launch_project(const ProjArgs& a, const void* h, const void* wt, cudaStream_t st);
 // C [M][ldc] fp32 = A [M][K] x B [N][K]^T, bf16 operands, K a multiple of 8.
 cudaError_t launch_gemm_f32(const void* a, const void* b, float* c, int M, int N, int K,
-                            long long ldc, unsigned* err, cudaStream_t st);
+                            long long ldc, unsigned* err, cudaStream_t st, int kb = 0,
+                            int kt_split = 0);
 cudaError_t launch_attention_probs(const void* q, const void* kv, const float* lse, int T, int S,
                                    int H, int q_pos0, float sm_scale, float* p, long long ldp,
                                    float* z, long long ldz, unsigned* err, cudaStream_t st);
 cudaError_t launch_indexer_kl(const float* I, long long ldi, const float* p, long long ldp, int T,
                               int S, int q_pos0, float* loss, float* grad, long long ldg,
                               cudaStream_t st);
-cudaError_t launch_indexer_backward(const IndexerBwdArgs& a, cudaStream_t st);
+size_t indexer_backward_workspace(int T, int S, int Hi);
+cudaError_t launch_indexer_backward(const IndexerBwdArgs& a, void* workspace, unsigned* err,
+                                    cudaStream_t st);
 cudaError_t launch_sparse_mla(const MlaArgs& a, const void* q, const void* kv, long long kv_rows,
                               long long q_rows, cudaStream_t st);
 

@@ -17,7 +17,10 @@
 // code = e4m3(y / scale), rounded to nearest even and saturated at +-448.
 //
 // The same GEMM with a plain epilogue (every output written in fp32) serves
-// the attention logits of the indexer's warm-up target.
+// the indexer's warm-up objective: the attention logits of its target, and
+// the products of its backward. For those, B's K coordinate may wrap (A holds
+// several K-blocks that all multiply the same B), and a launch may split K
+// over grid.z, split z writing its partial product at y + z * M * ldy.
 #include "common.cuh"
 #include "dsa_internal.h"
 #include <cuda_fp8.h>
@@ -50,7 +53,12 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant
   unsigned* err = P.err;
   if (launch_aborted(err)) return;
   const int n0 = blockIdx.x * kBN, m0 = blockIdx.y * kBM;
-  const int nk = (P.d + kBK - 1) / kBK;
+  // K steps of this CTA: all of them, or split z of a split-K launch
+  const int nk_all = (P.d + kBK - 1) / kBK;
+  const int per = P.kt_split > 0 ? P.kt_split : nk_all;
+  const int kt0 = blockIdx.z * per;
+  const int nk = min(per, nk_all - kt0);
+  const int kbw = P.kb > 0 ? P.kb : P.d;          // B's K extent: its coordinate wraps
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
     for (int i = 0; i < kPStages; ++i) {
@@ -75,15 +83,16 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
       int issued = 0;
-      for (int kt = 0; kt < nk; ++kt) {
-        const int st = kt % kPStages;
-        if (kt >= kPStages &&
-            !mbar_wait(smem_u32(&sm.empty[st]), ((kt / kPStages) + 1) & 1, abort_flag, err))
+      for (int i = 0; i < nk; ++i) {
+        const int st = i % kPStages;
+        if (i >= kPStages &&
+            !mbar_wait(smem_u32(&sm.empty[st]), ((i / kPStages) + 1) & 1, abort_flag, err))
           break;
         const uint32_t full = smem_u32(&sm.full[st]);
+        const int k = (kt0 + i) * kBK;
         mbar_expect_tx(full, kATile + kBTile);
-        tma_load_2d(smem_u32(sm.a[st]), &tm_h, full, kt * kBK, m0);
-        tma_load_2d(smem_u32(sm.b[st]), &tm_w, full, kt * kBK, n0);
+        tma_load_2d(smem_u32(sm.a[st]), &tm_h, full, k, m0);
+        tma_load_2d(smem_u32(sm.b[st]), &tm_w, full, k % kbw, n0);
         ++issued;
       }
       for (int i = issued > kPStages ? issued - kPStages : 0; i < issued; ++i)
@@ -123,10 +132,16 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant
         tmem_ld32(tmem + lane_base + 32 * c, y);
         if (t >= P.T || col0 >= P.N) continue;
         if constexpr (kPlain) {
-          float* dst = P.y + t * P.ldy + col0;
+          float* dst = P.y + blockIdx.z * P.zstride + t * P.ldy + col0;
+          if (col0 + 32 <= P.N) {        // rows and y 16-byte aligned (ldy % 4 == 0)
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (col0 + j < P.N) dst[j] = y[j];
+            for (int j = 0; j < 32; j += 4)
+              *reinterpret_cast<float4*>(dst + j) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < P.N) dst[j] = y[j];
+          }
           continue;
         }
         if (col0 < nqk) {
@@ -207,15 +222,18 @@ cudaError_t launch_gemm(const ProjArgs& a, const void* h, const void* wt, cudaSt
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   cudaError_t e = make_tmap_2d(&th, h, bf, a.d, a.T, static_cast<uint64_t>(a.d) * 2, kBK, kBM,
                                CU_TENSOR_MAP_SWIZZLE_128B);
+  const int kbw = a.kb > 0 ? a.kb : a.d;
   if (e == cudaSuccess)
-    e = make_tmap_2d(&tw, wt, bf, a.d, a.N, static_cast<uint64_t>(a.d) * 2, kBK, kBN,
+    e = make_tmap_2d(&tw, wt, bf, kbw, a.N, static_cast<uint64_t>(kbw) * 2, kBK, kBN,
                      CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(ProjSmem) + 1024;
   e = cudaFuncSetAttribute(proj_gemm_kernel<kPlain>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid((a.N + kBN - 1) / kBN, (a.T + kBM - 1) / kBM);
+  const int nk = (a.d + kBK - 1) / kBK;
+  const int splits = a.kt_split > 0 ? (nk + a.kt_split - 1) / a.kt_split : 1;
+  dim3 grid((a.N + kBN - 1) / kBN, (a.T + kBM - 1) / kBM, splits);
   proj_gemm_kernel<kPlain><<<grid, kProjThreads, smem, st>>>(th, tw, a);
   return cudaGetLastError();
 }
@@ -228,13 +246,16 @@ cudaError_t launch_project(const ProjArgs& a, const void* h, const void* wt, cud
 }
 
 cudaError_t launch_gemm_f32(const void* a, const void* b, float* c, int M, int N, int K,
-                            long long ldc, unsigned* err, cudaStream_t st) {
+                            long long ldc, unsigned* err, cudaStream_t st, int kb, int kt_split) {
   ProjArgs P;
   P.T = M;
   P.N = N;
   P.d = K;
+  P.kb = kb;
+  P.kt_split = kt_split;
   P.y = c;
   P.ldy = ldc;
+  P.zstride = static_cast<long long>(M) * ldc;
   P.err = err;
   return launch_gemm<true>(P, a, b, st);
 }

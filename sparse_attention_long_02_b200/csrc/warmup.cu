@@ -12,13 +12,14 @@
 // I = sum_h w * ReLU(scale * qf . kf) to the dequantised inputs qf, kf and w;
 // the ReLU's decision is taken on the raw FP8 dot product, as in the forward.
 //
-// The attention logits of the target come from the tcgen05 GEMM; the rest are
-// plain CUDA-core kernels in fp32 (one CTA per query row, or per block of
-// keys): the objective is a training-time step, measured but not tuned like
-// the inference path.
+// The attention logits of the target and the three products of the backward
+// are tcgen05 GEMMs; the reductions and coefficients around them are
+// CUDA-core kernels in fp32 over coalesced rows.
 #include "common.cuh"
 #include "dsa_internal.h"
 #include <cuda_fp8.h>
+#include <cuda_bf16.h>
+#include <algorithm>
 
 namespace dsa {
 namespace {
@@ -112,128 +113,181 @@ __global__ void __launch_bounds__(kWThreads) kl_kernel(const float* __restrict__
   if (threadIdx.x == 0) loss[t] = kl;
 }
 
-constexpr int kQKeys = 32;     // keys per block in the per-query kernel
-constexpr int kKKeys = 16;     // keys per CTA in the per-key kernel
-
 // The ReLU's decision is taken on the raw e4m3 dot product xr = q8 . k8 (the
 // scales are positive), as the forward indexer takes it; the scales enter the
-// magnitudes only: x = q_scale * k_scale * xr.
-//
-// Per query t, over its keys in blocks of 32:
-//   dq[t,h,:] = w[t,h] scale sum_s g[t,s] [xr > 0] k_scale[s] k8[s,:]
-//   dw[t,h]   = sum_s g[t,s] scale q_scale[t] k_scale[s] max(xr, 0)
-__global__ void __launch_bounds__(kWThreads) bwd_query_kernel(const IndexerBwdArgs A) {
-  extern __shared__ float smem[];
-  const int Hi = A.Hi;
-  float* qr = smem;                          // [Hi][128] e4m3 values
-  float* kr = qr + Hi * 128;                 // [32][128] e4m3 values
-  float* xs = kr + kQKeys * 128;             // [32][Hi] raw dot products
-  float* gs = xs + kQKeys * Hi;              // [32] g * k_scale
-  const long long t = blockIdx.x;
-  const long long n = min(static_cast<long long>(A.q_pos0) + t + 1, static_cast<long long>(A.S));
-  const float qsc = A.q_scale ? A.q_scale[t] : 1.f;
-  for (int j = threadIdx.x; j < Hi * 128; j += kWThreads) qr[j] = e4m3_value(A.q8[t * Hi * 128 + j]);
-  constexpr int kOut = 32;                   // outputs per thread: Hi * 128 / 256 <= 32
-  float acc[kOut];
-#pragma unroll
-  for (int i = 0; i < kOut; ++i) acc[i] = 0.f;
-  float dw = 0.f;
-  const float* g = A.grad + t * A.ldg;
-  for (long long s0 = 0; s0 < n; s0 += kQKeys) {
-    __syncthreads();
-    for (int j = threadIdx.x; j < kQKeys * 128; j += kWThreads) {
-      const long long s = s0 + j / 128;
-      kr[j] = s < n ? e4m3_value(A.k8[s * 128 + (j % 128)]) : 0.f;
-    }
-    if (threadIdx.x < kQKeys) {
-      const long long s = s0 + threadIdx.x;
-      gs[threadIdx.x] = s < n ? g[s] * (A.k_scale ? A.k_scale[s] : 1.f) : 0.f;
-    }
-    __syncthreads();
-    for (int j = threadIdx.x; j < kQKeys * Hi; j += kWThreads) {
-      const int ks = j / Hi, h = j % Hi;
-      float x = 0.f;
-      for (int d = 0; d < 128; ++d) x = fmaf(qr[h * 128 + d], kr[ks * 128 + d], x);
-      xs[ks * Hi + h] = x;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < kOut; ++i) {
-      const int o = threadIdx.x + kWThreads * i;
-      if (o < Hi * 128) {
-        const int h = o / 128, d = o % 128;
-        float a = acc[i];
-        for (int ks = 0; ks < kQKeys; ++ks)
-          if (xs[ks * Hi + h] > 0.f) a = fmaf(gs[ks], kr[ks * 128 + d], a);
-        acc[i] = a;
-      }
-    }
-    if (threadIdx.x < Hi)
-      for (int ks = 0; ks < kQKeys; ++ks)
-        dw = fmaf(gs[ks], fmaxf(xs[ks * Hi + threadIdx.x], 0.f), dw);
-  }
-#pragma unroll
-  for (int i = 0; i < kOut; ++i) {
-    const int o = threadIdx.x + kWThreads * i;
-    if (o < Hi * 128) A.dq[t * Hi * 128 + o] = acc[i] * A.w[t * Hi + o / 128] * A.scale;
-  }
-  if (threadIdx.x < Hi) A.dw[t * Hi + threadIdx.x] = dw * A.scale * qsc;
+// magnitudes only: x = q_scale * k_scale * xr. With r = (t, h) a row of the
+// T*Hi query heads and pos(t) = min(q_pos0 + t, S - 1):
+//   dq[r,:] = sum_s Cq[r,s] k8[s,:],  Cq[r,s] = [s <= pos(t)][xr > 0] g[t,s] k_scale[s] w[r] scale
+//   dk[s,:] = sum_r Ck[s,r] q8[r,:],  Ck[s,r] = [s <= pos(t)][xr > 0] g[t,s] q_scale[t] w[r] scale
+//   dw[r]   = scale q_scale[t] sum_{s <= pos(t)} g[t,s] k_scale[s] max(xr, 0)
+// xr, dq and dk are tcgen05 GEMMs. The e4m3 codes are exact in bf16, and each
+// fp32 coefficient is written as three bf16 pieces whose sum is exactly that
+// coefficient (8 + 8 + 8 significant bits); the pieces lie side by side along
+// K against the same B, so every product in the tensor core is exact and the
+// accumulation is fp32.
+
+__device__ __forceinline__ void split3(float v, __nv_bfloat16& a, __nv_bfloat16& b,
+                                       __nv_bfloat16& c) {
+  a = __float2bfloat16_rn(v);
+  const float r1 = v - __bfloat162float(a);      // exact: at most 16 significant bits
+  b = __float2bfloat16_rn(r1);
+  c = __float2bfloat16_rn(r1 - __bfloat162float(b));
 }
 
-// Per block of 16 keys, over the queries that see them:
-//   dk[s,:] = scale sum_t sum_h g[t,s] w[t,h] [xr > 0] q_scale[t] q8[t,h,:]
-__global__ void __launch_bounds__(kWThreads) bwd_key_kernel(const IndexerBwdArgs A) {
-  extern __shared__ float smem[];
-  const int Hi = A.Hi;
-  float* kr = smem;                          // [16][128] e4m3 values
-  float* qr = kr + kKKeys * 128;             // [Hi][128] e4m3 values of query t
-  float* xs = qr + Hi * 128;                 // [16][Hi] coefficients
-  float* gs = xs + kKKeys * Hi;              // [16]
-  float* ws = gs + kKKeys;                   // [Hi]
-  const long long s0 = static_cast<long long>(blockIdx.x) * kKKeys;
-  for (int j = threadIdx.x; j < kKKeys * 128; j += kWThreads) {
-    const long long s = s0 + j / 128;
-    kr[j] = s < A.S ? e4m3_value(A.k8[s * 128 + (j % 128)]) : 0.f;
-  }
-  constexpr int kOut = kKKeys * 128 / kWThreads;   // 8
-  float acc[kOut];
+__device__ __forceinline__ uint2 pack4(__nv_bfloat16 a, __nv_bfloat16 b, __nv_bfloat16 c,
+                                       __nv_bfloat16 d) {
+  uint2 u;
+  u.x = static_cast<uint32_t>(__bfloat16_as_ushort(a)) |
+        (static_cast<uint32_t>(__bfloat16_as_ushort(b)) << 16);
+  u.y = static_cast<uint32_t>(__bfloat16_as_ushort(c)) |
+        (static_cast<uint32_t>(__bfloat16_as_ushort(d)) << 16);
+  return u;
+}
+
+// Writes the three pieces of four consecutive coefficients v[0..3] at column c
+// of a row whose pieces start every `piece` elements.
+__device__ __forceinline__ void store_split4(__nv_bfloat16* row, long long piece, long long c,
+                                             const float (&v)[4]) {
+  __nv_bfloat16 p[3][4];
 #pragma unroll
-  for (int i = 0; i < kOut; ++i) acc[i] = 0.f;
-  // queries that see key s0 (position q_pos0 + t >= s0)
-  const long long t0 = max(0ll, s0 - A.q_pos0);
-  for (long long t = t0; t < A.T; ++t) {
-    __syncthreads();
-    for (int j = threadIdx.x; j < Hi * 128; j += kWThreads) qr[j] = e4m3_value(A.q8[t * Hi * 128 + j]);
-    const long long pos = static_cast<long long>(A.q_pos0) + t;
-    const float qsc = A.q_scale ? A.q_scale[t] : 1.f;
-    if (threadIdx.x < kKKeys) {
-      const long long s = s0 + threadIdx.x;
-      gs[threadIdx.x] = (s < A.S && s <= pos) ? A.grad[t * A.ldg + s] * qsc : 0.f;
-    }
-    for (int h = threadIdx.x; h < Hi; h += kWThreads) ws[h] = A.w[t * Hi + h];
-    __syncthreads();
-    for (int j = threadIdx.x; j < kKKeys * Hi; j += kWThreads) {
-      const int ks = j / Hi, h = j % Hi;
-      float x = 0.f;
-      for (int d = 0; d < 128; ++d) x = fmaf(qr[h * 128 + d], kr[ks * 128 + d], x);
-      xs[ks * Hi + h] = x > 0.f ? gs[ks] * ws[h] : 0.f;
-    }
-    __syncthreads();
+  for (int j = 0; j < 4; ++j) split3(v[j], p[0][j], p[1][j], p[2][j]);
 #pragma unroll
-    for (int i = 0; i < kOut; ++i) {
-      const int o = threadIdx.x + kWThreads * i;   // (key, dim) = (o / 128, o % 128)
-      const int ks = o / 128, d = o % 128;
-      float a = acc[i];
-      for (int h = 0; h < Hi; ++h) a = fmaf(xs[ks * Hi + h], qr[h * 128 + d], a);
-      acc[i] = a;
-    }
+  for (int k = 0; k < 3; ++k)
+    *reinterpret_cast<uint2*>(row + k * piece + c) = pack4(p[k][0], p[k][1], p[k][2], p[k][3]);
+}
+
+// e4m3 rows [rows][128] -> bf16 copies: dst [rows][128] and its transpose
+// dstT [128][ldT] (columns rows .. ldT - 1 zero). One CTA per 64 rows.
+__global__ void __launch_bounds__(kWThreads) to_bf16_kernel(const uint8_t* __restrict__ src,
+                                                            long long rows,
+                                                            __nv_bfloat16* __restrict__ dst,
+                                                            __nv_bfloat16* __restrict__ dstT,
+                                                            long long ldT) {
+  __shared__ float tile[64][129];
+  const long long r0 = static_cast<long long>(blockIdx.x) * 64;
+  for (int j = threadIdx.x; j < 64 * 128; j += kWThreads) {
+    const int i = j / 128, d = j % 128;
+    const long long r = r0 + i;
+    const float v = r < rows ? e4m3_value(src[r * 128 + d]) : 0.f;
+    tile[i][d] = v;
+    if (r < rows) dst[r * 128 + d] = __float2bfloat16_rn(v);
   }
+  __syncthreads();
+  for (int j = threadIdx.x; j < 64 * 128; j += kWThreads) {
+    const int d = j / 64, i = j % 64;
+    dstT[d * ldT + r0 + i] = __float2bfloat16_rn(tile[i][d]);
+  }
+}
+
+// One CTA per query-head row r: the pieces of Cq[r, 0 .. Sp) and dw[r].
+__global__ void __launch_bounds__(kWThreads) coef_q_kernel(const IndexerBwdArgs A,
+                                                           const float* __restrict__ x,
+                                                           long long ldx,
+                                                           __nv_bfloat16* __restrict__ cq,
+                                                           long long Sp) {
+  __shared__ float red[kWThreads / 32];
+  const long long r = blockIdx.x, t = r / A.Hi;
+  const long long pos = min(static_cast<long long>(A.q_pos0) + t, static_cast<long long>(A.S) - 1);
+  const float wsc = A.w[r] * A.scale;
+  const float* xr = x + r * ldx;
+  const float* g = A.grad + t * A.ldg;
+  __nv_bfloat16* row = cq + r * 3 * Sp;
+  float dw = 0.f;
+  for (long long s = 4ll * threadIdx.x; s < Sp; s += 4 * kWThreads) {
+    float4 x4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (s < A.S) x4 = *reinterpret_cast<const float4*>(xr + s);   // s + 3 < ldx
+    const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
+    float v[4];
 #pragma unroll
-  for (int i = 0; i < kOut; ++i) {
-    const int o = threadIdx.x + kWThreads * i;
-    const long long s = s0 + o / 128;
-    if (s < A.S) A.dk[s * 128 + (o % 128)] = acc[i] * A.scale;
+    for (int j = 0; j < 4; ++j) {
+      v[j] = 0.f;
+      if (s + j <= pos) {
+        const float gk = g[s + j] * (A.k_scale ? A.k_scale[s + j] : 1.f);
+        if (xv[j] > 0.f) {
+          v[j] = gk * wsc;
+          dw = fmaf(gk, xv[j], dw);
+        }
+      }
+    }
+    store_split4(row, Sp, s, v);
   }
+  dw = block_sum(dw, red);
+  if (threadIdx.x == 0) A.dw[r] = dw * A.scale * (A.q_scale ? A.q_scale[t] : 1.f);
+}
+
+// Grid (S, column blocks of 1024): the pieces of Ck[s, 0 .. Kp) for key s,
+// from xt = xr transposed ([S][ldxt]).
+__global__ void __launch_bounds__(kWThreads) coef_k_kernel(const IndexerBwdArgs A,
+                                                           const float* __restrict__ xt,
+                                                           long long ldxt,
+                                                           __nv_bfloat16* __restrict__ ck,
+                                                           long long Kp) {
+  const long long s = blockIdx.x;
+  const long long c = 4 * (static_cast<long long>(blockIdx.y) * kWThreads + threadIdx.x);
+  if (c >= Kp) return;
+  const long long R = static_cast<long long>(A.T) * A.Hi;
+  float4 x4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (c < R) x4 = *reinterpret_cast<const float4*>(xt + s * ldxt + c);   // c + 3 < ldxt
+  const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
+  float v[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    v[j] = 0.f;
+    const long long r = c + j, t = r / A.Hi;
+    if (r < R && A.q_pos0 + t >= s && xv[j] > 0.f)
+      v[j] = A.grad[t * A.ldg + s] * (A.q_scale ? A.q_scale[t] : 1.f) * A.w[r] * A.scale;
+  }
+  store_split4(ck + s * 3 * Kp, Kp, c, v);
+}
+
+// dk = sum over the splits of the split-K partial products.
+__global__ void __launch_bounds__(kWThreads) sum_splits_kernel(const float* __restrict__ part,
+                                                               int splits, long long n,
+                                                               float* __restrict__ out) {
+  const long long i = static_cast<long long>(blockIdx.x) * kWThreads + threadIdx.x;
+  if (i >= n) return;
+  float a = 0.f;
+  for (int z = 0; z < splits; ++z) a += part[z * n + i];
+  out[i] = a;
+}
+
+long long round_to(long long v, long long m) { return (v + m - 1) / m * m; }
+
+// Workspace of the backward, each part 256-byte aligned.
+struct BwdLayout {
+  long long R, Sp, Kp, ldx, ldxt;
+  int splits, kps;
+  size_t x, c, qb, qbt, kb, kbt, part, total;
+};
+
+BwdLayout bwd_layout(int T, int S, int Hi) {
+  BwdLayout L;
+  L.R = static_cast<long long>(T) * Hi;
+  L.Sp = round_to(S, 64);
+  L.Kp = round_to(L.R, 64);
+  L.ldx = round_to(S, 4);
+  L.ldxt = round_to(L.R, 4);
+  // dk: S / 128 row tiles of one 128-column tile; split K to fill the 148 SMs
+  const int m_tiles = (S + 127) / 128;
+  const int nk = static_cast<int>(3 * L.Kp / 64);
+  L.splits = std::max(1, std::min(nk, 148 / m_tiles));
+  L.kps = (nk + L.splits - 1) / L.splits;
+  L.splits = (nk + L.kps - 1) / L.kps;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) / 256 * 256;
+    return o;
+  };
+  L.x = take(4 * static_cast<size_t>(std::max(L.R * L.ldx, static_cast<long long>(S) * L.ldxt)));
+  L.c = take(2 * static_cast<size_t>(std::max(L.R * 3 * L.Sp, static_cast<long long>(S) * 3 * L.Kp)));
+  L.qb = take(2 * static_cast<size_t>(L.R) * 128);
+  L.qbt = take(2 * static_cast<size_t>(L.Kp) * 128);
+  L.kb = take(2 * static_cast<size_t>(S) * 128);
+  L.kbt = take(2 * static_cast<size_t>(L.Sp) * 128);
+  L.part = take(4 * static_cast<size_t>(L.splits) * S * 128);
+  L.total = off;
+  return L;
 }
 
 }  // namespace
@@ -254,20 +308,44 @@ cudaError_t launch_indexer_kl(const float* I, long long ldi, const float* p, lon
   return cudaGetLastError();
 }
 
-cudaError_t launch_indexer_backward(const IndexerBwdArgs& a, cudaStream_t st) {
-  const size_t sq = sizeof(float) * (a.Hi * 128 + kQKeys * 128 + kQKeys * a.Hi + kQKeys);
-  const size_t sk = sizeof(float) * (kKKeys * 128 + a.Hi * 128 + kKKeys * a.Hi + kKKeys + a.Hi);
-  cudaError_t e = cudaFuncSetAttribute(bwd_query_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(sq));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(bwd_key_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(sk));
+size_t indexer_backward_workspace(int T, int S, int Hi) { return bwd_layout(T, S, Hi).total; }
+
+cudaError_t launch_indexer_backward(const IndexerBwdArgs& a, void* workspace, unsigned* err,
+                                    cudaStream_t st) {
+  const BwdLayout L = bwd_layout(a.T, a.S, a.Hi);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* x = reinterpret_cast<float*>(ws + L.x);
+  __nv_bfloat16* c = reinterpret_cast<__nv_bfloat16*>(ws + L.c);
+  __nv_bfloat16* qb = reinterpret_cast<__nv_bfloat16*>(ws + L.qb);
+  __nv_bfloat16* qbt = reinterpret_cast<__nv_bfloat16*>(ws + L.qbt);
+  __nv_bfloat16* kb = reinterpret_cast<__nv_bfloat16*>(ws + L.kb);
+  __nv_bfloat16* kbt = reinterpret_cast<__nv_bfloat16*>(ws + L.kbt);
+  float* part = reinterpret_cast<float*>(ws + L.part);
+  const int R = static_cast<int>(L.R);
+  to_bf16_kernel<<<static_cast<unsigned>(L.Kp / 64), kWThreads, 0, st>>>(a.q8, L.R, qb, qbt, L.Kp);
+  to_bf16_kernel<<<static_cast<unsigned>(L.Sp / 64), kWThreads, 0, st>>>(a.k8, a.S, kb, kbt, L.Sp);
+  cudaError_t e = cudaGetLastError();
+  // xr [R][S] -> Cq, dw -> dq
+  if (e == cudaSuccess) e = launch_gemm_f32(qb, kb, x, R, a.S, 128, L.ldx, err, st);
   if (e != cudaSuccess) return e;
-  bwd_query_kernel<<<a.T, kWThreads, sq, st>>>(a);
+  coef_q_kernel<<<R, kWThreads, 0, st>>>(a, x, L.ldx, c, L.Sp);
   e = cudaGetLastError();
+  if (e == cudaSuccess)
+    e = launch_gemm_f32(c, kbt, a.dq, R, 128, static_cast<int>(3 * L.Sp), 128, err, st,
+                        static_cast<int>(L.Sp));
+  // xr transposed [S][R] -> Ck -> dk (split K, then the sum of the splits)
+  if (e == cudaSuccess) e = launch_gemm_f32(kb, qb, x, a.S, R, 128, L.ldxt, err, st);
   if (e != cudaSuccess) return e;
-  bwd_key_kernel<<<(a.S + kKKeys - 1) / kKKeys, kWThreads, sk, st>>>(a);
+  coef_k_kernel<<<dim3(a.S, static_cast<unsigned>((L.Kp / 4 + kWThreads - 1) / kWThreads)),
+                  kWThreads, 0, st>>>(a, x, L.ldxt, c, L.Kp);
+  e = cudaGetLastError();
+  if (e == cudaSuccess)
+    e = launch_gemm_f32(c, qbt, part, a.S, 128, static_cast<int>(3 * L.Kp), 128, err, st,
+                        static_cast<int>(L.Kp), L.kps);
+  if (e != cudaSuccess) return e;
+  const long long n = static_cast<long long>(a.S) * 128;
+  sum_splits_kernel<<<static_cast<unsigned>((n + kWThreads - 1) / kWThreads), kWThreads, 0, st>>>(
+      part, L.splits, n, a.dk);
   return cudaGetLastError();
 }
 

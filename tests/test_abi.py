@@ -76,6 +76,17 @@ def test_host_validation_rejects_before_launch(dsa):
                                       fake, 4 * 2 * 8 * 4 - 1, None) == -3
     assert L.dsa_attention_probs_mean(fake, fake, fake, 4, 8, 2, 0, ctypes.c_float(0.1), fake, 7,
                                       fake, 1 << 20, None) == -1
+    # warm-up backward: workspace missing / too small; misaligned dq
+    need = L.dsa_indexer_backward_workspace_size(4, 8, 2)
+    assert L.dsa_indexer_backward(fake, None, fake, None, fake, 4, 8, 2, 0, ctypes.c_float(1.0),
+                                  fake, 8, fake, fake, fake, None, 0, None) == -3
+    assert L.dsa_indexer_backward(fake, None, fake, None, fake, 4, 8, 2, 0, ctypes.c_float(1.0),
+                                  fake, 8, fake, fake, fake, fake, need - 1, None) == -3
+    assert L.dsa_indexer_backward(fake, None, fake, None, fake, 4, 8, 2, 0, ctypes.c_float(1.0),
+                                  fake, 8, ctypes.c_void_p((1 << 20) + 4), fake, fake, fake,
+                                  need, None) == -1
+    assert L.dsa_indexer_backward(fake, None, fake, None, fake, 4, 8, 3, 0, ctypes.c_float(1.0),
+                                  fake, 8, fake, fake, fake, fake, need, None) == -2
     # empty problems are a no-op
     assert L.dsa_topk(fake, 0, 4, 4, 0, 4, fake, None) == 0
 
@@ -94,3 +105,10 @@ def test_workspace_sizes(dsa):
     # warm-up target: T * H rows of fp32 logits, S rounded up to 4
     assert L.dsa_attention_probs_workspace_size(2048, 2048, 128) == 2048 * 128 * 2048 * 4
     assert L.dsa_attention_probs_workspace_size(3, 10, 2) == 3 * 2 * 12 * 4
+    # warm-up backward: fp32 products, three bf16 pieces per coefficient, bf16
+    # copies of q and k with their transposes, split-K partials of dk
+    R, S = 2048 * 64, 2048
+    parts = [4 * R * S, 2 * 3 * R * S, 2 * R * 128, 2 * R * 128, 2 * S * 128, 2 * S * 128,
+             4 * 9 * S * 128]
+    assert L.dsa_indexer_backward_workspace_size(2048, 2048, 64) == sum(parts)
+    assert L.dsa_indexer_backward_workspace_size(4, 8, 3) == 0

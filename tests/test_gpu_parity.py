@@ -405,9 +405,12 @@ def test_warmup_target_kl_and_backward(dsa):
         np.testing.assert_allclose(got.cpu().double().numpy(), ref, rtol=0, atol=1e-4 * mag)
 
 
-@pytest.mark.parametrize("T,S,q_pos0,Hi", [(37, 300, 263, 64), (64, 64, 0, 1)])
+@pytest.mark.parametrize("T,S,q_pos0,Hi", [(37, 300, 263, 64), (64, 64, 0, 1), (40, 300, 0, 8),
+                                           (150, 1000, 850, 16)])
 def test_warmup_backward_offset_rows(dsa, T, S, q_pos0, Hi):
-    """Backward for a chunk of rows at an offset (keys 0 .. q_pos0 + t) and for one head."""
+    """Backward for a chunk of rows at an offset (keys 0 .. q_pos0 + t), for one head, and
+    for keys no row sees (S past the last row's position): several GEMM tiles, split-K
+    steps and a ragged tail in each product."""
     rng = np.random.default_rng(T + S + Hi)
     q8 = torch.from_numpy(rng.integers(-8, 9, size=(T, Hi, 128))).float().to(
         torch.float8_e4m3fn).view(torch.uint8)
