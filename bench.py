@@ -522,7 +522,20 @@ def oracle_sample(inp, n_rows=32, threads=None):
     return dict(value=len(rows) / wall, unit="tokens/s", cores=threads, kind="oracle",
                 sample=f"{len(rows)} query rows of the L={T} prefill, evenly spaced in t "
                        f"(incl. the last), whole path per row, {threads} threads; "
-                       f"{wall:.1f} s wall", wall_s=wall)
+                       f"{wall:.1f} s wall", wall_s=wall, cpu_model=cpu_model(),
+                host_cpus=os.cpu_count())
+
+
+def cpu_model():
+    """The host CPU's model name, from /proc/cpuinfo (None where it is absent)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 # ------------------------------------------------------------------- main
@@ -617,6 +630,20 @@ def main():
             "sparse_mla": {"ms": dres["sparse_mla"], "bound": "hbm", "achieved": mla_gbs,
                            "peak": pk["hbm"], "unit": "GB/s", "frac": mla_gbs / pk["hbm"]},
             "indexer_topk_ms": dres["total"] - dres["sparse_mla"]}
+        # decode is HBM-bound in both stages: the indexer's algorithmic bytes (the
+        # visible k8 rows, scales, q8, w, idx out) and the MLA's (selected rows, q, out,
+        # lse), each at the measured copy bandwidth, or its flops at the tensor peak
+        it_ms = dres["total"] - dres["sparse_mla"]
+        t_idx = max(dwork["idx_bytes"] / (pk["hbm"] * 1e9), dwork["idx_flops"] / (fp8_sus * 1e12))
+        t_mla = max(dwork["mla_bytes"] / (pk["hbm"] * 1e9),
+                    dwork["mla_flops"] / (pk["bf16_sus"] * 1e12))
+        line["decode"]["indexer_topk"] = {
+            "ms": it_ms, "bound": "hbm", "unit": "GB/s",
+            "achieved": dwork["idx_bytes"] / (it_ms * 1e-3) / 1e9, "peak": pk["hbm"],
+            "frac": 1e3 * t_idx / it_ms,
+            "note": "indexer + top-k timed together, against the indexer's algorithmic bytes"}
+        line["decode"]["end_to_end_roofline"] = {"ms": 1e3 * (t_idx + t_mla),
+                                                 "frac": 1e3 * (t_idx + t_mla) / dres["total"]}
     if args.next:
         line["next"] = time_next(dsa)
     if not args.no_e2e:
