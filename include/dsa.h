@@ -147,7 +147,8 @@ int dsa_sparse_mla_fwd(const void *q, const void *kv, const int32_t *idx,
  * head gets a weight a_h, a linear map of the same hidden state. The outputs
  * are the FP8 inputs dsa_indexer_scores takes.
  *
- *   h       [T][d] bf16 hidden states, d a multiple of 8
+ *   h       [T][d] bf16 hidden states, d a multiple of 8; T at most
+ *           65535 * 128 (the GEMM's row tiles)
  *   wt      [Hi*128 + 128 + Hi][d] bf16: the rows of W_Q (Hi heads x 128),
  *           then W_K (128), then W_a (Hi), each row one output's weights
  *   rope    [T][64][2] fp32 (cos, sin) of each token's position for the 64
@@ -186,7 +187,7 @@ int dsa_project_indexer_inputs(const void *h, const void *wt, const float *rope,
  *   sets covering every causal key (dsa_window_indices with window >= S);
  *   p [T][ldp] fp32 out. The logits q . kv go through a tensor-core GEMM into
  *   the caller's workspace of dsa_attention_probs_workspace_size(T, S, H)
- *   bytes (T * H rows of S fp32, S rounded up to 4).
+ *   bytes (T * H rows of S fp32, S rounded up to 4); T * H at most 65535 * 128.
  * dsa_indexer_kl:
  *   loss[t] = sum_s p[t][s] (log p[t][s] - log r[t][s]), r = softmax(I[t, :]);
  *   grad[t][s] = r[t][s] - p[t][s] (dloss/dI), 0 past the row's keys.
@@ -201,7 +202,7 @@ int dsa_project_indexer_inputs(const void *h, const void *wt, const float *rope,
  *   core GEMMs through the caller's workspace of
  *   dsa_indexer_backward_workspace_size(T, S, Hi) bytes, about
  *   T * Hi * S * 10 bytes (keep T * Hi * S near 2^28 or below by chunking the
- *   rows); T * Hi and S at most 2^23.
+ *   rows); T * Hi and S at most 65535 * 128 (the GEMM's row tiles).
  * Each returns DSA_ERR_INVALID_ARG (nothing launched) on bad arguments,
  * DSA_ERR_WORKSPACE for a missing or short workspace, and
  * DSA_ERR_UNSUPPORTED for an indexer head count outside {1, 2, 4, ..., 64}.

@@ -53,6 +53,9 @@ EncodeTiledFn encode_tiled() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// The tcgen05 GEMM tiles its M rows 128 to a CTA along grid.y (at most 65535).
+constexpr long long kMaxGemmRows = 65535ll * 128;
+
 thread_local char g_last_error[256] = "";
 
 int status_of(cudaError_t e) {
@@ -225,8 +228,8 @@ int dsa_project_indexer_inputs(const void* h, const void* wt, const float* rope,
                                int Hi, void* q8, float* q_scale, void* k8, float* k_scale, float* a,
                                void* workspace, size_t ws_bytes, dsa_stream_t stream) {
   if (!h || !wt || !rope || !q8 || !q_scale || !k8 || !k_scale || !a || T < 0 || d < 8 ||
-      (d & 7) || !aligned16(h) || !aligned16(wt) || !aligned16(rope) || !aligned16(q8) ||
-      !aligned16(k8) || !aligned16(a))
+      (d & 7) || T > kMaxGemmRows || !aligned16(h) || !aligned16(wt) || !aligned16(rope) ||
+      !aligned16(q8) || !aligned16(k8) || !aligned16(a))
     return DSA_ERR_INVALID_ARG;
   if (!valid_hi(Hi)) return DSA_ERR_UNSUPPORTED;
   if (T == 0) return DSA_OK;
@@ -265,7 +268,7 @@ int dsa_attention_probs_mean(const void* q, const void* kv, const float* lse, in
                              void* workspace, size_t ws_bytes, dsa_stream_t stream) {
   if (!q || !kv || !lse || !p || T < 0 || S <= 0 || q_pos0 < 0 || H < 1 || H > 128 ||
       ldp < S || !(sm_scale > 0.f) || !aligned16(q) || !aligned16(kv) ||
-      static_cast<long long>(T) * H > (1ll << 30))
+      static_cast<long long>(T) * H > kMaxGemmRows)
     return DSA_ERR_INVALID_ARG;
   if (T == 0) return DSA_OK;
   const size_t need = dsa_attention_probs_workspace_size(T, S, H);
@@ -297,7 +300,7 @@ int dsa_indexer_backward(const void* q8, const float* q_scale, const void* k8, c
                          void* workspace, size_t ws_bytes, dsa_stream_t stream) {
   if (!q8 || !k8 || !w || !grad || !dq || !dk || !dw || T < 0 || S <= 0 || q_pos0 < 0 ||
       ldg < S || !(scale > 0.f) || !aligned16(dq) || !aligned16(dk) ||
-      S > (1 << 23) || static_cast<long long>(T) * Hi > (1ll << 23))
+      S > kMaxGemmRows || static_cast<long long>(T) * Hi > kMaxGemmRows)
     return DSA_ERR_INVALID_ARG;
   if (!valid_hi(Hi)) return DSA_ERR_UNSUPPORTED;
   if (T == 0) return DSA_OK;

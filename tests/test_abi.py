@@ -87,6 +87,18 @@ def test_host_validation_rejects_before_launch(dsa):
                                   need, None) == -1
     assert L.dsa_indexer_backward(fake, None, fake, None, fake, 4, 8, 3, 0, ctypes.c_float(1.0),
                                   fake, 8, fake, fake, fake, fake, need, None) == -2
+    # GEMM row tiles: at most 65535 tiles of 128 rows
+    big = 65535 * 128
+    assert L.dsa_project_indexer_inputs(fake, fake, fake, big + 1, 64, 4, fake, fake, fake, fake,
+                                        fake, fake, 1 << 40, None) == -1
+    assert L.dsa_attention_probs_mean(fake, fake, fake, big // 2 + 1, 8, 2, 0,
+                                      ctypes.c_float(0.1), fake, 8, fake, 1 << 40, None) == -1
+    assert L.dsa_indexer_backward(fake, None, fake, None, fake, big // 4 + 1, 8, 4, 0,
+                                  ctypes.c_float(1.0), fake, 8, fake, fake, fake, fake, 1 << 40,
+                                  None) == -1
+    assert L.dsa_indexer_backward(fake, None, fake, None, fake, 4, big + 1, 4, 0,
+                                  ctypes.c_float(1.0), fake, big + 1, fake, fake, fake, fake,
+                                  1 << 40, None) == -1
     # empty problems are a no-op
     assert L.dsa_topk(fake, 0, 4, 4, 0, 4, fake, None) == 0
 
