@@ -146,8 +146,9 @@ int run_indexer(const void* q8, const float* q_scale, const void* k8, const floa
 }
 
 int run_topk(const float* scores, int rows, int S, int64_t ld, int q_pos0, const int* seq_len,
-             int nq, int k, int32_t* idx, cudaStream_t st) {
+             int nq, int k, int32_t* idx, cudaStream_t st, bool narrow = false) {
   TopkArgs a;
+  a.narrow = narrow;
   a.scores = scores;
   a.ld = ld;
   a.rows = rows;
@@ -401,7 +402,7 @@ int dsa_forward(const void* q8, const float* q_scale, const void* k8, const floa
                 void* out, float* lse, void* workspace, size_t ws_bytes, dsa_stream_t stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (!q8 || !k8 || !w || !q || !kv || !out || T < 0 || S < 0 || q_pos0 < 0 || k <= 0 ||
-      (k & 3) || !(scale > 0.f) || !(sm_scale > 0.f))
+      k > 65536 || (k & 3) || !(scale > 0.f) || !(sm_scale > 0.f))
     return DSA_ERR_INVALID_ARG;
   if (!valid_hi(Hi)) return DSA_ERR_UNSUPPORTED;
   if (H < 1 || H > 128) return DSA_ERR_UNSUPPORTED;
@@ -427,9 +428,12 @@ int dsa_forward(const void* q8, const float* q_scale, const void* k8, const floa
                               w + static_cast<size_t>(c0) * Hi, n, S, Hi, q_pos0 + c0, scale, sc,
                               ld, stream);
   };
-  auto topk_chunk = [&](int c0, float* sc, cudaStream_t on) {
+  // beside the next chunk's indexer, the selection runs in the narrow CTAs
+  // that fit on an SM next to an indexer CTA
+  auto topk_chunk = [&](int c0, float* sc, cudaStream_t on, bool beside) {
     const int n = std::min(rows, T - c0);
-    return dsa_topk(sc, n, S, ld, q_pos0 + c0, k, idx + static_cast<size_t>(c0) * k, on);
+    return run_topk(sc, n, S, ld, q_pos0 + c0, nullptr, 1, k,
+                    idx + static_cast<size_t>(c0) * k, on, beside);
   };
   std::unique_lock<std::mutex> lock(g_overlap_mu);
   Overlap* ov = nbuf == 2 ? overlap_for_current_device() : nullptr;
@@ -438,7 +442,7 @@ int dsa_forward(const void* q8, const float* q_scale, const void* k8, const floa
     for (int c0 = 0; c0 < T; c0 += rows) {
       int s = indexer_chunk(c0, scores[0]);
       if (s != DSA_OK) return s;
-      s = topk_chunk(c0, scores[0], st);
+      s = topk_chunk(c0, scores[0], st, false);
       if (s != DSA_OK) return s;
     }
     return dsa_sparse_mla_fwd(q, kv, idx, T, S, H, k, sm_scale, out, lse, st);
@@ -457,7 +461,7 @@ int dsa_forward(const void* q8, const float* q_scale, const void* k8, const floa
     if ((e = cudaEventRecord(ov->idx_done[b], st)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(ov->side, ov->idx_done[b], 0)) != cudaSuccess)
       return status_of(e);
-    s = topk_chunk(c0, scores[b], ov->side);
+    s = topk_chunk(c0, scores[b], ov->side, true);
     if (s != DSA_OK) return s;
     if ((e = cudaEventRecord(ov->topk_done[b], ov->side)) != cudaSuccess) return status_of(e);
   }

@@ -37,6 +37,7 @@ struct TopkArgs {
   int nq = 1;
   int* idx = nullptr;
   unsigned* err = nullptr;
+  bool narrow = false;                    // 256-thread CTAs (beside the indexer)
 };
 
 struct ProjArgs {

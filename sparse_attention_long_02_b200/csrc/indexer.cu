@@ -46,7 +46,7 @@ struct IdxSmem {
 };
 
 template <int HI, bool PAGED>
-__global__ void __launch_bounds__(kIdxThreads, 1)
+__global__ void __maxnreg__(128)
 indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const IndexerArgs a) {
   constexpr int QB = (256 / HI) < 64 ? (256 / HI) : 64;   // queries per CTA (prefill)
@@ -284,6 +284,10 @@ cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const Index
   auto kern = indexer_kernel<HI, PAGED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
+  // the whole shared carveout, so a top-k CTA fits beside this one
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   kern<<<grid, kIdxThreads, smem, st>>>(tq, tk, a);
   return cudaGetLastError();
