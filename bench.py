@@ -186,7 +186,7 @@ def decode_work(lens, nq, Hi, H, k):
 # DRAM bytes (read + write) per launch of the current kernels at the full 128K prefill, from
 # one-pass ncu captures (dram__bytes_read.sum + dram__bytes_write.sum): the sparse MLA's one
 # launch, and the mean of the indexer's 32 chunk launches. Reset to None when a kernel changes.
-NCU_TRAFFIC = {"sparse_mla": 62.05e9 + 17.24e9, "indexer": None}
+NCU_TRAFFIC = {"sparse_mla": 62.05e9 + 17.24e9, "indexer": 0.1654e9 + 1.0175e9}
 
 
 def peaks():
