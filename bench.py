@@ -53,6 +53,10 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--next", action="store_true",
                     help="also time dense causal and sliding-window attention beside DSA at 16K")
+    ap.add_argument("--shard", default="problems", choices=["problems", "rows"],
+                    help="problems: one prefill per GPU (weak scaling, the default); rows: one "
+                         "prefill's query rows split over the GPUs by causal cost (strong "
+                         "scaling)")
     return ap.parse_args()
 
 
@@ -257,6 +261,37 @@ class Prefill:
             e1.synchronize()
             tot["sparse_mla"] += e0.elapsed_time(e1)
         return {s: v / reps for s, v in tot.items()}
+
+
+class RowShard:
+    """This rank's share of one prefill: whole chunks of rows, balanced over the
+    ranks by causal cost (dsa_plan_prefill_chunks; every rank computes the same
+    plan), each run as its own dsa_forward over the key prefix its rows see.
+    The caches are whole on every GPU; no data crosses between GPUs."""
+
+    def __init__(self, dsa, cfg, inp, world, rank):
+        self.dsa, self.inp = dsa, inp
+        T, H, k = inp["T"], inp["H"], inp["k"]
+        self.chunk = cfg.chunk or T
+        self.starts = dsa.plan_prefill_chunks(T, inp["S"], inp["Hi"], H, k, self.chunk, world,
+                                              rank)
+        self.ws = torch.empty(dsa.forward_workspace_size(self.chunk, inp["S"], inp["Hi"], H, k),
+                              dtype=torch.uint8, device="cuda")
+        self.out = torch.empty(T, H, 512, dtype=torch.bfloat16, device="cuda")
+        self.lse = torch.empty(T, H, dtype=torch.float32, device="cuda")
+        self.idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+        self.launches = 3 * len(self.starts)       # indexer, top-k, sparse MLA per chunk
+        self.rows = sum(min(self.chunk, T - c0) for c0 in self.starts)
+
+    def step(self):
+        i = self.inp
+        cut = lambda x, a, b: None if x is None else x[a:b]
+        for c0 in self.starts:
+            e = min(c0 + self.chunk, i["T"])
+            self.dsa.forward(i["q8"][c0:e], cut(i["q_scale"], c0, e), i["k8"][:e],
+                             cut(i["k_scale"], 0, e), i["w"][c0:e], i["q"][c0:e], i["kv"][:e],
+                             i["k"], i["scale"], i["sm_scale"], q_pos0=c0, idx=self.idx[c0:e],
+                             out=self.out[c0:e], lse=self.lse[c0:e], workspace=self.ws)
 
 
 def time_steps(fn, steps, warmup, ranks, dsa, clock_gpu):
@@ -581,11 +616,22 @@ def main():
     import sparse_attention_long_02_b200 as dsa
     pk = peaks()
     fp8_sus = 2 * pk["bf16_sus"]
-    cfg, inp = prefill_inputs(args.L or W.CONFIGS[PREFILL_CFG].L, ranks.rank)
+    rows_mode = args.shard == "rows"
+    # rows: every rank holds the same prefill and runs its share of the rows
+    cfg, inp = prefill_inputs(args.L or W.CONFIGS[PREFILL_CFG].L, 0 if rows_mode else ranks.rank)
     L = inp["T"]
-    pf = Prefill(dsa, cfg, inp)
-    ms, clocks = time_steps(pf.step, args.steps, args.warmup, ranks, dsa, ranks.local)
-    tokens = L * ranks.world
+    shard = None
+    if rows_mode:
+        shard = RowShard(dsa, cfg, inp, ranks.world, ranks.rank)
+        ms, clocks = time_steps(shard.step, args.steps, args.warmup, ranks, dsa, ranks.local)
+        tokens = L
+        del shard.ws, shard.out, shard.lse, shard.idx
+        torch.cuda.empty_cache()
+        pf = Prefill(dsa, cfg, inp)
+    else:
+        pf = Prefill(dsa, cfg, inp)
+        ms, clocks = time_steps(pf.step, args.steps, args.warmup, ranks, dsa, ranks.local)
+        tokens = L * ranks.world
     value = tokens / (ms / 1e3)
 
     work = prefill_work(L, inp["Hi"], inp["H"], inp["k"])
@@ -612,12 +658,18 @@ def main():
     t_roof = max(work["idx_flops"] / (fp8_sus * 1e12), work["idx_bytes"] / (pk["hbm"] * 1e9)) + \
         max(work["mla_flops"] / (pk["bf16_sus"] * 1e12), work["mla_bytes"] / (pk["hbm"] * 1e9))
 
+    config = config_obj(L, pf.chunk)
+    if rows_mode:
+        config["shard"] = (f"rows: the {math.ceil(L / pf.chunk)} chunks of one prefill over "
+                           f"{ranks.world} GPU(s) by causal cost; rank 0 runs "
+                           f"{len(shard.starts)} chunks ({shard.rows} rows)")
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ranks.world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True, "scaling": "strong" if rows_mode else "weak",
+            "vs_baseline": None,
             "dtype": "fp8 indexer / bf16 MLA, fp32 accumulate", "data": "synthetic",
-            "config": config_obj(L, pf.chunk), "clocks": clocks,
-            "gpu_launches": pf.launches * args.steps,
+            "config": config, "clocks": clocks,
+            "gpu_launches": (shard.launches if rows_mode else pf.launches) * args.steps,
             "roofline": roof, "stages": stages,
             "end_to_end_roofline": {"ms": 1e3 * t_roof, "frac": 1e3 * t_roof / ms}}
     if not args.no_decode:
@@ -646,7 +698,7 @@ def main():
                                                  "frac": 1e3 * (t_idx + t_mla) / dres["total"]}
     if args.next:
         line["next"] = time_next(dsa)
-    if not args.no_e2e:
+    if not args.no_e2e and not rows_mode:       # e2e: the default mode's whole prefill per GPU
         e_ms, h2d, d2h = e2e_prefill(pf, max(1, min(args.steps, 3)))
         line["e2e"] = {"value": tokens / (ranks.max(e_ms) / 1e3), "unit": "tokens/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}

@@ -340,6 +340,37 @@ int dsa_sparse_mla_decode_paged(const void *q, const void *kv_pool,
                                 int k, float sm_scale, void *out, float *lse,
                                 dsa_stream_t stream);
 
+/*
+ * Splitting the work over several GPUs (host only: no CUDA call, nothing
+ * launched). The pages describe no distributed step; every prefill row and
+ * every decode sequence is independent given the caches, which each GPU
+ * holds whole. The causal prefix makes a row's cost grow with its position,
+ * so units are balanced by estimated cost (BF16-flop equivalents of one row
+ * seeing n keys: 128*Hi*n for the FP8 indexer at twice the BF16 rate, plus
+ * 2176*H*min(n, k) for the sparse MLA) with the longest-first greedy rule:
+ * units by cost, largest first (ties: lower unit), each to the least-loaded
+ * worker so far (ties: lower worker). Every worker computes the same plan,
+ * so the call needs no communication; the parts are disjoint and together
+ * cover every unit.
+ *
+ * dsa_plan_prefill_chunks: the prefill's rows 0 .. T-1 (row t at position
+ *   q_pos0 + t, seeing keys 0 .. min(q_pos0 + t, S - 1)) in chunks of `chunk`
+ *   rows; writes the first rows of worker `part`'s chunks (ascending) to
+ *   first_rows and returns how many. Chunk c covers rows
+ *   [c*chunk, min((c+1)*chunk, T)); each runs as its own dsa_forward with
+ *   q_pos0 + c*chunk.
+ * dsa_plan_decode_sequences: the B sequences of a decode batch (nq queries
+ *   each, query j seeing seq_len[b] - nq + j + 1 keys); writes worker `part`'s
+ *   sequence numbers (ascending) to seqs and returns how many.
+ * Both return DSA_ERR_INVALID_ARG for bad sizes, 1 <= parts <= 4096 and
+ * 0 <= part < parts violated, seq_len[b] < nq, or an output array shorter
+ * than the worker's share (max_chunks / max_seqs entries).
+ */
+int dsa_plan_prefill_chunks(int T, int S, int q_pos0, int Hi, int H, int k, int chunk,
+                            int parts, int part, int32_t *first_rows, int max_chunks);
+int dsa_plan_decode_sequences(const int32_t *seq_len, int B, int nq, int Hi, int H, int k,
+                              int parts, int part, int32_t *seqs, int max_seqs);
+
 #ifdef __cplusplus
 }
 #endif

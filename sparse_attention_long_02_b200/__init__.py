@@ -58,6 +58,8 @@ _sig("dsa_decode_paged", I32, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32
      F32, F32, P, P, P, P, SZ, P)
 _sig("dsa_decode_paged_noalloc", I32, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32,
      I32, F32, F32, P, P, P, P)
+_sig("dsa_plan_prefill_chunks", I32, I32, I32, I32, I32, I32, I32, I32, I32, I32, P, I32)
+_sig("dsa_plan_decode_sequences", I32, P, I32, I32, I32, I32, I32, I32, I32, P, I32)
 _sig("dsa_sparse_mla_decode_paged", I32, P, P, P, P, P, I32, I32, I32, I32, I32, I32, F32, P,
      P, P)
 
@@ -373,3 +375,25 @@ def decode_paged_noalloc(q8, q_scale, w, q, k8_pool, k_scale_pool, kv_pool, bloc
                                          float(scale), float(sm_scale), _p(idx), _p(out), _p(lse),
                                          _stream(stream)), "dsa_decode_paged_noalloc")
     return out, lse, idx
+
+
+def plan_prefill_chunks(T, S, Hi, H, k, chunk, parts, part, q_pos0=0):
+    """First rows of worker `part`'s chunks of a T-row prefill split over `parts`
+    workers, balanced by causal cost (host only)."""
+    nch = max(1, (T + chunk - 1) // chunk)
+    out = (ctypes.c_int32 * nch)()
+    n = _lib.dsa_plan_prefill_chunks(T, S, q_pos0, Hi, H, k, chunk, parts, part, out, nch)
+    _check(min(n, 0), "dsa_plan_prefill_chunks")
+    return list(out[:n])
+
+
+def plan_decode_sequences(seq_len, nq, Hi, H, k, parts, part):
+    """Sequence numbers of worker `part`'s share of a decode batch, balanced by
+    context length (host only)."""
+    lens = [int(x) for x in (seq_len.tolist() if hasattr(seq_len, "tolist") else seq_len)]
+    B = len(lens)
+    arr = (ctypes.c_int32 * max(1, B))(*lens)
+    out = (ctypes.c_int32 * max(1, B))()
+    n = _lib.dsa_plan_decode_sequences(arr, B, nq, Hi, H, k, parts, part, out, max(1, B))
+    _check(min(n, 0), "dsa_plan_decode_sequences")
+    return list(out[:n])

@@ -5,6 +5,7 @@ import importlib.util
 import os
 import re
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -124,3 +125,69 @@ def test_workspace_sizes(dsa):
              4 * 9 * S * 128]
     assert L.dsa_indexer_backward_workspace_size(2048, 2048, 64) == sum(parts)
     assert L.dsa_indexer_backward_workspace_size(4, 8, 3) == 0
+
+
+def _row_cost(n, Hi, H, k):
+    """Cost of one query row seeing n keys: FP8 indexer flops at half weight plus MLA flops."""
+    return 128 * Hi * n + 2176 * H * min(n, k)
+
+
+@pytest.mark.parametrize("T,S,q_pos0,chunk,parts", [(131072, 131072, 0, 4096, 2),
+                                                    (131072, 131072, 0, 4096, 8),
+                                                    (10000, 20000, 7000, 999, 3),
+                                                    (5, 5, 0, 4096, 4)])
+def test_prefill_plan_covers_every_chunk_once_and_balances(dsa, T, S, q_pos0, chunk, parts):
+    Hi, H, k = 64, 128, 2048
+    plans = [dsa.plan_prefill_chunks(T, S, Hi, H, k, chunk, parts, p, q_pos0=q_pos0)
+             for p in range(parts)]
+    got = sorted(c for plan in plans for c in plan)
+    assert got == list(range(0, T, chunk))                 # disjoint and complete
+    for plan in plans:
+        assert plan == sorted(plan)
+
+    def chunk_cost(c0):
+        return sum(_row_cost(min(q_pos0 + t, S - 1) + 1, Hi, H, k)
+                   for t in range(c0, min(c0 + chunk, T)))
+
+    costs = {c0: chunk_cost(c0) for c0 in got}
+    loads = [sum(costs[c] for c in plan) for plan in plans]
+    # longest-first greedy: the heaviest worker exceeds the mean by at most one unit
+    assert max(loads) <= sum(loads) / parts + max(costs.values()) + 1e-6
+    # an idle worker only where there are fewer chunks than workers
+    assert min(len(p) for p in plans) >= (1 if len(got) >= parts else 0)
+
+
+def test_prefill_plan_is_the_longest_first_rule(dsa):
+    # three chunks of one row each at positions 0, 1, 2 over two workers: the
+    # costliest (row 2) goes to worker 0, then row 1 to worker 1, then row 0 to
+    # worker 1 (the lighter one)
+    assert dsa.plan_prefill_chunks(3, 3, 1, 1, 2048, 1, 2, 0) == [2]
+    assert dsa.plan_prefill_chunks(3, 3, 1, 1, 2048, 1, 2, 1) == [0, 1]
+    # one worker takes every chunk in order
+    assert dsa.plan_prefill_chunks(9, 9, 1, 1, 4, 2, 1, 0) == [0, 2, 4, 6, 8]
+
+
+def test_decode_plan_balances_by_context(dsa):
+    rng = np.random.default_rng(5)
+    lens = np.exp(rng.uniform(np.log(512), np.log(131072), 128)).astype(np.int32)
+    Hi, H, k, nq, parts = 64, 128, 2048, 2, 4
+    plans = [dsa.plan_decode_sequences(lens, nq, Hi, H, k, parts, p) for p in range(parts)]
+    assert sorted(b for plan in plans for b in plan) == list(range(128))
+    cost = [sum(_row_cost(int(n) - nq + j + 1, Hi, H, k) for j in range(nq)) for n in lens]
+    loads = [sum(cost[b] for b in plan) for plan in plans]
+    assert max(loads) <= sum(loads) / parts + max(cost) + 1e-6
+
+
+def test_plan_rejects_bad_arguments(dsa):
+    L = dsa.lib()
+    out = (ctypes.c_int32 * 8)()
+    assert L.dsa_plan_prefill_chunks(16, 16, 0, 4, 8, 4, 4, 0, 0, out, 8) == -1    # parts 0
+    assert L.dsa_plan_prefill_chunks(16, 16, 0, 4, 8, 4, 4, 2, 2, out, 8) == -1    # part >= parts
+    assert L.dsa_plan_prefill_chunks(16, 16, 0, 4, 8, 4, 0, 1, 0, out, 8) == -1    # chunk 0
+    assert L.dsa_plan_prefill_chunks(16, 16, 0, 4, 8, 4, 4, 1, 0, out, 3) == -1    # out too short
+    assert L.dsa_plan_prefill_chunks(16, 16, 0, 4, 8, 4, 4, 1, 0, None, 8) == -1
+    assert L.dsa_plan_prefill_chunks(16, 16, 0, 4, 8, 4, 4, 1, 0, out, 8) == 4
+    lens = (ctypes.c_int32 * 2)(1, 9)
+    assert L.dsa_plan_decode_sequences(lens, 2, 2, 4, 8, 4, 1, 0, out, 8) == -1   # seq_len < nq
+    assert L.dsa_plan_decode_sequences(None, 2, 1, 4, 8, 4, 1, 0, out, 8) == -1
+    assert L.dsa_plan_decode_sequences(lens, 2, 1, 4, 8, 4, 1, 0, out, 8) == 2

@@ -83,3 +83,46 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert p.exitcode == 0
     rank, out = q.get(timeout=5)
     assert rank == 1 and out == ""
+
+
+def _plan_rank(rank, world, port, q):
+    os.environ.update({"RANK": str(rank), "LOCAL_RANK": str(rank), "WORLD_SIZE": str(world),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    sys.path.insert(0, ROOT)
+    import torch
+    import torch.distributed as dist
+    import bench
+    import sparse_attention_long_02_b200 as dsa
+    ranks = bench.Ranks(world, backend="gloo")
+    L, chunk = 131072, 4096
+    mine = dsa.plan_prefill_chunks(L, L, 64, 128, 2048, chunk, ranks.world, ranks.rank)
+    # every rank's share, gathered: the plan needs no communication, so the
+    # shares must tile the rows without overlap
+    buf = torch.full((L // chunk,), -1, dtype=torch.int64)
+    buf[:len(mine)] = torch.tensor(mine, dtype=torch.int64)
+    parts = [torch.empty_like(buf) for _ in range(world)]
+    dist.all_gather(parts, buf)
+    # rows each rank runs, and the whole-job value at a per-rank time of 10 + r ms
+    rows = sum(min(chunk, L - c0) for c0 in mine)
+    t_max = ranks.max(10.0 + rank)
+    ranks.close()
+    q.put((rank, [p[p >= 0].tolist() for p in parts], rows, t_max))
+
+
+def test_row_shards_tile_one_prefill_over_two_ranks():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_plan_rank, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=5) for _ in range(world))
+    assert res[0][1] == res[1][1]                       # both ranks see the same plan
+    shares = res[0][1]
+    assert sorted(c for s in shares for c in s) == list(range(0, 131072, 4096))
+    assert res[0][2] + res[1][2] == 131072              # all rows, once
+    # strong scaling: one prefill's tokens over the slowest rank's time
+    assert res[0][3] == res[1][3] == 11.0
