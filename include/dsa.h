@@ -265,6 +265,35 @@ int dsa_forward(const void *q8, const float *q_scale, const void *k8,
                 dsa_stream_t stream);
 
 /*
+ * The same prefill with the top-k fused into the indexer, so no score row
+ * reaches HBM: same arguments, layouts and results as dsa_forward (the
+ * selection is the k largest scores, ties to the smaller key). Per chunk of
+ * `chunk` rows:
+ *  - the indexer scores each row against a sample of the keys (the first 256
+ *    of every 4096, copied into the workspace);
+ *  - per row, a threshold from its sampled scores with, in expectation, about
+ *    1.4 k of its keys at or above it;
+ *  - the indexer runs again over every key, appending only the (key, score)
+ *    pairs at or above the threshold to the row's candidate list;
+ *  - with k to 4096 candidates the k largest are among them and are chosen
+ *    exactly; any other row (rare) has its scores recomputed on CUDA cores
+ *    and selected in full.
+ * The workspace, dsa_forward_fused_workspace_size(...) bytes (0: not
+ * supported), holds the sample, the candidate lists and one scratch score
+ * row per recompute CTA: about 1.4 GB at T = S = 131072 with 4096-row chunks
+ * and k = 2048 (idx included), against 5.4 GB for dsa_forward.
+ * Supports k <= 2048 and S <= 131072 (DSA_ERR_UNSUPPORTED otherwise); q8 and
+ * k8 16-byte aligned; the workspace 256-byte aligned.
+ */
+size_t dsa_forward_fused_workspace_size(int T, int S, int Hi, int H, int k, int chunk);
+int dsa_forward_fused(const void *q8, const float *q_scale, const void *k8,
+                      const float *k_scale, const float *w, const void *q,
+                      const void *kv, int T, int S, int Hi, int H, int q_pos0, int k,
+                      int chunk, float scale, float sm_scale, int32_t *idx_out,
+                      void *out, float *lse, void *workspace, size_t ws_bytes,
+                      dsa_stream_t stream);
+
+/*
  * Batched decode over a paged cache (blocks of 64 tokens).
  *
  *   q8 [B][nq][Hi][128] e4m3, q_scale [B][nq] fp32 (or NULL), w [B][nq][Hi]

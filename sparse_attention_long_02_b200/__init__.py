@@ -51,6 +51,9 @@ _sig("dsa_indexer_backward", I32, P, P, P, P, P, I32, I32, I32, I32, F32, P, I64
      P)
 _sig("dsa_project_indexer_inputs", I32, P, P, P, I32, I32, I32, P, P, P, P, P, P, SZ, P)
 _sig("dsa_forward_workspace_size", SZ, I32, I32, I32, I32, I32, I32)
+_sig("dsa_forward_fused_workspace_size", SZ, I32, I32, I32, I32, I32, I32)
+_sig("dsa_forward_fused", I32, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, F32, F32,
+     P, P, P, P, SZ, P)
 _sig("dsa_forward", I32, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, F32, F32,
      P, P, P, P, SZ, P)
 _sig("dsa_decode_paged_workspace_size", SZ, I32, I32, I32, I32, I32, I32)
@@ -290,6 +293,36 @@ def forward(q8, q_scale, k8, k_scale, w, q, kv, k, scale, sm_scale, q_pos0=0, ch
                             _p(kv), T, S, Hi, H, q_pos0, k, chunk, float(scale), float(sm_scale),
                             _p(idx), _p(out), _p(lse), _p(workspace), workspace.numel(),
                             _stream(stream)), "dsa_forward")
+    return out, lse, idx
+
+
+def forward_fused_workspace_size(T, S, Hi, H, k, chunk=0) -> int:
+    return int(_lib.dsa_forward_fused_workspace_size(T, S, Hi, H, k, chunk))
+
+
+def forward_fused(q8, q_scale, k8, k_scale, w, q, kv, k, scale, sm_scale, q_pos0=0, chunk=0,
+                  idx=None, out=None, lse=None, workspace=None, return_idx=True, stream=None):
+    """Whole prefill path with the top-k fused into the indexer (no score rows in
+    HBM) -> (out, lse, idx or None); the same results as forward()."""
+    q8, k8 = _u8(q8), _u8(k8)
+    q, kv = _dev(q, torch.bfloat16), _dev(kv, torch.bfloat16)
+    T, Hi = q8.shape[0], q8.shape[1]
+    S, H = k8.shape[0], q.shape[1]
+    dev = q.device
+    if out is None:
+        out = torch.empty(T, H, 512, dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty(T, H, dtype=torch.float32, device=dev)
+    if idx is None and return_idx:
+        idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+    if workspace is None:
+        need = forward_fused_workspace_size(T, S, Hi, H, k, chunk)
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(_lib.dsa_forward_fused(_p(q8), _p(_dev(q_scale, torch.float32)), _p(k8),
+                                  _p(_dev(k_scale, torch.float32)), _p(_dev(w, torch.float32)),
+                                  _p(q), _p(kv), T, S, Hi, H, q_pos0, k, chunk, float(scale),
+                                  float(sm_scale), _p(idx), _p(out), _p(lse), _p(workspace),
+                                  workspace.numel(), _stream(stream)), "dsa_forward_fused")
     return out, lse, idx
 
 

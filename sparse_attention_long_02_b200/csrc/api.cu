@@ -385,6 +385,48 @@ int dsa_sparse_mla_decode_paged(const void* q, const void* kv_pool, const int32_
                     block_table, seq_len, max_blocks, nblk, nq, static_cast<cudaStream_t>(stream));
 }
 
+namespace {
+
+// Sampled keys (the first 256 of every 4096) among keys 0 .. S-1.
+long long sample_count(int S) {
+  const long long p = S - 1;
+  return (p >> 12) * 256 + std::min<long long>(p & 4095, 255) + 1;
+}
+
+// Workspace of the fused path, each part 256-byte aligned.
+struct FusedLayout {
+  long long M, ldm, ld;
+  size_t k8s, kss, sample, tau, cnt, ckey, cidx, fail, scratch, idx, total;
+};
+
+FusedLayout fused_layout(int T, int S, int k, int chunk) {
+  FusedLayout L;
+  const size_t rows = chunk <= 0 ? T : std::min(chunk, T);
+  L.M = sample_count(S);
+  L.ldm = static_cast<long long>(round_up(static_cast<size_t>(L.M), 4));
+  L.ld = static_cast<long long>(round_up(static_cast<size_t>(S), 4));
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += round_up(bytes, 256);
+    return o;
+  };
+  L.k8s = take(static_cast<size_t>(L.M) * 128);
+  L.kss = take(static_cast<size_t>(L.M) * 4);
+  L.sample = take(rows * L.ldm * 4);
+  L.tau = take(rows * 4);
+  L.cnt = take(rows * 4);
+  L.ckey = take(rows * kFusedCandCap * 4);
+  L.cidx = take(rows * kFusedCandCap * 4);
+  L.fail = take(4 + rows * 4);
+  L.scratch = take(static_cast<size_t>(kFusedSlots) * L.ld * 4);
+  L.idx = take(static_cast<size_t>(T) * k * 4);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
 size_t dsa_forward_workspace_size(int T, int S, int Hi, int H, int k, int chunk) {
   (void)Hi;
   (void)H;
@@ -469,6 +511,131 @@ int dsa_forward(const void* q8, const float* q_scale, const void* k8, const floa
     if ((e = cudaStreamWaitEvent(st, ov->topk_done[b], 0)) != cudaSuccess) return status_of(e);
   lock.unlock();
   return dsa_sparse_mla_fwd(q, kv, idx, T, S, H, k, sm_scale, out, lse, st);
+}
+
+size_t dsa_forward_fused_workspace_size(int T, int S, int Hi, int H, int k, int chunk) {
+  (void)Hi;
+  (void)H;
+  if (T <= 0 || S <= 0 || k <= 0 || k > 2048 || S > kFusedMaxS) return 0;
+  return fused_layout(T, S, k, chunk).total;
+}
+
+int dsa_forward_fused(const void* q8, const float* q_scale, const void* k8, const float* k_scale,
+                      const float* w, const void* q, const void* kv, int T, int S, int Hi, int H,
+                      int q_pos0, int k, int chunk, float scale, float sm_scale, int32_t* idx_out,
+                      void* out, float* lse, void* workspace, size_t ws_bytes,
+                      dsa_stream_t stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!q8 || !k8 || !w || !q || !kv || !out || T < 0 || S < 0 || q_pos0 < 0 || k <= 0 ||
+      (k & 3) || !(scale > 0.f) || !(sm_scale > 0.f) || !aligned16(q8) || !aligned16(k8))
+    return DSA_ERR_INVALID_ARG;
+  if (!valid_hi(Hi)) return DSA_ERR_UNSUPPORTED;
+  if (H < 1 || H > 128) return DSA_ERR_UNSUPPORTED;
+  if (k > 2048 || S > kFusedMaxS) return DSA_ERR_UNSUPPORTED;
+  if (T == 0) return DSA_OK;
+  if (S == 0) return DSA_ERR_INVALID_ARG;
+  const size_t need = dsa_forward_fused_workspace_size(T, S, Hi, H, k, chunk);
+  if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return DSA_ERR_WORKSPACE;
+  const FusedLayout L = fused_layout(T, S, k, chunk);
+  char* ws = static_cast<char*>(workspace);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
+  if (!aligned16(idx)) return DSA_ERR_INVALID_ARG;
+  unsigned* err = device_error_word();
+  if (!err) return DSA_ERR_CUDA;
+  const int rows = chunk <= 0 ? T : std::min(chunk, T);
+  // the sampled keys (the first 256 of every 4096) in a compact cache: one
+  // strided copy for the whole segments, one for the last, partial one
+  uint8_t* k8s = reinterpret_cast<uint8_t*>(ws + L.k8s);
+  float* kss = k_scale ? reinterpret_cast<float*>(ws + L.kss) : nullptr;
+  const size_t full = static_cast<size_t>(S) / 4096;
+  const size_t tail = std::min<size_t>(static_cast<size_t>(S) % 4096, 256);
+  const uint8_t* k8b = static_cast<const uint8_t*>(k8);
+  cudaError_t e = cudaSuccess;
+  if (full > 0)
+    e = cudaMemcpy2DAsync(k8s, 256 * 128, k8b, 4096 * 128, 256 * 128, full,
+                          cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess && tail > 0)
+    e = cudaMemcpyAsync(k8s + full * 256 * 128, k8b + full * 4096 * 128, tail * 128,
+                        cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess && kss && full > 0)
+    e = cudaMemcpy2DAsync(kss, 256 * 4, k_scale, 4096 * 4, 256 * 4, full,
+                          cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess && kss && tail > 0)
+    e = cudaMemcpyAsync(kss + full * 256, k_scale + full * 4096, tail * 4,
+                        cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return status_of(e);
+  for (int c0 = 0; c0 < T; c0 += rows) {
+    const int n = std::min(rows, T - c0);
+    const uint8_t* q8c = static_cast<const uint8_t*>(q8) + static_cast<size_t>(c0) * Hi * 128;
+    const float* qsc = q_scale ? q_scale + c0 : nullptr;
+    const float* wc = w + static_cast<size_t>(c0) * Hi;
+    // 1. each row's scores against the sampled keys
+    // the sampled keys the chunk's last row sees
+    const long long m_c =
+        sample_count(static_cast<int>(std::min<long long>(static_cast<long long>(q_pos0) + c0 + n,
+                                                          S)));
+    IndexerArgs a;
+    a.T = n;
+    a.S = static_cast<int>(m_c);
+    a.Hi = Hi;
+    a.q_pos0 = q_pos0 + c0;
+    a.scale = scale;
+    a.w = wc;
+    a.q_scale = qsc;
+    a.k_scale = kss;
+    a.scores = reinterpret_cast<float*>(ws + L.sample);
+    a.ld = L.ldm;
+    a.err = err;
+    e = launch_indexer(a, q8c, k8s, m_c, st);
+    // 2. the rows' thresholds
+    FusedSelArgs F;
+    F.T = n;
+    F.S = S;
+    F.q_pos0 = q_pos0 + c0;
+    F.k = k;
+    F.Hi = Hi;
+    F.scale = scale;
+    F.sample = a.scores;
+    F.ld_sample = L.ldm;
+    F.tau = reinterpret_cast<unsigned*>(ws + L.tau);
+    F.cand_count = reinterpret_cast<unsigned*>(ws + L.cnt);
+    F.cand_key = reinterpret_cast<unsigned*>(ws + L.ckey);
+    F.cand_idx = reinterpret_cast<int*>(ws + L.cidx);
+    F.cand_cap = kFusedCandCap;
+    F.fail_count = reinterpret_cast<unsigned*>(ws + L.fail);
+    F.fail_rows = reinterpret_cast<int*>(ws + L.fail) + 1;
+    F.q8 = q8c;
+    F.q_scale = qsc;
+    F.k8 = k8b;
+    F.k_scale = k_scale;
+    F.w = wc;
+    F.scratch = reinterpret_cast<float*>(ws + L.scratch);
+    F.ld = L.ld;
+    F.slots = kFusedSlots;
+    F.idx = idx + static_cast<size_t>(c0) * k;
+    F.err = err;
+    if (e == cudaSuccess) e = launch_fused_tau(F, st);
+    // 3. the filter-mode indexer: candidate lists instead of scores
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.cnt, 0, static_cast<size_t>(n) * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.fail, 0, 4, st);
+    IndexerArgs b = a;
+    b.S = S;
+    b.k_scale = k_scale;
+    b.scores = nullptr;
+    b.ld = 0;
+    b.tau = F.tau;
+    b.cand_count = reinterpret_cast<unsigned*>(ws + L.cnt);
+    b.cand_key = reinterpret_cast<unsigned*>(ws + L.ckey);
+    b.cand_idx = reinterpret_cast<int*>(ws + L.cidx);
+    b.cand_cap = kFusedCandCap;
+    if (e == cudaSuccess) e = launch_indexer(b, q8c, k8b, S, st);
+    // 4. the exact selection among the candidates; 5. the rest recomputed
+    if (e == cudaSuccess) e = launch_fused_select(F, st);
+    if (e == cudaSuccess) e = launch_fused_fallback(F, st);
+    if (e != cudaSuccess) return status_of(e);
+  }
+  return dsa_sparse_mla_fwd(q, kv, idx, T, S, H, k, sm_scale, out, lse, stream);
 }
 
 size_t dsa_decode_paged_workspace_size(int B, int nq, int max_blocks, int Hi, int H, int k) {

@@ -24,6 +24,13 @@ struct IndexerArgs {
   int max_blocks = 0, nblk = 0, nq = 1, B = 0, max_ctx = 0;
   const int* seq_len = nullptr;
   unsigned* err = nullptr;
+  // filter mode (prefill): with tau set, no scores are written; every score
+  // whose order key is >= tau[t] goes to row t's candidate list instead
+  const unsigned* tau = nullptr;          // [T] order-key thresholds
+  unsigned* cand_count = nullptr;         // [T], zero before the launch
+  unsigned* cand_key = nullptr;           // [T][cand_cap]
+  int* cand_idx = nullptr;                // [T][cand_cap]
+  int cand_cap = 0;
   // filled in by launch_indexer
   int n_mma = 0, q_box_rows = 0, tmem_cols = 0, tiles_per_cta = 0;
 };
@@ -38,6 +45,35 @@ struct TopkArgs {
   int* idx = nullptr;
   unsigned* err = nullptr;
   bool narrow = false;                    // 256-thread CTAs (beside the indexer)
+};
+
+// The prefill's selection without a score matrix in HBM: a threshold per row
+// from the scores over the sampled keys, the filter-mode indexer's candidate
+// lists, an exact select among them, and a CUDA-core recompute for the rows
+// whose candidates miss [k, cand_cap].
+struct FusedSelArgs {
+  int T = 0, S = 0, q_pos0 = 0, k = 0, Hi = 0;
+  float scale = 1.f;
+  const float* sample = nullptr;          // [T][ld_sample] scores over the sampled keys
+  long long ld_sample = 0;
+  unsigned* tau = nullptr;                // [T] order-key thresholds
+  const unsigned* cand_count = nullptr;   // [T]
+  const unsigned* cand_key = nullptr;     // [T][cand_cap]
+  const int* cand_idx = nullptr;          // [T][cand_cap]
+  int cand_cap = 0;
+  unsigned* fail_count = nullptr;         // [1], zero before the select
+  int* fail_rows = nullptr;               // [T]
+  // inputs of the recompute (rows of this call; keys of the whole cache)
+  const uint8_t* q8 = nullptr;
+  const float* q_scale = nullptr;
+  const uint8_t* k8 = nullptr;
+  const float* k_scale = nullptr;
+  const float* w = nullptr;
+  float* scratch = nullptr;               // [slots][ld] one score row per fallback CTA
+  long long ld = 0;
+  int slots = 0;
+  int* idx = nullptr;                     // [T][k] out
+  unsigned* err = nullptr;
 };
 
 struct ProjArgs {
@@ -95,6 +131,12 @@ cudaError_t make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType
 cudaError_t launch_indexer(const IndexerArgs& a, const void* q8, const void* k8, long long k_rows,
                            cudaStream_t st);
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st);
+cudaError_t launch_fused_tau(const FusedSelArgs& a, cudaStream_t st);
+cudaError_t launch_fused_select(const FusedSelArgs& a, cudaStream_t st);
+cudaError_t launch_fused_fallback(const FusedSelArgs& a, cudaStream_t st);
+constexpr int kFusedCandCap = 4096;       // candidates per row
+constexpr int kFusedSlots = 148;          // fallback CTAs (one score row each)
+constexpr int kFusedMaxS = 131072;        // longest row the fused selection takes
 cudaError_t launch_window(int T, int S, int q_pos0, int window, int k, int* idx, cudaStream_t st);
 cudaError_t launch_project(const ProjArgs& a, const void* h, const void* wt, cudaStream_t st);
 // C [M][ldc] fp32 = A [M][K] x B [N][K]^T, bf16 operands, K a multiple of 8.

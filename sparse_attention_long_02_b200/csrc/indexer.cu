@@ -26,6 +26,12 @@ namespace dsa {
 namespace {
 
 constexpr int kIdxThreads = 384;
+
+// Order-preserving 32-bit key of a float score (larger score, larger key).
+__device__ __forceinline__ uint32_t score_key(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
 constexpr int kKeyTile = 128;      // keys per MMA tile (M)
 constexpr int kStages = 4;         // key-tile ring depth
 constexpr int kKTileBytes = kKeyTile * 128;
@@ -201,6 +207,22 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       return __ldg(a.k_scale + s);
     };
     float ks_next = key_scale(g);
+    // filter mode: the last appended query's ballot and its atomic's result
+    bool pend = false, p_keep = false;
+    uint32_t p_key = 0;
+    unsigned p_ball = 0, p_base = 0;
+    long long p_t = 0;
+    int p_s = 0;
+    auto flush_pending = [&]() {
+      if (!pend) return;                           // warp-uniform
+      const unsigned base = __shfl_sync(0xffffffffu, p_base, 0);
+      const unsigned slot = base + __popc(p_ball & ((1u << lane) - 1u));
+      if (p_keep && slot < static_cast<unsigned>(a.cand_cap)) {
+        a.cand_key[p_t * a.cand_cap + slot] = p_key;
+        a.cand_idx[p_t * a.cand_cap + slot] = p_s;
+      }
+      pend = false;
+    };
     for (int i = g; i < ntiles; i += 2) {
       const float ks = ks_next;
       ks_next = key_scale(i + 2);
@@ -216,10 +238,34 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.t_empty[g]));
       };
+      // Called by the whole warp with the same qq. Scores mode writes the
+      // row; filter mode appends (order key, key) of every score at or above
+      // the row's threshold to its candidate list: one atomic per warp and
+      // query, whose slot is used only at the next call, so that a chunk of
+      // the epilogue runs while the atomic returns.
       auto emit = [&](int qq, float acc) {
-        if (qq >= nqb || !key_ok) return;
+        if (qq >= nqb) return;
         const long long t = q0 + qq;
         const long long pos = pos0 + qq;
+        if (a.tau) {
+          flush_pending();
+          const uint32_t key = score_key(acc * ks);
+          const bool keep = key_ok && s <= pos && key >= a.tau[t];
+          const unsigned ball = __ballot_sync(0xffffffffu, keep);
+          if (ball) {
+            unsigned base = 0;
+            if (lane == 0) base = atomicAdd(a.cand_count + t, static_cast<unsigned>(__popc(ball)));
+            pend = true;
+            p_key = key;
+            p_keep = keep;
+            p_ball = ball;
+            p_base = base;
+            p_t = t;
+            p_s = static_cast<int>(s);
+          }
+          return;
+        }
+        if (!key_ok) return;
         float* out = a.scores + t * a.ld;
         out[s] = (s <= pos) ? acc * ks : -INFINITY;
       };
@@ -269,6 +315,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
       }
     }
+    flush_pending();
   }
   tc_fence_before();
   __syncthreads();

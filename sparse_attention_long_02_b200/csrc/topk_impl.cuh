@@ -349,6 +349,42 @@ __device__ void bitmap_scan(const unsigned* bm, long long n, TopkSmem& sm, F emi
   }
 }
 
+// With every key of a row of n (n <= kSampledMaxN) at or above some
+// threshold in sm.cand_key / sm.cand_idx (ncand of them, any order, at least
+// k): the k largest, ties to the smaller index, written to out in index
+// order. An exact select in shared memory gives the k-th largest key and how
+// many of its ties to take; two bitmaps of the row (above it / equal to it)
+// and ordered scans put the selection in index order.
+__device__ void select_from_candidates(long long n, int k, int ncand, int* out, TopkSmem& sm) {
+  const int tid = threadIdx.x;
+  uint32_t thr;
+  unsigned need;
+  smem_select<3>(sm.cand_key, ncand, static_cast<unsigned>(k), sm.hist, sm, &thr, &need);
+  unsigned* gt = sm.hist;
+  unsigned* eq = reinterpret_cast<unsigned*>(sm.sure);
+  const int words = static_cast<int>((n + 31) >> 5);
+  for (int w = tid; w < words; w += kTopkThreads) {
+    gt[w] = 0u;
+    eq[w] = 0u;
+  }
+  __syncthreads();
+  for (int j = tid; j < ncand; j += kTopkThreads) {
+    const uint32_t u = sm.cand_key[j];
+    const int ix = sm.cand_idx[j];
+    if (u > thr) atomicOr(&gt[ix >> 5], 1u << (ix & 31));
+    else if (u == thr) atomicOr(&eq[ix >> 5], 1u << (ix & 31));
+  }
+  __syncthreads();
+  // the first `need` ties in index order join the selection
+  bitmap_scan(eq, n, sm, [&](unsigned r, int ix) {
+    if (r < need) atomicOr(&gt[ix >> 5], 1u << (ix & 31));
+  });
+  __syncthreads();
+  bitmap_scan(gt, n, sm, [&](unsigned r, int ix) {
+    if (r < static_cast<unsigned>(k)) out[r] = ix;
+  });
+}
+
 // Sampled path. The k-th largest key is estimated from a sample of the row
 // (the first 256 keys of every 4096) with a margin; one sweep then keeps
 // every key at or above the estimate, appended in any order with one shared
@@ -436,56 +472,22 @@ __device__ bool select_sampled(const float4* x4, long long n, long long n4, int 
   __syncthreads();
   const unsigned kept = sm.s_count;
   if (kept < static_cast<unsigned>(k) || kept > static_cast<unsigned>(kCandCap)) return false;
-  const int ncand = static_cast<int>(kept);
-  uint32_t thr;
-  unsigned need;
-  smem_select<3>(sm.cand_key, ncand, static_cast<unsigned>(k), sm.hist, sm, &thr, &need);
-  // bitmaps of the row: gt = keys above thr, eq = keys equal to it
-  unsigned* gt = sm.hist;
-  unsigned* eq = reinterpret_cast<unsigned*>(sm.sure);
-  const int words = static_cast<int>((n + 31) >> 5);
-  for (int w = tid; w < words; w += kTopkThreads) {
-    gt[w] = 0u;
-    eq[w] = 0u;
-  }
-  __syncthreads();
-  for (int j = tid; j < ncand; j += kTopkThreads) {
-    const uint32_t u = sm.cand_key[j];
-    const int ix = sm.cand_idx[j];
-    if (u > thr) atomicOr(&gt[ix >> 5], 1u << (ix & 31));
-    else if (u == thr) atomicOr(&eq[ix >> 5], 1u << (ix & 31));
-  }
-  __syncthreads();
-  // the first `need` ties in index order join the selection
-  bitmap_scan(eq, n, sm, [&](unsigned r, int ix) {
-    if (r < need) atomicOr(&gt[ix >> 5], 1u << (ix & 31));
-  });
-  __syncthreads();
-  bitmap_scan(gt, n, sm, [&](unsigned r, int ix) {
-    if (r < static_cast<unsigned>(k)) out[r] = ix;
-  });
+  select_from_candidates(n, k, static_cast<int>(kept), out, sm);
   return true;
 }
 
-__global__ void __launch_bounds__(kTopkThreads, DSA_TOPK_MIN_CTAS) topk_kernel(const TopkArgs a) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
-  const int r = blockIdx.x;
+// The selection of one row of n scores (k of them, sorted by index, -1
+// padded): every key when n <= k, else the sampled path, falling back to the
+// two-pass paths.
+__device__ void select_row(const float* row, long long n, int k, int* out, TopkSmem& sm) {
   const int tid = threadIdx.x;
-  int* out = a.idx + static_cast<long long>(r) * a.k;
-  long long n = row_length(a, r);
-  if (n < 0) n = 0;
-  if (n > a.ld) {                       // cannot happen for validated calls
-    if (tid == 0) raise_error(a.err, kErrBounds);
-    n = a.ld;
-  }
-  if (n <= a.k) {                       // short context: every key
-    for (int j = tid; j < a.k; j += kTopkThreads) out[j] = j < n ? j : -1;
+  if (n <= k) {                         // short context: every key
+    for (int j = tid; j < k; j += kTopkThreads) out[j] = j < n ? j : -1;
     return;
   }
-  const float4* x4 = reinterpret_cast<const float4*>(a.scores + static_cast<long long>(r) * a.ld);
+  const float4* x4 = reinterpret_cast<const float4*>(row);
   const long long n4 = (n + 3) >> 2;
-  if (a.k <= 2048 && n >= 4ll * a.k && n <= kSampledMaxN && select_sampled(x4, n, n4, a.k, out, sm))
+  if (k <= 2048 && n >= 4ll * k && n <= kSampledMaxN && select_sampled(x4, n, n4, k, out, sm))
     return;
   __syncthreads();
   // pass 1: 12-bit histogram of the whole row
@@ -500,17 +502,34 @@ __global__ void __launch_bounds__(kTopkThreads, DSA_TOPK_MIN_CTAS) topk_kernel(c
       if (4 * i + c < n) atomicAdd(&sm.hist[order_key(e[c]) >> 20], 1u);
   }
   __syncthreads();
-  find_bucket(sm.hist, kBins, static_cast<unsigned>(a.k), &sm.s_bucket, &sm.s_above);
+  find_bucket(sm.hist, kBins, static_cast<unsigned>(k), &sm.s_bucket, &sm.s_above);
   const unsigned b = sm.s_bucket, above = sm.s_above, in_bucket = sm.hist[b];
   __syncthreads();
-  if (a.k <= kFastMaxK && in_bucket <= static_cast<unsigned>(kCandCap))
-    select_fast(x4, n, n4, a.k, out, sm, b, above);
+  if (k <= kFastMaxK && in_bucket <= static_cast<unsigned>(kCandCap))
+    select_fast(x4, n, n4, k, out, sm, b, above);
   else
-    select_general(x4, n, n4, a.k, out, sm);
+    select_general(x4, n, n4, k, out, sm);
 }
+
+#ifdef DSA_TOPK_LAUNCH
+__global__ void __launch_bounds__(kTopkThreads, DSA_TOPK_MIN_CTAS) topk_kernel(const TopkArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
+  const int r = blockIdx.x;
+  int* out = a.idx + static_cast<long long>(r) * a.k;
+  long long n = row_length(a, r);
+  if (n < 0) n = 0;
+  if (n > a.ld) {                       // cannot happen for validated calls
+    if (threadIdx.x == 0) raise_error(a.err, kErrBounds);
+    n = a.ld;
+  }
+  select_row(a.scores + static_cast<long long>(r) * a.ld, n, a.k, out, sm);
+}
+#endif
 
 }  // namespace
 
+#ifdef DSA_TOPK_LAUNCH
 cudaError_t DSA_TOPK_LAUNCH(const TopkArgs& a, cudaStream_t st) {
   if (a.rows <= 0) return cudaSuccess;
   const size_t smem = sizeof(TopkSmem);
@@ -524,5 +543,6 @@ cudaError_t DSA_TOPK_LAUNCH(const TopkArgs& a, cudaStream_t st) {
   topk_kernel<<<a.rows, kTopkThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
+#endif
 
 }  // namespace dsa

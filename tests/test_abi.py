@@ -100,6 +100,19 @@ def test_host_validation_rejects_before_launch(dsa):
     assert L.dsa_indexer_backward(fake, None, fake, None, fake, 4, big + 1, 4, 0,
                                   ctypes.c_float(1.0), fake, big + 1, fake, fake, fake, fake,
                                   1 << 40, None) == -1
+    # fused prefill: k above 2048 or rows above 131072 keys unsupported; workspace checked
+    assert L.dsa_forward_fused(fake, None, fake, None, fake, fake, fake, 8, 8, 4, 8, 0, 4096, 0,
+                               ctypes.c_float(1.0), ctypes.c_float(0.1), None, fake, None, fake,
+                               1 << 40, None) == -2
+    assert L.dsa_forward_fused(fake, None, fake, None, fake, fake, fake, 8, 131073, 4, 8, 0, 4, 0,
+                               ctypes.c_float(1.0), ctypes.c_float(0.1), None, fake, None, fake,
+                               1 << 40, None) == -2
+    assert L.dsa_forward_fused(fake, None, fake, None, fake, fake, fake, 8, 8, 4, 8, 0, 4, 0,
+                               ctypes.c_float(1.0), ctypes.c_float(0.1), None, fake, None, None, 0,
+                               None) == -3
+    assert L.dsa_forward_fused(None, None, fake, None, fake, fake, fake, 8, 8, 4, 8, 0, 4, 0,
+                               ctypes.c_float(1.0), ctypes.c_float(0.1), None, fake, None, fake,
+                               1 << 40, None) == -1
     # empty problems are a no-op
     assert L.dsa_topk(fake, 0, 4, 4, 0, 4, fake, None) == 0
 
@@ -115,6 +128,16 @@ def test_workspace_sizes(dsa):
     assert L.dsa_decode_paged_workspace_size(64, 1, 512, 64, 128, 2048) == \
         64 * 512 * 64 * 4 + 64 * 2048 * 4
     assert L.dsa_forward_workspace_size(0, 8, 4, 8, 4, 0) == 0
+    # fused prefill: the sampled keys (the first 256 of every 4096) and their
+    # scales, per chunk row the sample scores, threshold, count and 4096
+    # candidates, the failure list, 148 scratch score rows, and idx
+    r256 = lambda x: (x + 255) // 256 * 256
+    T, S, k, rows = 131072, 131072, 2048, 4096
+    M = 32 * 256
+    parts = [M * 128, M * 4, rows * M * 4, rows * 4, rows * 4, rows * 4096 * 4, rows * 4096 * 4,
+             4 + rows * 4, 148 * S * 4, T * k * 4]
+    assert L.dsa_forward_fused_workspace_size(T, S, 64, 128, k, rows) == sum(r256(x) for x in parts)
+    assert L.dsa_forward_fused_workspace_size(T, S, 64, 128, 4096, rows) == 0
     # warm-up target: T * H rows of fp32 logits, S rounded up to 4
     assert L.dsa_attention_probs_workspace_size(2048, 2048, 128) == 2048 * 128 * 2048 * 4
     assert L.dsa_attention_probs_workspace_size(3, 10, 2) == 3 * 2 * 12 * 4

@@ -119,6 +119,79 @@ def test_forward_end_to_end_on_grid(dsa, cfg1):
     assert_mla_close(out, ref["out"], lse, ref["lse"])
 
 
+@pytest.mark.parametrize("chunk", [300, 0])
+def test_forward_fused_end_to_end_on_grid(dsa, cfg1, chunk):
+    """The top-k fused into the indexer (no score rows in HBM): bit-exact
+    selection on the exact grid, in chunks and in one piece."""
+    inp, ref = cfg1
+    g = cuda(inp)
+    out, lse, idx = dsa.forward_fused(g["q8"], None, g["k8"], None, g["w"], g["q"], g["kv"],
+                                      inp["k"], inp["scale"], inp["sm_scale"], chunk=chunk)
+    no_device_error(dsa)
+    got = idx.cpu().numpy()
+    for r in range(inp["T"]):
+        assert set(got[r][got[r] >= 0]) == set(ref["idx"][r][ref["idx"][r] >= 0]), r
+    assert_mla_close(out, ref["out"], lse, ref["lse"])
+
+
+def test_forward_fused_recomputes_rows_whose_threshold_misses(dsa):
+    """Keys at the sampled positions (the first 256 of every 4096) hold each
+    row's largest scores, all distinct from the rest, so the threshold taken
+    from the sample lies above the k-th score, fewer than k candidates are
+    kept, and the row's scores are recomputed on CUDA cores. Exact-grid
+    integers keep every score exact: the selection must equal the oracle's."""
+    rng = np.random.default_rng(61)
+    L, Hi, H, k = 6000, 4, 8, 256
+    pos = np.arange(L)
+    sampled = (pos % 4096) < 256
+    ones = np.where(sampled, rng.integers(32, 129, L), rng.integers(0, 17, L))
+    kf = (np.arange(128)[None, :] < ones[:, None]).astype(np.float32)      # q.k = ones[s]
+    k8 = torch.from_numpy(kf).to(torch.float8_e4m3fn).view(torch.uint8)
+    q8 = torch.ones(L, Hi, 128).to(torch.float8_e4m3fn).view(torch.uint8)
+    w = torch.full((L, Hi), 0.25)
+    q = torch.from_numpy(rng.normal(size=(L, H, 576))).to(torch.bfloat16)
+    kv = torch.from_numpy(rng.normal(size=(L, 576))).to(torch.bfloat16)
+    inp = dict(q8=q8, q_scale=None, k8=k8, k_scale=None, w=w, q=q, kv=kv, scale=1 / 16,
+               sm_scale=1 / 24, k=k, q_pos0=0, T=L, S=L, Hi=Hi, H=H)
+    g = cuda(inp)
+    out, lse, idx = dsa.forward_fused(g["q8"], None, g["k8"], None, g["w"], g["q"], g["kv"], k,
+                                      inp["scale"], inp["sm_scale"], chunk=2048)
+    no_device_error(dsa)
+    _, _, idx_ref = dsa.forward(g["q8"], None, g["k8"], None, g["w"], g["q"], g["kv"], k,
+                                inp["scale"], inp["sm_scale"], chunk=2048)
+    got, exp = idx.cpu().numpy(), idx_ref.cpu().numpy()
+    for r in range(L):                   # the chunked path, bit-exact on this grid
+        assert set(got[r][got[r] >= 0]) == set(exp[r][exp[r] >= 0]), r
+    rows = np.array([0, 255, 256, 1500, 2047, 4095, 4096, 4400, 5999])
+    ref = oracle.forward(inp, rows=rows)
+    for i, r in enumerate(rows):
+        assert set(got[r][got[r] >= 0]) == set(ref["idx"][i][ref["idx"][i] >= 0]), r
+    assert_mla_close(out[rows], ref["out"], lse[rows], ref["lse"])
+
+
+def test_forward_fused_matches_forward_on_16k_planted(dsa):
+    """Config 2 (L = 16384, planted keys): the fused path selects what the
+    chunked path selects; a row may differ only where the chunked path's own
+    score of a differing key is within 1e-3 of the row's k-th score."""
+    inp = W.make_prefill(W.CONFIGS[2], device="cuda")
+    args = (inp["q8"], inp["q_scale"], inp["k8"], inp["k_scale"], inp["w"], inp["q"], inp["kv"],
+            inp["k"], inp["scale"], inp["sm_scale"])
+    _, _, idx_f = dsa.forward_fused(*args, chunk=4096)
+    no_device_error(dsa)
+    _, _, idx_c = dsa.forward(*args, chunk=4096)
+    no_device_error(dsa)
+    a, b = idx_f.cpu().numpy(), idx_c.cpu().numpy()
+    diff = [r for r in range(a.shape[0]) if set(a[r]) != set(b[r])]
+    assert len(diff) <= 8, len(diff)
+    for r in diff:
+        sc = dsa.indexer_scores(inp["q8"][r:r + 1], inp["q_scale"][r:r + 1], inp["k8"],
+                                inp["k_scale"], inp["w"][r:r + 1], inp["scale"], q_pos0=r)
+        row = sc[0].double().cpu().numpy()
+        tau = min(row[i] for i in b[r] if i >= 0)
+        for i in set(a[r]) ^ set(b[r]):
+            assert abs(row[i] - tau) <= IDX_REL * abs(tau) + 1e-30, (r, i)
+
+
 # ------------------------------------------------------ random FP8 inputs
 
 def _random_prefill(L, Hi, H, k, seed, plant=True):
