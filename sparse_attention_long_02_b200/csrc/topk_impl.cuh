@@ -1,11 +1,12 @@
 // topk_impl.cuh -- per-query top-k selection over score rows.
 //
-// Compiled twice, as 512-thread CTAs (topk.cu: rows that have the GPU to
+// Compiled as 512-thread CTAs (topk.cu: rows that have the GPU to
 // themselves) and as 256-thread CTAs (topk_narrow.cu: the chunks of a prefill,
 // whose selection runs on a side stream beside the next chunk's indexer; a
 // 256-thread CTA at <= 64 registers fits on an SM beside a 128-register
-// indexer CTA). The including file defines DSA_TOPK_THREADS, DSA_TOPK_MIN_CTAS
-// and DSA_TOPK_LAUNCH, the name of the launcher.
+// indexer CTA); fused_topk.cu uses its device functions only. The including
+// file defines DSA_TOPK_THREADS and DSA_TOPK_MIN_CTAS, and DSA_TOPK_LAUNCH,
+// the name of the row-per-CTA kernel's launcher, where it wants that kernel.
 //
 // Step 3 of the four-step workflow ("DeepSeek-V3.2-Exp 模型优势与 DSA 工作原理",
 // section 4): each query keeps its k highest-scoring keys, or every key when
