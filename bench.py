@@ -51,6 +51,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--path", default="scores", choices=["fused", "scores"],
+                    help="fused: dsa_forward_fused (top-k fused into the indexer, no score rows "
+                         "in HBM); scores: dsa_forward (each chunk's scores in HBM, read back by "
+                         "the top-k)")
     ap.add_argument("--next", action="store_true",
                     help="also time dense causal and sliding-window attention beside DSA at 16K")
     ap.add_argument("--shard", default="problems", choices=["problems", "rows"],
@@ -217,20 +221,24 @@ def prefill_inputs(L, rank):
 class Prefill:
     """Preallocated buffers and one call of the whole path per step."""
 
-    def __init__(self, dsa, cfg, inp):
-        self.dsa, self.cfg, self.inp = dsa, cfg, inp
+    def __init__(self, dsa, cfg, inp, path="scores"):
+        self.dsa, self.cfg, self.inp, self.path = dsa, cfg, inp, path
         T, H, k = inp["T"], inp["H"], inp["k"]
         self.chunk = cfg.chunk or T
-        self.ws = torch.empty(dsa.forward_workspace_size(T, inp["S"], inp["Hi"], H, k, self.chunk),
+        size = dsa.forward_fused_workspace_size if path == "fused" else dsa.forward_workspace_size
+        self.run = dsa.forward_fused if path == "fused" else dsa.forward
+        self.ws = torch.empty(size(T, inp["S"], inp["Hi"], H, k, self.chunk),
                               dtype=torch.uint8, device="cuda")
         self.out = torch.empty(T, H, 512, dtype=torch.bfloat16, device="cuda")
         self.lse = torch.empty(T, H, dtype=torch.float32, device="cuda")
         self.idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
-        self.launches = 2 * math.ceil(T / self.chunk) + 1
+        # per chunk: indexer + top-k (scores), or sample indexer, threshold, filter
+        # indexer, select and recompute (fused); then one sparse MLA launch
+        self.launches = (5 if path == "fused" else 2) * math.ceil(T / self.chunk) + 1
 
     def step(self):
         i = self.inp
-        self.dsa.forward(i["q8"], i["q_scale"], i["k8"], i["k_scale"], i["w"], i["q"], i["kv"],
+        self.run(i["q8"], i["q_scale"], i["k8"], i["k_scale"], i["w"], i["q"], i["kv"],
                          i["k"], i["scale"], i["sm_scale"], chunk=self.chunk, idx=self.idx,
                          out=self.out, lse=self.lse, workspace=self.ws)
 
@@ -239,7 +247,10 @@ class Prefill:
         d, i = self.dsa, self.inp
         T, S, Hi, k = i["T"], i["S"], i["Hi"], i["k"]
         ld = (S + 3) // 4 * 4
-        scores = self.ws[: self.chunk * ld * 4].view(torch.float32).view(self.chunk, ld)
+        if self.ws.numel() >= self.chunk * ld * 4:
+            scores = self.ws[: self.chunk * ld * 4].view(torch.float32).view(self.chunk, ld)
+        else:                                 # the fused path's workspace holds no score rows
+            scores = torch.empty(self.chunk, ld, dtype=torch.float32, device="cuda")
         tot = {"indexer": 0.0, "topk": 0.0, "sparse_mla": 0.0}
         for _ in range(reps):
             for c0 in range(0, T, self.chunk):
@@ -627,9 +638,9 @@ def main():
         tokens = L
         del shard.ws, shard.out, shard.lse, shard.idx
         torch.cuda.empty_cache()
-        pf = Prefill(dsa, cfg, inp)
+        pf = Prefill(dsa, cfg, inp, args.path)
     else:
-        pf = Prefill(dsa, cfg, inp)
+        pf = Prefill(dsa, cfg, inp, args.path)
         ms, clocks = time_steps(pf.step, args.steps, args.warmup, ranks, dsa, ranks.local)
         tokens = L * ranks.world
     value = tokens / (ms / 1e3)
@@ -659,6 +670,9 @@ def main():
         max(work["mla_flops"] / (pk["bf16_sus"] * 1e12), work["mla_bytes"] / (pk["hbm"] * 1e9))
 
     config = config_obj(L, pf.chunk)
+    config["path"] = ("dsa_forward_fused: top-k fused into the indexer, no score rows in HBM"
+                      if args.path == "fused" else
+                      "dsa_forward: each chunk's scores in HBM, top-k beside the next indexer")
     if rows_mode:
         config["shard"] = (f"rows: the {math.ceil(L / pf.chunk)} chunks of one prefill over "
                            f"{ranks.world} GPU(s) by causal cost; rank 0 runs "

@@ -24,12 +24,13 @@
 //      the gathered tile, into the TMEM logit buffer;
 //   3. eight softmax warps, two per TMEM lane quarter (thread = head, each
 //      warp of a pair taking 32 of the 64 keys), scale their partial logits
-//      into the log2 domain and stage them as fp16 in shared memory; the
-//      exchange warp sends the whole 16 KB tile to the peer CTA with one bulk
+//      into the log2 domain and stage them, in fp32, in shared memory; the
+//      exchange warp sends the whole 32 KB tile to the peer CTA with one bulk
 //      copy (the TMA engine, off the load/store path the gather uses). Tile
 //      i+1 is staged and sent while tile i is finished, so the transfer runs
-//      under the softmax arithmetic. Both CTAs add the same two fp16 partials,
-//      so they see identical logits; they mask unselected slots, agree on
+//      under the softmax arithmetic. Both CTAs add the same two fp32
+//      partials (fp32 addition commutes), so they see identical logits with
+//      nothing rounded below fp32; they mask unselected slots, agree on
 //      the tile maximum through shared memory, run the online softmax in the
 //      exp2 domain and store P (bf16) into the TMEM P buffer; the
 //      running maximum is re-based only when it grows by more than 8 (log2
@@ -39,14 +40,13 @@
 // The final output is O / l in bf16 and lse = (m + log2 l) * ln 2.
 #include "common.cuh"
 #include "dsa_internal.h"
-#include <cuda_fp16.h>
 
 namespace dsa {
 namespace {
 
 constexpr int kMlaThreads = 512;
 constexpr int kTileKeys = 64;
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kAtoms = 4;                        // 128-B swizzled atoms of 64 dims
 constexpr int kAtomBytesQ = 128 * 128;           // 128 heads x 64 dims bf16
 constexpr int kRopeBytesQ = 128 * 64;            // 128 heads x 32 dims bf16 (64-B swizzle)
@@ -55,36 +55,37 @@ constexpr int kRopeBytesKV = kTileKeys * 64;     // 64 keys x 32 dims bf16
 constexpr int kGatherWarps = 6;                  // warps 0, 2, 3, 12, 13, 14
 constexpr int kSoftmaxWarps = 8;                 // warps 4-11
 constexpr int kExchangeWarp = 15;
-constexpr uint32_t kXBytes = 128 * kTileKeys * 2;   // one tile of fp16 partial logits
+constexpr uint32_t kXBytes = 128 * kTileKeys * 4;   // one tile of fp32 partial logits
 constexpr uint32_t kColO = 0;                    // TMEM columns [0,256): output
 constexpr uint32_t kColQ = 256;                  // [256,400): Q_c, bf16 pairs (256 + 32 dims)
 constexpr uint32_t kColP = 416;                  // [416,448): P, bf16 pairs
 constexpr uint32_t kColS = 448;                  // [448,512): logits
-// Q arrives by TMA in ring stages 2-3 (72 KB) and is moved into TMEM before
-// the gather first reaches stage 2.
-constexpr int kQStage = 2;
+// Q arrives by TMA in the exchange buffers (the latent atoms in x, the rope
+// block in stage) and is moved into TMEM before the first exchange, so the
+// whole KV ring is free for the gather from the first tile.
 constexpr float kRebase = 8.0f;                  // lazy rescale threshold (log2 units)
 
-// Rows of 64 fp16 partials (128 B, one per head); the 16-B chunk c of row h
+// Rows of 64 fp32 partials (256 B, one per head); the 16-B chunk c of row h
 // sits at chunk c ^ (h & 7), so eight consecutive heads hit distinct banks.
 struct MlaSmem {
   uint8_t kv[kStages][kAtoms][kAtomBytesKV];
   uint8_t kv_rope[kStages][kRopeBytesKV];
-  uint4 x[2][128 * 8];                           // the peer's partials, by tile parity
-  uint4 stage[2][128 * 8];                       // this CTA's partials (bulk copy source)
+  uint4 x[2][128 * 16];                          // the peer's partials, by tile parity
+  uint4 stage[128 * 16];                         // this CTA's partials (bulk copy source)
   float pair_max[2][2][128];                     // [tile parity][key half][head]
   unsigned valid[kStages][2];                    // selected-slot bits of each half tile
   unsigned long long q_full;                     // Q has landed in its staging slots
-  unsigned long long q_ready;                    // Q is in TMEM (stages 2-3 are free)
+  unsigned long long q_ready;                    // Q is in TMEM (its staging slots are free)
+  unsigned long long peer_q;                     // the peer's Q is in its TMEM: its x may be sent to
   unsigned long long kv_full[kStages];
   unsigned long long kv_empty[kStages];
   unsigned long long s_full;
   unsigned long long s_empty;
   unsigned long long p_full;
   unsigned long long p_empty;
-  // per buffer (tile parity):
-  unsigned long long stage_full[2];              // the eight softmax warps have staged a tile
-  unsigned long long stage_free[2];              // the peer has received the tile staged here
+  unsigned long long stage_full;                 // the eight softmax warps have staged a tile
+  unsigned long long stage_free;                 // the peer has received the tile staged here
+  // per receive buffer (tile parity):
   unsigned long long x_full[2];                  // the peer's partials have landed in x
   unsigned long long x_free[2];                  // the peer has read what this CTA sent it
   unsigned long long x_read[2];                  // the softmax warps have read x
@@ -94,9 +95,10 @@ struct MlaSmem {
   int abort_flag;
 };
 
-static_assert(2 * kAtoms * kAtomBytesKV == kAtoms * kAtomBytesQ, "Q latent staging = 2 stages");
-static_assert(2 * kRopeBytesKV == kRopeBytesQ, "Q rope staging = 2 stages");
-static_assert(kQStage + 2 <= kStages, "Q staging inside the ring");
+// Q staging: latent atoms 0-1 in x[0], 2-3 in x[1], the rope block in stage.
+static_assert(sizeof(MlaSmem::x[0]) == 2 * kAtomBytesQ, "two Q atoms per receive buffer");
+static_assert(sizeof(MlaSmem::stage) >= kRopeBytesQ, "Q rope block fits the stage buffer");
+static_assert(kAtomBytesKV % 1024 == 0 && kRopeBytesKV % 1024 == 0, "1024-B aligned staging");
 
 // Physical row of slot value `v` (a logical position), or -1 if skipped.
 __device__ __forceinline__ int kv_row(const MlaArgs& A, int v, int seq, int limit) {
@@ -140,6 +142,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&sm.q_full), 1);
     mbar_init(smem_u32(&sm.q_ready), 4);         // the four warps that move Q into TMEM
+    mbar_init(smem_u32(&sm.peer_q), 1);          // one arrival from the peer
     for (int i = 0; i < kStages; ++i) {
       // one cp.async-completion arrival per gathering thread + the slot writer
       mbar_init(smem_u32(&sm.kv_full[i]), 32 * kGatherWarps + 1);
@@ -149,9 +152,9 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mbar_init(smem_u32(&sm.s_empty), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.p_full), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.p_empty), 1);
+    mbar_init(smem_u32(&sm.stage_full), kSoftmaxWarps);
+    mbar_init(smem_u32(&sm.stage_free), 1);      // one arrival from the peer per use
     for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&sm.stage_full[b]), kSoftmaxWarps);
-      mbar_init(smem_u32(&sm.stage_free[b]), 1);  // one arrival from the peer per use
       mbar_init(smem_u32(&sm.x_full[b]), 1);      // own expect_tx + the peer's copied bytes
       mbar_init(smem_u32(&sm.x_free[b]), 1);      // one arrival from the peer per use
       mbar_init(smem_u32(&sm.x_read[b]), kSoftmaxWarps);
@@ -181,10 +184,10 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (warp == 0 && lane == 0) {
       const uint32_t qf = smem_u32(&sm.q_full);
       mbar_expect_tx(qf, kAtoms * kAtomBytesQ + kRopeBytesQ);
-      const uint32_t qs = smem_u32(sm.kv[kQStage][0]);
       for (int a = 0; a < kAtoms; ++a)
-        tma_load_2d(qs + a * kAtomBytesQ, &tm_q, qf, dim0 + 64 * a, r * A.H);
-      tma_load_2d(smem_u32(sm.kv_rope[kQStage]), &tm_qr, qf, rope0, r * A.H);
+        tma_load_2d(smem_u32(sm.x[a >> 1]) + (a & 1) * kAtomBytesQ, &tm_q, qf, dim0 + 64 * a,
+                    r * A.H);
+      tma_load_2d(smem_u32(sm.stage), &tm_qr, qf, rope0, r * A.H);
     }
     int v0 = lane < A.k ? __ldg(sel + lane) : -1;
     int v1 = lane + 32 < A.k ? __ldg(sel + lane + 32) : -1;
@@ -197,7 +200,6 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         v1 = j0 + 32 < A.k ? __ldg(sel + j0 + 32) : -1;
       }
       const int r0 = kv_row(A, c0, seq, limit), r1 = kv_row(A, c1, seq, limit);
-      if (i == kQStage && !warp_wait(smem_u32(&sm.q_ready), 0, abort_flag, err)) break;
       if (i >= kStages &&
           !warp_wait(smem_u32(&sm.kv_empty[st]), ((i / kStages) + 1) & 1, abort_flag, err))
         break;
@@ -227,41 +229,48 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (warp == 0 && lane == 0) mbar_drain(smem_u32(&sm.q_full), 0);
   } else if (warp == kExchangeWarp && !aborted) {
     // ---------------------------------------------------- exchange warp
-    // Tile j's partials travel from stage[j & 1] to the peer's x[j & 1] in
-    // one bulk copy, once they are staged and the peer has read tile j-2 out
-    // of that buffer. This warp also tells the peer when its copy of tile i
-    // has landed here (its stage buffer may be refilled) and when x has been
-    // read (it may send into that buffer again). Cluster-scope releases come
-    // from this warp only, so they never queue behind the softmax warps.
+    // Tile j's partials travel from stage to the peer's x[j & 1] in one bulk
+    // copy, once they are staged and the peer has read tile j-2 out of that
+    // buffer (for the first two tiles: once the peer has moved its Q, which
+    // is staged in x, into TMEM). This warp also tells the peer when its copy
+    // of tile i has landed here (its stage buffer may be refilled) and when x
+    // has been read (it may send into that buffer again). Cluster-scope
+    // releases come from this warp only, so they never queue behind the
+    // softmax warps.
     if (lane == 0) {
       int sent = 0;
       auto send = [&](int j) -> bool {
         const int b = j & 1;
-        if (!mbar_wait(smem_u32(&sm.stage_full[b]), (j >> 1) & 1, abort_flag, err)) return false;
+        if (!mbar_wait(smem_u32(&sm.stage_full), j & 1, abort_flag, err)) return false;
         if (j >= 2 && !mbar_wait<true>(smem_u32(&sm.x_free[b]), ((j - 2) >> 1) & 1, abort_flag, err))
           return false;
-        bulk_copy_to_peer(mapa(smem_u32(sm.x[b]), peer), smem_u32(sm.stage[b]), kXBytes,
+        bulk_copy_to_peer(mapa(smem_u32(sm.x[b]), peer), smem_u32(sm.stage), kXBytes,
                           mapa(smem_u32(&sm.x_full[b]), peer));
         sent = j + 1;
         return true;
       };
       for (int j = 0; j < 2 && j < ntiles; ++j)                 // the peer's tiles 0 and 1
         mbar_expect_tx(smem_u32(&sm.x_full[j]), kXBytes);
-      bool ok = send(0);
+      // this CTA's Q has left x: the peer may send into it
+      bool ok = mbar_wait(smem_u32(&sm.q_ready), 0, abort_flag, err);
+      if (ok) mbar_arrive_remote(mapa(smem_u32(&sm.peer_q), peer));
+      ok = ok && mbar_wait<true>(smem_u32(&sm.peer_q), 0, abort_flag, err);
+      ok = ok && (ntiles == 0 || send(0));
       for (int i = 0; ok && i < ntiles; ++i) {
         const int b = i & 1;
         if (i + 1 < ntiles && !(ok = send(i + 1))) break;
         if (!(ok = mbar_wait<true>(smem_u32(&sm.x_full[b]), (i >> 1) & 1, abort_flag, err))) break;
-        mbar_arrive_remote(mapa(smem_u32(&sm.stage_free[b]), peer));
+        mbar_arrive_remote(mapa(smem_u32(&sm.stage_free), peer));
         if (i + 2 < ntiles) mbar_expect_tx(smem_u32(&sm.x_full[b]), kXBytes);   // tile i+2
         if (!(ok = mbar_wait(smem_u32(&sm.x_read[b]), (i >> 1) & 1, abort_flag, err))) break;
         mbar_arrive_remote(mapa(smem_u32(&sm.x_free[b]), peer));
       }
       // A copy reads this CTA's stage buffer until it lands: wait for the
-      // peer's word on the last two before this CTA may leave.
-      for (int j = sent > 2 ? sent - 2 : 0; j < sent; ++j) {
-        const uint32_t bar = smem_u32(&sm.stage_free[j & 1]);
-        if (!mbar_wait<true>(bar, (j >> 1) & 1, abort_flag, err)) mbar_drain(bar, (j >> 1) & 1);
+      // peer's word on the last one before this CTA may leave (the softmax
+      // warps waited for every earlier one before restaging).
+      if (sent > 0) {
+        const uint32_t bar = smem_u32(&sm.stage_free);
+        if (!mbar_wait<true>(bar, (sent - 1) & 1, abort_flag, err)) mbar_drain(bar, (sent - 1) & 1);
       }
     }
   } else if (warp == 1 && !aborted) {
@@ -328,10 +337,10 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       // pairs, lane = head): 256 latent dims from the 128-B swizzled atoms,
       // then the 32 rope dims from the 64-B swizzled block.
       if ((ok = warp_wait(smem_u32(&sm.q_full), 0, abort_flag, err))) {
-        const uint8_t* qs = sm.kv[kQStage][0];
 #pragma unroll 1
         for (int a = 0; a < kAtoms; ++a) {
-          const uint4* row = reinterpret_cast<const uint4*>(qs + a * kAtomBytesQ + h * 128);
+          const uint8_t* qs = reinterpret_cast<const uint8_t*>(sm.x[a >> 1]) + (a & 1) * kAtomBytesQ;
+          const uint4* row = reinterpret_cast<const uint4*>(qs + h * 128);
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             uint32_t pk[16];
@@ -347,7 +356,8 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           }
         }
         {
-          const uint4* row = reinterpret_cast<const uint4*>(sm.kv_rope[kQStage] + h * 64);
+          const uint4* row = reinterpret_cast<const uint4*>(
+              reinterpret_cast<const uint8_t*>(sm.stage) + h * 64);
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -365,14 +375,10 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
     }
     // This warp's half of tile j's partial logits, scaled into log2 units
-    // and rounded to fp16: staged for the peer and kept here, so that both
-    // CTAs add the same two fp16 values. fp16 keeps 11 bits of each partial
-    // (relative error 2^-11, below the bf16 rounding P gets before the PV
-    // product) and halves the bytes crossing the network between the two
-    // SMs, the scarce resource.
-    uint32_t own[16];
-    auto stage_tile = [&](int j, uint32_t (&keep)[16]) -> bool {
-      const int b = j & 1;
+    // (fp32), staged for the peer. The stage buffer is single: tile j may
+    // be staged once the copy of tile j-1 has landed at the peer, which is
+    // also after this CTA has read tile j-1's own partials back (below).
+    auto stage_tile = [&](int j) -> bool {
       float v32[32];
       if (!warp_wait(smem_u32(&sm.s_full), j & 1, abort_flag, err)) return false;
       tc_fence_after();
@@ -380,29 +386,23 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty));
-      // the buffer held tile j-2: its copy must have landed at the peer
-      if (j >= 2 &&
-          !warp_wait<true>(smem_u32(&sm.stage_free[b]), ((j - 2) >> 1) & 1, abort_flag, err))
+      if (j >= 1 &&
+          !warp_wait<true>(smem_u32(&sm.stage_free), (j - 1) & 1, abort_flag, err))
         return false;
-      uint4* dst = sm.stage[b] + h * 8;
+      uint4* dst = sm.stage + h * 16;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          __half2 hv = __floats2half2_rn(v32[8 * c + 2 * e] * A.sm_scale_log2,
-                                         v32[8 * c + 2 * e + 1] * A.sm_scale_log2);
-          w[e] = *reinterpret_cast<uint32_t*>(&hv);
-          keep[4 * c + e] = w[e];
-        }
-        dst[(4 * g + c) ^ (h & 7)] = make_uint4(w[0], w[1], w[2], w[3]);
-      }
+      for (int c = 0; c < 8; ++c)
+        dst[(8 * g + c) ^ (h & 7)] =
+            make_uint4(__float_as_uint(v32[4 * c] * A.sm_scale_log2),
+                       __float_as_uint(v32[4 * c + 1] * A.sm_scale_log2),
+                       __float_as_uint(v32[4 * c + 2] * A.sm_scale_log2),
+                       __float_as_uint(v32[4 * c + 3] * A.sm_scale_log2));
       fence_proxy_async_smem();           // generic writes -> the bulk copy's reads
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.stage_full[b]));
+      if (lane == 0) mbar_arrive(smem_u32(&sm.stage_full));
       return true;
     };
-    if (ok && ntiles > 0) ok = stage_tile(0, own);
+    if (ok && ntiles > 0) ok = stage_tile(0);
     for (int i = 0; ok && i < ntiles; ++i) {
       const int st = i % kStages, b = i & 1;
       // which slots of this half tile are selected (staged by the gather warp)
@@ -412,24 +412,22 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (!(ok = warp_wait<true>(smem_u32(&sm.x_full[b]), (i >> 1) & 1, abort_flag, err))) break;
       float s[32];
       {
-        const uint4* xp = sm.x[b] + h * 8;
+        const uint4* xp = sm.x[b] + h * 16;
+        const uint4* op = sm.stage + h * 16;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 v = xp[(4 * g + c) ^ (h & 7)];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t we = e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w;
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&we));
-            const float2 o = __half22float2(*reinterpret_cast<const __half2*>(&own[4 * c + e]));
-            s[8 * c + 2 * e] = o.x + f.x;
-            s[8 * c + 2 * e + 1] = o.y + f.y;
-          }
+        for (int c = 0; c < 8; ++c) {
+          const uint4 f = xp[(8 * g + c) ^ (h & 7)];
+          const uint4 o = op[(8 * g + c) ^ (h & 7)];
+          s[4 * c] = __uint_as_float(o.x) + __uint_as_float(f.x);
+          s[4 * c + 1] = __uint_as_float(o.y) + __uint_as_float(f.y);
+          s[4 * c + 2] = __uint_as_float(o.z) + __uint_as_float(f.z);
+          s[4 * c + 3] = __uint_as_float(o.w) + __uint_as_float(f.w);
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.x_read[b]));
       // the next tile's partials go out while this one is finished
-      if (i + 1 < ntiles && !(ok = stage_tile(i + 1, own))) break;
+      if (i + 1 < ntiles && !(ok = stage_tile(i + 1))) break;
       if (valid != 0xffffffffu) {
 #pragma unroll
         for (int j = 0; j < 32; ++j)

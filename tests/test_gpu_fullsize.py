@@ -1,7 +1,9 @@
 """Parity at the benchmark sizes, in the launch configuration bench.py times.
 
 The GPU runs the whole path at full size: the prefill configs through
-dsa_forward with their chunking, the decode configs through dsa_decode_paged.
+dsa_forward_fused (the top-k fused into the indexer, the path bench.py times)
+and through dsa_forward (scores in HBM), both with their chunking; the decode
+configs through dsa_decode_paged.
 The oracle then recomputes sampled rows one by one: the indexer scores of the
 row, its selection (exact, or within the tie rule on random inputs) and the
 attention on the GPU's own selection (bf16 tolerances).
@@ -12,7 +14,8 @@ import torch
 
 import oracle
 import workloads as W
-from test_gpu_parity import assert_mla_close, assert_sets_within_tolerance, no_device_error
+from test_gpu_parity import (assert_mla_close, assert_sets_within_tolerance, kv_norm_max,
+                             lse_atol, no_device_error)
 
 pytestmark = pytest.mark.gpu
 
@@ -27,15 +30,20 @@ def _host(t):
     return t.detach().cpu()
 
 
-def _prefill_rows(dsa, cfg_id, rows):
+def _prefill_rows(dsa, cfg_id, rows, fused):
+    """Every sampled row's selection against the oracle's (exact, or within the
+    tie rule judged on the oracle's own scores; no row is exempt), and its
+    attention on the GPU's selection against the oracle on that selection."""
     cfg = W.CONFIGS[cfg_id]
     inp = W.make_prefill(cfg, device="cuda")
     T, S, k = inp["T"], inp["S"], inp["k"]
-    chunk = cfg.chunk or T
-    out, lse, idx = dsa.forward(inp["q8"], inp["q_scale"], inp["k8"], inp["k_scale"], inp["w"],
-                                inp["q"], inp["kv"], k, inp["scale"], inp["sm_scale"], chunk=chunk)
+    chunk = cfg.chunk or 4096
+    run = dsa.forward_fused if fused else dsa.forward
+    out, lse, idx = run(inp["q8"], inp["q_scale"], inp["k8"], inp["k_scale"], inp["w"],
+                        inp["q"], inp["kv"], k, inp["scale"], inp["sm_scale"], chunk=chunk)
     no_device_error(dsa)
     k8, ks, kv = _host(inp["k8"]), _host(inp["k_scale"]), _host(inp["kv"])
+    kn = kv_norm_max(kv)
     for r in rows:
         sub = dict(T=1, S=S, k=k, q_pos0=r, scale=inp["scale"], sm_scale=inp["sm_scale"],
                    q8=_host(inp["q8"][r:r + 1]), q_scale=_host(inp["q_scale"][r:r + 1]),
@@ -45,19 +53,26 @@ def _prefill_rows(dsa, cfg_id, rows):
         gidx = _host(idx[r:r + 1]).numpy()
         assert_sets_within_tolerance(gidx, ref["idx"], ref["I"], k)
         o, l = oracle.sparse_mla(sub["q"], kv, gidx, inp["sm_scale"])
-        assert_mla_close(out[r:r + 1], o, lse[r:r + 1], l)
+        assert_mla_close(out[r:r + 1], o, lse[r:r + 1], l,
+                         lse_atol(sub["q"], kn, inp["sm_scale"], l, k))
     del inp, out, lse, idx
     torch.cuda.empty_cache()
 
 
-def test_prefill_128k_in_4096_row_chunks(dsa):
+ROWS_128K = [0, 2046, 2047, 2048, 4095, 4096, 40961, 65537, 98303, 131071]
+ROWS_16K = [0, 2047, 2048, 4095, 4096, 9000, 12287, 16383]
+
+
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "scores_in_hbm"])
+def test_prefill_128k_in_4096_row_chunks(dsa, fused):
     """Config 4 (L = 131072): rows at both ends, on chunk edges, at the k boundary."""
-    _prefill_rows(dsa, 4, [0, 2046, 2047, 2048, 4095, 4096, 65537, 131071])
+    _prefill_rows(dsa, 4, ROWS_128K, fused)
 
 
-def test_prefill_16k(dsa):
-    """Config 2 (L = 16384, planted keys), one chunk."""
-    _prefill_rows(dsa, 2, [0, 2047, 2048, 9000, 16383])
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "scores_in_hbm"])
+def test_prefill_16k(dsa, fused):
+    """Config 2 (L = 16384, planted keys) in 4096-row chunks, as bench.py runs it."""
+    _prefill_rows(dsa, 2, ROWS_16K, fused)
 
 
 def _decode_seqs(dsa, inp, seqs):
@@ -73,10 +88,12 @@ def _decode_seqs(dsa, inp, seqs):
     for i, b in enumerate(seqs):
         gidx = _host(idx[b]).numpy()
         assert_sets_within_tolerance(gidx, ref["idx"][i], ref["I"][i], g["k"])
-        kv_seq = oracle.gather_sequence(kvp.view(torch.int16).numpy(), table[b], int(lens[b]))
-        o, l = oracle.sparse_mla(_host(inp["q"][b]), torch.from_numpy(kv_seq).view(torch.bfloat16),
-                                 gidx, g["sm_scale"])
-        assert_mla_close(out[b], o, lse[b], l)
+        kv_seq = torch.from_numpy(
+            oracle.gather_sequence(kvp.view(torch.int16).numpy(), table[b], int(lens[b]))
+        ).view(torch.bfloat16)
+        o, l = oracle.sparse_mla(_host(inp["q"][b]), kv_seq, gidx, g["sm_scale"])
+        assert_mla_close(out[b], o, lse[b], l,
+                         lse_atol(_host(inp["q"][b]), kv_seq, g["sm_scale"], l, g["k"]))
 
 
 def test_decode_64_by_32k_paged(dsa):
