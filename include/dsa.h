@@ -86,6 +86,26 @@ const char *dsa_last_error_string(void);
 int dsa_get_device_error(dsa_stream_t stream);
 
 /*
+ * Debug aid for failure handling; the pages have no counterpart. With a bit
+ * of `mask` set, every later launch of the named kernel on the current
+ * device first makes its MMA-issuing thread wait on a barrier that nothing
+ * arrives at. That wait, bounded like every wait in the library (1 s), runs
+ * out; the kernel records DSA_ERR_TIMEOUT in the device's error word and
+ * leaves through its give-up path (every CTA drains its own copies in
+ * flight and frees its tensor memory), and later kernels of the library
+ * return at once until dsa_get_device_error() clears the word. Nothing
+ * faults or traps. mask = 0 restores normal operation.
+ *   DSA_DEBUG_STALL_INDEXER  the indexer (dsa_indexer_scores, and the
+ *                            indexer launches inside dsa_forward,
+ *                            dsa_forward_fused and dsa_decode_paged)
+ *   DSA_DEBUG_STALL_MLA      the sparse MLA (every entry point that runs it)
+ * Synchronises the device. Returns DSA_ERR_INVALID_ARG for unknown bits.
+ */
+#define DSA_DEBUG_STALL_INDEXER 1u
+#define DSA_DEBUG_STALL_MLA 2u
+int dsa_debug_stall(unsigned mask);
+
+/*
  * Stage 1, lightning indexer scores (section 4 step 2 of page 3).
  *
  *   q8      [T][Hi][128] e4m3 codes of the indexer queries
@@ -240,7 +260,11 @@ int dsa_window_indices(int T, int S, int q_pos0, int window, int k, int32_t *idx
                        dsa_stream_t stream);
 
 /*
- * Whole prefill path: indexer -> top-k -> sparse MLA for T query rows at
+ * Whole prefill path: indexer -> top-k -> sparse MLA, the chain of steps 2
+ * to 4 of the four-step workflow ("DeepSeek-V3.2-Exp 模型优势与 DSA 工作原理",
+ * section 4: scores, top-k selection, attention over the selected positions
+ * only) run over a whole prompt, the prefill phase page 1 distinguishes
+ * from decoding ("m.gxzdkb.com/media/457.html", section "秘密武器"), for T query rows at
  * positions q_pos0 .. q_pos0 + T - 1 against S cached keys (S >= q_pos0 + T
  * for a self-contained prefill). Query rows are scored in chunks of `chunk`
  * rows (0 = all rows at once); the workspace holds the scores of two chunks
@@ -294,7 +318,13 @@ int dsa_forward_fused(const void *q8, const float *q_scale, const void *k8,
                       dsa_stream_t stream);
 
 /*
- * Batched decode over a paged cache (blocks of 64 tokens).
+ * Batched decode over a paged cache (blocks of 64 tokens): the same three
+ * steps (page 3, section 4, steps 2-4) for the few new tokens of each
+ * sequence, the decoding phase page 1 (section "秘密武器") contrasts with
+ * prefill, each new query scoring and selecting from its own sequence's
+ * cached keys. The pages do not describe the cache's memory layout; the
+ * paged blocks of 64 tokens with a per-sequence block table are this
+ * library's layout for a batch of sequences of different lengths.
  *
  *   q8 [B][nq][Hi][128] e4m3, q_scale [B][nq] fp32 (or NULL), w [B][nq][Hi]
  *   q  [B][nq][H][576] bf16
@@ -346,6 +376,10 @@ int dsa_decode_paged(const void *q8, const float *q_scale, const float *w,
  *    ordering between them) race on it; serialise them. Every byte a call
  *    reads from the scratch is written earlier in the same call, so the
  *    previous call's leftovers never leak into a result.
+ *  - The array's device address is cached per device for the life of the
+ *    process. After cudaDeviceReset() (or anything else that unloads the
+ *    library's module from a device) the cached address is stale: do not
+ *    call this entry point on that device again in the same process.
  */
 int dsa_decode_paged_noalloc(const void *q8, const float *q_scale,
                              const float *w, const void *q,
@@ -357,7 +391,9 @@ int dsa_decode_paged_noalloc(const void *q8, const float *q_scale,
                              void *out, float *lse, dsa_stream_t stream);
 
 /*
- * The sparse MLA stage of the paged decode on its own: like
+ * The sparse MLA stage of the paged decode on its own (page 3, section 4,
+ * step 4, and section 3 "稀疏多潜在注意力": softmax attention of every head
+ * over the selected rows of the shared latent cache): like
  * dsa_sparse_mla_fwd, but `idx` [B*nq][k] holds logical positions of each
  * sequence, translated through block_table into kv_pool rows. A position
  * past the query's own position counts as out of range.

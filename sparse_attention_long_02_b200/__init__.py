@@ -38,6 +38,7 @@ _sig("dsa_status_string", ctypes.c_char_p, I32)
 _sig("dsa_version", I32)
 _sig("dsa_last_error_string", ctypes.c_char_p)
 _sig("dsa_get_device_error", I32, P)
+_sig("dsa_debug_stall", I32, ctypes.c_uint)
 _sig("dsa_indexer_scores", I32, P, P, P, P, P, I32, I32, I32, I32, F32, P, I64, P)
 _sig("dsa_topk", I32, P, I32, I32, I64, I32, I32, P, P)
 _sig("dsa_sparse_mla_fwd", I32, P, P, P, I32, I32, I32, I32, F32, P, P, P)
@@ -128,6 +129,17 @@ def _dev(t, dtype=None):
 
 def _ld(S):
     return (S + 3) // 4 * 4
+
+
+DEBUG_STALL_INDEXER = 1
+DEBUG_STALL_MLA = 2
+
+
+def debug_stall(mask: int) -> None:
+    """Debug aid: later launches of the named kernels (DEBUG_STALL_INDEXER,
+    DEBUG_STALL_MLA) on the current device wait on a barrier nothing arrives
+    at until their bounded wait runs out; 0 restores normal operation."""
+    _check(_lib.dsa_debug_stall(mask), "dsa_debug_stall")
 
 
 def get_device_error(stream=None) -> int:

@@ -10,8 +10,9 @@
 
 namespace dsa {
 
-// Per-device error word; kernels get its address as an argument.
-__device__ unsigned g_error_word;
+// Per-device status words, [0] the error bits and [1] the debug bits;
+// kernels get the address of [0] as an argument.
+__device__ unsigned g_error_word[2];
 
 namespace {
 
@@ -196,6 +197,15 @@ int dsa_get_device_error(dsa_stream_t stream) {
   if (v & kErrTimeout) return DSA_ERR_TIMEOUT;
   if (v & kErrBounds) return DSA_ERR_DEVICE_BOUNDS;
   return DSA_OK;
+}
+
+int dsa_debug_stall(unsigned mask) {
+  if (mask & ~static_cast<unsigned>(DSA_DEBUG_STALL_INDEXER | DSA_DEBUG_STALL_MLA))
+    return DSA_ERR_INVALID_ARG;
+  unsigned* p = device_error_word();
+  if (!p) return DSA_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return DSA_ERR_CUDA;
+  return status_of(cudaMemcpy(p + 1, &mask, sizeof mask, cudaMemcpyHostToDevice));
 }
 
 int dsa_indexer_scores(const void* q8, const float* q_scale, const void* k8, const float* k_scale,

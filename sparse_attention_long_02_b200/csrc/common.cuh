@@ -14,11 +14,21 @@
 namespace dsa {
 
 // ---------------------------------------------------------------- errors
-// Bits of the per-device error word (see dsa_get_device_error).
+// Every kernel gets the address of its device's status words: [0] holds the
+// error bits below (see dsa_get_device_error), [1] the debug bits set by
+// dsa_debug_stall (0 in normal use).
 enum : unsigned {
   kErrTimeout = 1u,   // a bounded wait gave up; the kernel returned early
   kErrBounds  = 2u,   // an index or block id was out of range and was skipped
 };
+enum : unsigned {
+  kDbgStallIndexer = 1u,  // the indexer's MMA issuer first waits on a barrier nothing arrives at
+  kDbgStallMla     = 2u,  // the same for the sparse MLA's MMA issuer
+};
+
+__device__ __forceinline__ unsigned debug_bits(const unsigned* err) {
+  return reinterpret_cast<const volatile unsigned*>(err)[1];
+}
 
 // A wait that has not completed after this long is treated as a hang.
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;   // 1 s

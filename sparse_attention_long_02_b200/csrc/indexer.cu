@@ -171,6 +171,10 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait(smem_u32(&sm.q_full), 0, abort_flag, err);
+      // debug: mma_done completes only after the commit below, so this
+      // bounded wait runs out and the CTA leaves through its give-up path
+      if (ok && (debug_bits(err) & kDbgStallIndexer))
+        ok = mbar_wait(smem_u32(&sm.mma_done), 0, abort_flag, err);
       const uint64_t bdesc = sdesc_sw128(smem_u32(sm.q), 0, 1024);
       for (int i = 0; ok && i < ntiles; ++i) {
         const int st = i % kStages, buf = i & 1;

@@ -256,14 +256,18 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (ok) mbar_arrive_remote(mapa(smem_u32(&sm.peer_q), peer));
       ok = ok && mbar_wait<true>(smem_u32(&sm.peer_q), 0, abort_flag, err);
       ok = ok && (ntiles == 0 || send(0));
+      // The receipt of tile i is acknowledged before tile i+1 is sent: the
+      // peer stages its tile i+1 into its single stage buffer only after that
+      // acknowledgement, and this warp's send(i+1) waits for this CTA's own
+      // staging, which waits for the peer's acknowledgement of tile i.
       for (int i = 0; ok && i < ntiles; ++i) {
         const int b = i & 1;
-        if (i + 1 < ntiles && !(ok = send(i + 1))) break;
         if (!(ok = mbar_wait<true>(smem_u32(&sm.x_full[b]), (i >> 1) & 1, abort_flag, err))) break;
         mbar_arrive_remote(mapa(smem_u32(&sm.stage_free), peer));
         if (i + 2 < ntiles) mbar_expect_tx(smem_u32(&sm.x_full[b]), kXBytes);   // tile i+2
         if (!(ok = mbar_wait(smem_u32(&sm.x_read[b]), (i >> 1) & 1, abort_flag, err))) break;
         mbar_arrive_remote(mapa(smem_u32(&sm.x_free[b]), peer));
+        if (i + 1 < ntiles && !(ok = send(i + 1))) break;
       }
       // A copy reads this CTA's stage buffer until it lands: wait for the
       // peer's word on the last one before this CTA may leave (the softmax
@@ -279,6 +283,10 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const uint32_t id_qk = idesc_bf16(128, kTileKeys, false);
       const uint32_t id_pv = idesc_bf16(128, 256, true);
       bool ok = mbar_wait(smem_u32(&sm.q_ready), 0, abort_flag, err);
+      // debug: o_done completes only after the commit below, so this bounded
+      // wait runs out and both CTAs leave through their give-up paths
+      if (ok && (debug_bits(err) & kDbgStallMla))
+        ok = mbar_wait(smem_u32(&sm.o_done), 0, abort_flag, err);
       auto issue_pv = [&](int i) -> bool {
         const int st = i % kStages;
         if (!mbar_wait(smem_u32(&sm.p_full), i & 1, abort_flag, err)) return false;
