@@ -318,6 +318,18 @@ int dsa_forward_fused(const void *q8, const float *q_scale, const void *k8,
                       dsa_stream_t stream);
 
 /*
+ * Diagnostic for dsa_forward_fused (no counterpart on the pages): how many
+ * rows of the last call that used `workspace` (with the same T, S, k and
+ * chunk) missed their candidate window and were recomputed on CUDA cores.
+ * Synchronises `stream`; returns the count (>= 0) or a negative status.
+ * Recomputed scores are summed in another order than the tensor cores', so
+ * on inputs off the exact FP8 grid they equal the indexer's scores only to
+ * within fp32 rounding (their selection then agrees within the tie rule).
+ */
+int dsa_forward_fused_fallback_rows(const void *workspace, int T, int S, int k,
+                                    int chunk, dsa_stream_t stream);
+
+/*
  * Batched decode over a paged cache (blocks of 64 tokens): the same three
  * steps (page 3, section 4, steps 2-4) for the few new tokens of each
  * sequence, the decoding phase page 1 (section "秘密武器") contrasts with

@@ -55,6 +55,7 @@ _sig("dsa_forward_workspace_size", SZ, I32, I32, I32, I32, I32, I32)
 _sig("dsa_forward_fused_workspace_size", SZ, I32, I32, I32, I32, I32, I32)
 _sig("dsa_forward_fused", I32, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, F32, F32,
      P, P, P, P, SZ, P)
+_sig("dsa_forward_fused_fallback_rows", I32, P, I32, I32, I32, I32, P)
 _sig("dsa_forward", I32, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, F32, F32,
      P, P, P, P, SZ, P)
 _sig("dsa_decode_paged_workspace_size", SZ, I32, I32, I32, I32, I32, I32)
@@ -336,6 +337,15 @@ def forward_fused(q8, q_scale, k8, k_scale, w, q, kv, k, scale, sm_scale, q_pos0
                                   float(sm_scale), _p(idx), _p(out), _p(lse), _p(workspace),
                                   workspace.numel(), _stream(stream)), "dsa_forward_fused")
     return out, lse, idx
+
+
+def forward_fused_fallback_rows(workspace, T, S, k, chunk=0, stream=None) -> int:
+    """Rows of the last forward_fused call on `workspace` that were recomputed on
+    CUDA cores (their candidate count missed [k, 4096]); synchronises."""
+    n = _lib.dsa_forward_fused_fallback_rows(_p(workspace), T, S, k, chunk, _stream(stream))
+    if n < 0:
+        _check(n, "dsa_forward_fused_fallback_rows")
+    return n
 
 
 def decode_workspace_size(B, nq, max_blocks, Hi, H, k) -> int:

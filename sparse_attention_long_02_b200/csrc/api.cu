@@ -406,7 +406,7 @@ long long sample_count(int S) {
 // Workspace of the fused path, each part 256-byte aligned.
 struct FusedLayout {
   long long M, ldm, ld;
-  size_t k8s, kss, sample, tau, cnt, ckey, cidx, fail, scratch, idx, total;
+  size_t k8s, kss, sample, tau, cnt, ckey, cidx, fail, fail_total, scratch, idx, total;
 };
 
 FusedLayout fused_layout(int T, int S, int k, int chunk) {
@@ -429,6 +429,7 @@ FusedLayout fused_layout(int T, int S, int k, int chunk) {
   L.ckey = take(rows * kFusedCandCap * 4);
   L.cidx = take(rows * kFusedCandCap * 4);
   L.fail = take(4 + rows * 4);
+  L.fail_total = take(4);
   L.scratch = take(static_cast<size_t>(kFusedSlots) * L.ld * 4);
   L.idx = take(static_cast<size_t>(T) * k * 4);
   L.total = off;
@@ -574,6 +575,7 @@ int dsa_forward_fused(const void* q8, const float* q_scale, const void* k8, cons
   if (e == cudaSuccess && kss && tail > 0)
     e = cudaMemcpyAsync(kss + full * 256, k_scale + full * 4096, tail * 4,
                         cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.fail_total, 0, 4, st);
   if (e != cudaSuccess) return status_of(e);
   for (int c0 = 0; c0 < T; c0 += rows) {
     const int n = std::min(rows, T - c0);
@@ -615,6 +617,7 @@ int dsa_forward_fused(const void* q8, const float* q_scale, const void* k8, cons
     F.cand_cap = kFusedCandCap;
     F.fail_count = reinterpret_cast<unsigned*>(ws + L.fail);
     F.fail_rows = reinterpret_cast<int*>(ws + L.fail) + 1;
+    F.fail_total = reinterpret_cast<unsigned*>(ws + L.fail_total);
     F.q8 = q8c;
     F.q_scale = qsc;
     F.k8 = k8b;
@@ -646,6 +649,20 @@ int dsa_forward_fused(const void* q8, const float* q_scale, const void* k8, cons
     if (e != cudaSuccess) return status_of(e);
   }
   return dsa_sparse_mla_fwd(q, kv, idx, T, S, H, k, sm_scale, out, lse, stream);
+}
+
+int dsa_forward_fused_fallback_rows(const void* workspace, int T, int S, int k, int chunk,
+                                    dsa_stream_t stream) {
+  if (!workspace || T <= 0 || S <= 0 || k <= 0 || k > 2048 || S > kFusedMaxS)
+    return DSA_ERR_INVALID_ARG;
+  const FusedLayout L = fused_layout(T, S, k, chunk);
+  unsigned v = 0;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess)
+    e = cudaMemcpy(&v, static_cast<const char*>(workspace) + L.fail_total, sizeof v,
+                   cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return status_of(e);
+  return static_cast<int>(v);
 }
 
 size_t dsa_decode_paged_workspace_size(int B, int nq, int max_blocks, int Hi, int H, int k) {

@@ -62,6 +62,7 @@ struct FusedSelArgs {
   const int* cand_idx = nullptr;          // [T][cand_cap]
   int cand_cap = 0;
   unsigned* fail_count = nullptr;         // [1], zero before the select
+  unsigned* fail_total = nullptr;         // [1], rows sent to the recompute in the whole call
   int* fail_rows = nullptr;               // [T]
   // inputs of the recompute (rows of this call; keys of the whole cache)
   const uint8_t* q8 = nullptr;

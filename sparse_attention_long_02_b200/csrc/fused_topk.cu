@@ -80,7 +80,10 @@ __global__ void __launch_bounds__(kTopkThreads, 1) select_kernel(const FusedSelA
   const unsigned cnt = A.cand_count[r];
   if (cnt < static_cast<unsigned>(A.k) || cnt > static_cast<unsigned>(A.cand_cap) ||
       A.cand_cap > kCandCap || n > kSampledMaxN) {
-    if (tid == 0) A.fail_rows[atomicAdd(A.fail_count, 1u)] = r;
+    if (tid == 0) {
+      A.fail_rows[atomicAdd(A.fail_count, 1u)] = r;
+      atomicAdd(A.fail_total, 1u);
+    }
     return;
   }
   const unsigned* ck = A.cand_key + static_cast<long long>(r) * A.cand_cap;
@@ -102,7 +105,10 @@ __device__ __forceinline__ float e4m3_float(uint8_t c) {
 // One listed row per CTA at a time: its scores over keys 0 .. pos, the same
 // formula as the indexer (the dot product of the e4m3 codes in fp32, ReLU,
 // the folded weight w * scale * q_scale, the sum over heads, then k_scale),
-// into this CTA's scratch row; then the full top-k of that row.
+// into this CTA's scratch row; then the full top-k of that row. The sums run
+// in another order than the tensor cores' and the indexer epilogue's, so a
+// recomputed score equals the indexer's exactly only where every partial sum
+// is exact (the integer FP8 grid), and otherwise to within fp32 rounding.
 template <int HI>
 __global__ void __launch_bounds__(kTopkThreads, 1) fallback_kernel(const FusedSelArgs A) {
   extern __shared__ __align__(16) uint8_t smem_raw[];

@@ -60,9 +60,10 @@ constexpr uint32_t kColO = 0;                    // TMEM columns [0,256): output
 constexpr uint32_t kColQ = 256;                  // [256,400): Q_c, bf16 pairs (256 + 32 dims)
 constexpr uint32_t kColP = 416;                  // [416,448): P, bf16 pairs
 constexpr uint32_t kColS = 448;                  // [448,512): logits
-// Q arrives by TMA in the exchange buffers (the latent atoms in x, the rope
-// block in stage) and is moved into TMEM before the first exchange, so the
-// whole KV ring is free for the gather from the first tile.
+// Q arrives by TMA in the exchange buffers (latent atoms 0-1 in x, 2-3 in
+// stage[0], the rope block in stage[1]) and is moved into TMEM before the
+// first exchange, so the whole KV ring is free for the gather from the first
+// tile.
 constexpr float kRebase = 8.0f;                  // lazy rescale threshold (log2 units)
 
 // Rows of 64 fp32 partials (256 B, one per head); the 16-B chunk c of row h
@@ -70,8 +71,8 @@ constexpr float kRebase = 8.0f;                  // lazy rescale threshold (log2
 struct MlaSmem {
   uint8_t kv[kStages][kAtoms][kAtomBytesKV];
   uint8_t kv_rope[kStages][kRopeBytesKV];
-  uint4 x[2][128 * 16];                          // the peer's partials, by tile parity
-  uint4 stage[128 * 16];                         // this CTA's partials (bulk copy source)
+  uint4 x[128 * 16];                             // the peer's partials of the current tile
+  uint4 stage[2][128 * 16];                      // this CTA's partials (bulk copy source), by tile parity
   float pair_max[2][2][128];                     // [tile parity][key half][head]
   unsigned valid[kStages][2];                    // selected-slot bits of each half tile
   unsigned long long q_full;                     // Q has landed in its staging slots
@@ -83,32 +84,48 @@ struct MlaSmem {
   unsigned long long s_empty;
   unsigned long long p_full;
   unsigned long long p_empty;
-  unsigned long long stage_full;                 // the eight softmax warps have staged a tile
-  unsigned long long stage_free;                 // the peer has received the tile staged here
-  // per receive buffer (tile parity):
-  unsigned long long x_full[2];                  // the peer's partials have landed in x
-  unsigned long long x_free[2];                  // the peer has read what this CTA sent it
-  unsigned long long x_read[2];                  // the softmax warps have read x
+  // per send buffer (tile parity):
+  unsigned long long stage_full[2];              // the eight softmax warps have staged a tile
+  unsigned long long stage_free[2];              // the peer has received the tile staged here
+  unsigned long long x_full;                     // the peer's partials have landed in x
+  unsigned long long x_free;                     // the peer has read what this CTA sent it
+  unsigned long long x_read;                     // the softmax warps have read x
   unsigned long long pair;                       // the softmax warps have posted their maxima
   unsigned long long o_done;
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// Q staging: latent atoms 0-1 in x[0], 2-3 in x[1], the rope block in stage.
-static_assert(sizeof(MlaSmem::x[0]) == 2 * kAtomBytesQ, "two Q atoms per receive buffer");
-static_assert(sizeof(MlaSmem::stage) >= kRopeBytesQ, "Q rope block fits the stage buffer");
+static_assert(sizeof(MlaSmem::x) == 2 * kAtomBytesQ, "two Q atoms per exchange buffer");
+static_assert(sizeof(MlaSmem::stage[0]) == 2 * kAtomBytesQ, "two Q atoms per exchange buffer");
+static_assert(sizeof(MlaSmem::stage[1]) >= kRopeBytesQ, "Q rope block fits a stage buffer");
 static_assert(kAtomBytesKV % 1024 == 0 && kRopeBytesKV % 1024 == 0, "1024-B aligned staging");
 
-// Physical row of slot value `v` (a logical position), or -1 if skipped.
-__device__ __forceinline__ int kv_row(const MlaArgs& A, int v, int seq, int limit) {
+// Shared-memory address of Q staging atom a (0-3): atoms 0-1 in x, 2-3 in
+// stage[0]; and the generic pointer of a shared-memory address of `sm`.
+__device__ __forceinline__ uint32_t q_atom(MlaSmem& sm, int a) {
+  return (a < 2 ? smem_u32(sm.x) : smem_u32(sm.stage[0])) + (a & 1) * kAtomBytesQ;
+}
+__device__ __forceinline__ const uint8_t* smem_generic(MlaSmem& sm, uint32_t saddr) {
+  return reinterpret_cast<const uint8_t*>(&sm) + (saddr - smem_u32(&sm));
+}
+
+// Physical block of slot value `v` (a logical position) in the paged cache,
+// loaded a tile ahead of its use; -1 when no lookup is needed.
+__device__ __forceinline__ int kv_block(const MlaArgs& A, int v, int seq, int limit) {
+  if (!A.block_table || v < 0 || v >= limit) return -1;
+  return __ldg(A.block_table + static_cast<long long>(seq) * A.max_blocks + (v >> 6));
+}
+
+// Physical row of slot value `v` given its block `pb` (kv_block), or -1 if
+// the slot is skipped.
+__device__ __forceinline__ int kv_row(const MlaArgs& A, int v, int pb, int limit) {
   if (v < 0) return -1;
   if (v >= limit) {
     raise_error(A.err, kErrBounds);
     return -1;
   }
   if (!A.block_table) return v;
-  const int pb = A.block_table[static_cast<long long>(seq) * A.max_blocks + (v >> 6)];
   if (pb < 0 || pb >= A.nblk) {
     raise_error(A.err, kErrBounds);
     return -1;
@@ -152,13 +169,13 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mbar_init(smem_u32(&sm.s_empty), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.p_full), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.p_empty), 1);
-    mbar_init(smem_u32(&sm.stage_full), kSoftmaxWarps);
-    mbar_init(smem_u32(&sm.stage_free), 1);      // one arrival from the peer per use
     for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&sm.x_full[b]), 1);      // own expect_tx + the peer's copied bytes
-      mbar_init(smem_u32(&sm.x_free[b]), 1);      // one arrival from the peer per use
-      mbar_init(smem_u32(&sm.x_read[b]), kSoftmaxWarps);
+      mbar_init(smem_u32(&sm.stage_full[b]), kSoftmaxWarps);
+      mbar_init(smem_u32(&sm.stage_free[b]), 1);  // one arrival from the peer per use
     }
+    mbar_init(smem_u32(&sm.x_full), 1);          // own expect_tx + the peer's copied bytes
+    mbar_init(smem_u32(&sm.x_free), 1);          // one arrival from the peer per use
+    mbar_init(smem_u32(&sm.x_read), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.pair), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.o_done), 1);
     sm.abort_flag = aborted ? 1 : 0;
@@ -185,21 +202,29 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const uint32_t qf = smem_u32(&sm.q_full);
       mbar_expect_tx(qf, kAtoms * kAtomBytesQ + kRopeBytesQ);
       for (int a = 0; a < kAtoms; ++a)
-        tma_load_2d(smem_u32(sm.x[a >> 1]) + (a & 1) * kAtomBytesQ, &tm_q, qf, dim0 + 64 * a,
-                    r * A.H);
-      tma_load_2d(smem_u32(sm.stage), &tm_qr, qf, rope0, r * A.H);
+        tma_load_2d(q_atom(sm, a), &tm_q, qf, dim0 + 64 * a, r * A.H);
+      tma_load_2d(smem_u32(sm.stage[1]), &tm_qr, qf, rope0, r * A.H);
     }
-    int v0 = lane < A.k ? __ldg(sel + lane) : -1;
-    int v1 = lane + 32 < A.k ? __ldg(sel + lane + 32) : -1;
+    // Two-deep prefetch: the slots of tile i+2 and the block-table entries
+    // of tile i+1 are loading while tile i is issued.
+    auto slot = [&](int j) { return j < A.k ? __ldg(sel + j) : -1; };
+    int v0 = slot(lane), v1 = slot(lane + 32);                          // tile 0
+    int b0 = kv_block(A, v0, seq, limit), b1 = kv_block(A, v1, seq, limit);
+    int n0 = slot(kTileKeys + lane), n1 = slot(kTileKeys + lane + 32);  // tile 1
     for (int i = 0; i < ntiles; ++i) {
       const int st = i % kStages;
-      const int c0 = v0, c1 = v1;
-      const int j0 = (i + 1) * kTileKeys + lane;                    // prefetch the next tile
+      const int c0 = v0, c1 = v1, p0 = b0, p1 = b1;
       if (i + 1 < ntiles) {
-        v0 = j0 < A.k ? __ldg(sel + j0) : -1;
-        v1 = j0 + 32 < A.k ? __ldg(sel + j0 + 32) : -1;
+        v0 = n0;
+        v1 = n1;
+        b0 = kv_block(A, v0, seq, limit);
+        b1 = kv_block(A, v1, seq, limit);
       }
-      const int r0 = kv_row(A, c0, seq, limit), r1 = kv_row(A, c1, seq, limit);
+      if (i + 2 < ntiles) {
+        n0 = slot((i + 2) * kTileKeys + lane);
+        n1 = slot((i + 2) * kTileKeys + lane + 32);
+      }
+      const int r0 = kv_row(A, c0, p0, limit), r1 = kv_row(A, c1, p1, limit);
       if (i >= kStages &&
           !warp_wait(smem_u32(&sm.kv_empty[st]), ((i / kStages) + 1) & 1, abort_flag, err))
         break;
@@ -229,52 +254,49 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (warp == 0 && lane == 0) mbar_drain(smem_u32(&sm.q_full), 0);
   } else if (warp == kExchangeWarp && !aborted) {
     // ---------------------------------------------------- exchange warp
-    // Tile j's partials travel from stage to the peer's x[j & 1] in one bulk
-    // copy, once they are staged and the peer has read tile j-2 out of that
-    // buffer (for the first two tiles: once the peer has moved its Q, which
-    // is staged in x, into TMEM). This warp also tells the peer when its copy
-    // of tile i has landed here (its stage buffer may be refilled) and when x
-    // has been read (it may send into that buffer again). Cluster-scope
-    // releases come from this warp only, so they never queue behind the
-    // softmax warps.
+    // Tile j's partials travel from stage[j & 1] to the peer's x in one bulk
+    // copy, once they are staged and the peer has read tile j-1 out of x
+    // (for tile 0: once the peer has moved its Q, which is staged in x, into
+    // TMEM). The send side is double-buffered, so staging tile j+1 never
+    // waits for tile j's copy; the receive side is single, so the copy of
+    // tile j+1 starts once both CTAs have read tile j, while both finish it.
+    // This warp also tells the peer when its copy of tile i has landed here
+    // (that stage buffer may be refilled) and when x has been read (it may
+    // send the next tile). Cluster-scope releases come from this warp only,
+    // so they never queue behind the softmax warps.
     if (lane == 0) {
       int sent = 0;
       auto send = [&](int j) -> bool {
         const int b = j & 1;
-        if (!mbar_wait(smem_u32(&sm.stage_full), j & 1, abort_flag, err)) return false;
-        if (j >= 2 && !mbar_wait<true>(smem_u32(&sm.x_free[b]), ((j - 2) >> 1) & 1, abort_flag, err))
+        if (!mbar_wait(smem_u32(&sm.stage_full[b]), (j >> 1) & 1, abort_flag, err)) return false;
+        if (j >= 1 && !mbar_wait<true>(smem_u32(&sm.x_free), (j - 1) & 1, abort_flag, err))
           return false;
-        bulk_copy_to_peer(mapa(smem_u32(sm.x[b]), peer), smem_u32(sm.stage), kXBytes,
-                          mapa(smem_u32(&sm.x_full[b]), peer));
+        bulk_copy_to_peer(mapa(smem_u32(sm.x), peer), smem_u32(sm.stage[b]), kXBytes,
+                          mapa(smem_u32(&sm.x_full), peer));
         sent = j + 1;
         return true;
       };
-      for (int j = 0; j < 2 && j < ntiles; ++j)                 // the peer's tiles 0 and 1
-        mbar_expect_tx(smem_u32(&sm.x_full[j]), kXBytes);
+      if (ntiles > 0) mbar_expect_tx(smem_u32(&sm.x_full), kXBytes);        // the peer's tile 0
       // this CTA's Q has left x: the peer may send into it
       bool ok = mbar_wait(smem_u32(&sm.q_ready), 0, abort_flag, err);
       if (ok) mbar_arrive_remote(mapa(smem_u32(&sm.peer_q), peer));
       ok = ok && mbar_wait<true>(smem_u32(&sm.peer_q), 0, abort_flag, err);
       ok = ok && (ntiles == 0 || send(0));
-      // The receipt of tile i is acknowledged before tile i+1 is sent: the
-      // peer stages its tile i+1 into its single stage buffer only after that
-      // acknowledgement, and this warp's send(i+1) waits for this CTA's own
-      // staging, which waits for the peer's acknowledgement of tile i.
       for (int i = 0; ok && i < ntiles; ++i) {
-        const int b = i & 1;
-        if (!(ok = mbar_wait<true>(smem_u32(&sm.x_full[b]), (i >> 1) & 1, abort_flag, err))) break;
-        mbar_arrive_remote(mapa(smem_u32(&sm.stage_free), peer));
-        if (i + 2 < ntiles) mbar_expect_tx(smem_u32(&sm.x_full[b]), kXBytes);   // tile i+2
-        if (!(ok = mbar_wait(smem_u32(&sm.x_read[b]), (i >> 1) & 1, abort_flag, err))) break;
-        mbar_arrive_remote(mapa(smem_u32(&sm.x_free[b]), peer));
+        if (!(ok = mbar_wait<true>(smem_u32(&sm.x_full), i & 1, abort_flag, err))) break;
+        mbar_arrive_remote(mapa(smem_u32(&sm.stage_free[i & 1]), peer));
+        if (!(ok = mbar_wait(smem_u32(&sm.x_read), i & 1, abort_flag, err))) break;
+        // armed before the peer may send tile i+1 (it waits for x_free)
+        if (i + 1 < ntiles) mbar_expect_tx(smem_u32(&sm.x_full), kXBytes);
+        mbar_arrive_remote(mapa(smem_u32(&sm.x_free), peer));
         if (i + 1 < ntiles && !(ok = send(i + 1))) break;
       }
       // A copy reads this CTA's stage buffer until it lands: wait for the
-      // peer's word on the last one before this CTA may leave (the softmax
+      // peer's word on the last two before this CTA may leave (the softmax
       // warps waited for every earlier one before restaging).
-      if (sent > 0) {
-        const uint32_t bar = smem_u32(&sm.stage_free);
-        if (!mbar_wait<true>(bar, (sent - 1) & 1, abort_flag, err)) mbar_drain(bar, (sent - 1) & 1);
+      for (int j = sent > 2 ? sent - 2 : 0; j < sent; ++j) {
+        const uint32_t bar = smem_u32(&sm.stage_free[j & 1]);
+        if (!mbar_wait<true>(bar, (j >> 1) & 1, abort_flag, err)) mbar_drain(bar, (j >> 1) & 1);
       }
     }
   } else if (warp == 1 && !aborted) {
@@ -347,8 +369,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if ((ok = warp_wait(smem_u32(&sm.q_full), 0, abort_flag, err))) {
 #pragma unroll 1
         for (int a = 0; a < kAtoms; ++a) {
-          const uint8_t* qs = reinterpret_cast<const uint8_t*>(sm.x[a >> 1]) + (a & 1) * kAtomBytesQ;
-          const uint4* row = reinterpret_cast<const uint4*>(qs + h * 128);
+          const uint4* row = reinterpret_cast<const uint4*>(smem_generic(sm, q_atom(sm, a)) + h * 128);
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             uint32_t pk[16];
@@ -365,7 +386,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         {
           const uint4* row = reinterpret_cast<const uint4*>(
-              reinterpret_cast<const uint8_t*>(sm.stage) + h * 64);
+              reinterpret_cast<const uint8_t*>(sm.stage[1]) + h * 64);
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -383,10 +404,10 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
     }
     // This warp's half of tile j's partial logits, scaled into log2 units
-    // (fp32), staged for the peer. The stage buffer is single: tile j may
-    // be staged once the copy of tile j-1 has landed at the peer, which is
-    // also after this CTA has read tile j-1's own partials back (below).
+    // (fp32), staged for the peer in stage[j & 1] once the copy of tile j-2
+    // out of that buffer has landed.
     auto stage_tile = [&](int j) -> bool {
+      const int b = j & 1;
       float v32[32];
       if (!warp_wait(smem_u32(&sm.s_full), j & 1, abort_flag, err)) return false;
       tc_fence_after();
@@ -394,10 +415,10 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty));
-      if (j >= 1 &&
-          !warp_wait<true>(smem_u32(&sm.stage_free), (j - 1) & 1, abort_flag, err))
+      if (j >= 2 &&
+          !warp_wait<true>(smem_u32(&sm.stage_free[b]), ((j - 2) >> 1) & 1, abort_flag, err))
         return false;
-      uint4* dst = sm.stage + h * 16;
+      uint4* dst = sm.stage[b] + h * 16;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         dst[(8 * g + c) ^ (h & 7)] =
@@ -407,7 +428,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                        __float_as_uint(v32[4 * c + 3] * A.sm_scale_log2));
       fence_proxy_async_smem();           // generic writes -> the bulk copy's reads
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.stage_full));
+      if (lane == 0) mbar_arrive(smem_u32(&sm.stage_full[b]));
       return true;
     };
     if (ok && ntiles > 0) ok = stage_tile(0);
@@ -417,11 +438,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (!(ok = warp_wait(smem_u32(&sm.kv_full[st]), (i / kStages) & 1, abort_flag, err))) break;
       const unsigned valid = sm.valid[st][g];
       // own + peer partials, then hand x back
-      if (!(ok = warp_wait<true>(smem_u32(&sm.x_full[b]), (i >> 1) & 1, abort_flag, err))) break;
+      if (!(ok = warp_wait<true>(smem_u32(&sm.x_full), i & 1, abort_flag, err))) break;
       float s[32];
       {
-        const uint4* xp = sm.x[b] + h * 16;
-        const uint4* op = sm.stage + h * 16;
+        const uint4* xp = sm.x + h * 16;
+        const uint4* op = sm.stage[b] + h * 16;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const uint4 f = xp[(8 * g + c) ^ (h & 7)];
@@ -433,7 +454,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.x_read[b]));
+      if (lane == 0) mbar_arrive(smem_u32(&sm.x_read));
       // the next tile's partials go out while this one is finished
       if (i + 1 < ntiles && !(ok = stage_tile(i + 1))) break;
       if (valid != 0xffffffffu) {

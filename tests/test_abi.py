@@ -130,12 +130,12 @@ def test_workspace_sizes(dsa):
     assert L.dsa_forward_workspace_size(0, 8, 4, 8, 4, 0) == 0
     # fused prefill: the sampled keys (the first 256 of every 4096) and their
     # scales, per chunk row the sample scores, threshold, count and 4096
-    # candidates, the failure list, 148 scratch score rows, and idx
+    # candidates, the failure list, the call's failure total, 148 scratch score rows, and idx
     r256 = lambda x: (x + 255) // 256 * 256
     T, S, k, rows = 131072, 131072, 2048, 4096
     M = 32 * 256
     parts = [M * 128, M * 4, rows * M * 4, rows * 4, rows * 4, rows * 4096 * 4, rows * 4096 * 4,
-             4 + rows * 4, 148 * S * 4, T * k * 4]
+             4 + rows * 4, 4, 148 * S * 4, T * k * 4]
     assert L.dsa_forward_fused_workspace_size(T, S, 64, 128, k, rows) == sum(r256(x) for x in parts)
     assert L.dsa_forward_fused_workspace_size(T, S, 64, 128, 4096, rows) == 0
     # warm-up target: T * H rows of fp32 logits, S rounded up to 4
