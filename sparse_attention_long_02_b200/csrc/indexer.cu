@@ -36,11 +36,17 @@ constexpr int kKeyTile = 128;      // keys per MMA tile (M)
 constexpr int kStages = 4;         // key-tile ring depth
 constexpr int kKTileBytes = kKeyTile * 128;
 
+// Filter mode: each CTA first appends its candidates to per-query lists in
+// shared memory (this many bytes in all) and copies them out once at the end.
+constexpr int kCandSmemBytes = 64 * 1024;
+
 struct IdxSmem {
   // operand tiles first (1024-B aligned by construction of the offsets)
   uint8_t q[256 * 128];                 // B operand: QB*HI rows x 128 B
   uint8_t k[kStages][kKTileBytes];      // A operand ring
   float w[256];                         // w[t,h]*scale*q_scale[t] for the CTA's queries
+  uint32_t tau[64];                     // filter mode: the CTA's queries' thresholds
+  uint32_t cand_n[64];                  // filter mode: entries in each query's list
   unsigned long long q_full;
   unsigned long long k_full[kStages];
   unsigned long long k_empty[kStages];
@@ -59,9 +65,13 @@ __global__ void __maxnreg__(128)
 indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const IndexerArgs a) {
   constexpr int QB = (256 / HI) < 64 ? (256 / HI) : 64;   // queries per CTA (prefill)
+  constexpr int kCapS = kCandSmemBytes / (QB * 8);         // shared-memory entries per query
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   IdxSmem& sm = *reinterpret_cast<IdxSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // filter mode: [QB][kCapS] order keys, then [QB][kCapS] key positions
+  uint32_t* cs_key = reinterpret_cast<uint32_t*>(&sm + 1);
+  int* cs_idx = reinterpret_cast<int*>(cs_key + QB * kCapS);
   unsigned* err = a.err;
   if (launch_aborted(err)) return;
 
@@ -108,6 +118,11 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     mbar_init(smem_u32(&sm.mma_done), 1);
     sm.abort_flag = 0;
     fence_barrier_init();
+  }
+  if (!PAGED && a.tau && threadIdx.x < QB) {
+    const int qq = threadIdx.x;
+    sm.cand_n[qq] = 0;
+    sm.tau[qq] = qq < nqb ? a.tau[q0 + qq] : 0xffffffffu;
   }
   // folded per-(query, head) weights: w * scale * q_scale
   for (int j = threadIdx.x; j < ncol; j += blockDim.x) {
@@ -211,22 +226,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       return __ldg(a.k_scale + s);
     };
     float ks_next = key_scale(g);
-    // filter mode: the last appended query's ballot and its atomic's result
-    bool pend = false, p_keep = false;
-    uint32_t p_key = 0;
-    unsigned p_ball = 0, p_base = 0;
-    long long p_t = 0;
-    int p_s = 0;
-    auto flush_pending = [&]() {
-      if (!pend) return;                           // warp-uniform
-      const unsigned base = __shfl_sync(0xffffffffu, p_base, 0);
-      const unsigned slot = base + __popc(p_ball & ((1u << lane) - 1u));
-      if (p_keep && slot < static_cast<unsigned>(a.cand_cap)) {
-        a.cand_key[p_t * a.cand_cap + slot] = p_key;
-        a.cand_idx[p_t * a.cand_cap + slot] = p_s;
-      }
-      pend = false;
-    };
+    const unsigned lane_lt = (1u << lane) - 1u;
     for (int i = g; i < ntiles; i += 2) {
       const float ks = ks_next;
       ks_next = key_scale(i + 2);
@@ -244,28 +244,37 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       };
       // Called by the whole warp with the same qq. Scores mode writes the
       // row; filter mode appends (order key, key) of every score at or above
-      // the row's threshold to its candidate list: one atomic per warp and
-      // query, whose slot is used only at the next call, so that a chunk of
-      // the epilogue runs while the atomic returns.
+      // the query's threshold to the query's list in shared memory (one
+      // shared atomic per warp and query), or, once that list is full,
+      // straight to the row's list in global memory.
       auto emit = [&](int qq, float acc) {
         if (qq >= nqb) return;
         const long long t = q0 + qq;
         const long long pos = pos0 + qq;
-        if (a.tau) {
-          flush_pending();
+        if (!PAGED && a.tau) {
           const uint32_t key = score_key(acc * ks);
-          const bool keep = key_ok && s <= pos && key >= a.tau[t];
+          const bool keep = key_ok && s <= pos && key >= sm.tau[qq];
           const unsigned ball = __ballot_sync(0xffffffffu, keep);
           if (ball) {
             unsigned base = 0;
-            if (lane == 0) base = atomicAdd(a.cand_count + t, static_cast<unsigned>(__popc(ball)));
-            pend = true;
-            p_key = key;
-            p_keep = keep;
-            p_ball = ball;
-            p_base = base;
-            p_t = t;
-            p_s = static_cast<int>(s);
+            if (lane == 0) base = atomicAdd(&sm.cand_n[qq], static_cast<unsigned>(__popc(ball)));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            const unsigned slot = base + __popc(ball & lane_lt);
+            const bool local = slot < static_cast<unsigned>(kCapS);
+            if (keep && local) {
+              cs_key[qq * kCapS + slot] = key;
+              cs_idx[qq * kCapS + slot] = static_cast<int>(s);
+            }
+            const unsigned over = __ballot_sync(0xffffffffu, keep && !local);
+            if (over) {
+              unsigned gb = 0;
+              if (lane == 0) gb = atomicAdd(a.cand_count + t, static_cast<unsigned>(__popc(over)));
+              gb = __shfl_sync(0xffffffffu, gb, 0) + __popc(over & lane_lt);
+              if (keep && !local && gb < static_cast<unsigned>(a.cand_cap)) {
+                a.cand_key[t * a.cand_cap + gb] = key;
+                a.cand_idx[t * a.cand_cap + gb] = static_cast<int>(s);
+              }
+            }
           }
           return;
         }
@@ -319,13 +328,31 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
       }
     }
-    flush_pending();
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, a.tmem_cols);
+  }
+  // filter mode: each query's shared-memory list goes to the row's list in
+  // global memory with one atomic (entries past the row's capacity are
+  // dropped; the count still tells the select kernel the row overflowed)
+  if (!PAGED && a.tau) {
+    for (int qq = warp; qq < nqb; qq += kIdxThreads / 32) {
+      const unsigned n = min(sm.cand_n[qq], static_cast<unsigned>(kCapS));
+      if (n == 0) continue;
+      const long long t = q0 + qq;
+      unsigned gb = 0;
+      if (lane == 0) gb = atomicAdd(a.cand_count + t, n);
+      gb = __shfl_sync(0xffffffffu, gb, 0);
+      for (unsigned j = lane; j < n; j += 32) {
+        if (gb + j < static_cast<unsigned>(a.cand_cap)) {
+          a.cand_key[t * a.cand_cap + gb + j] = cs_key[qq * kCapS + j];
+          a.cand_idx[t * a.cand_cap + gb + j] = cs_idx[qq * kCapS + j];
+        }
+      }
+    }
   }
 }
 
@@ -334,7 +361,8 @@ cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const Index
                        dim3 grid, cudaStream_t st) {
   // Above half the SM's shared memory, so one CTA per SM: a second resident
   // CTA would only queue on the TMEM allocation.
-  const size_t smem = std::max<size_t>(sizeof(IdxSmem) + 1024, 120 * 1024);
+  const size_t smem = std::max<size_t>(sizeof(IdxSmem) + 1024, 120 * 1024) +
+                      (a.tau ? kCandSmemBytes : 0);
   auto kern = indexer_kernel<HI, PAGED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
