@@ -55,6 +55,11 @@ def parse():
                     help="fused: dsa_forward_fused (top-k fused into the indexer, no score rows "
                          "in HBM); scores: dsa_forward (each chunk's scores in HBM, read back by "
                          "the top-k)")
+    ap.add_argument("--profile", default="", choices=["", "chunk", "decode"],
+                    help="small cases for ncu captures: chunk = the last 4096 query rows of the "
+                         "128K prefill against its whole 131072-key caches (about 1.5 GB on the "
+                         "device), one whole-path call per step; decode = the B=64 x 32768 decode "
+                         "alone. Prints one JSON line with the per-call time")
     ap.add_argument("--next", action="store_true",
                     help="also time dense causal and sliding-window attention beside DSA at 16K")
     ap.add_argument("--shard", default="problems", choices=["problems", "rows"],
@@ -618,10 +623,60 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_case(args, dsa):
+    """One small case per step, for ncu captures of single kernels (see --profile)."""
+    if args.profile == "decode":
+        dres, dwork, nq = time_decode(dsa, max(args.steps, 1), args.warmup)
+        print(json.dumps({"profile": "decode", "ms": dres, "queries": nq,
+                          "mla_bytes": dwork["mla_bytes"], "idx_bytes": dwork["idx_bytes"]}))
+        return
+    cfg = W.CONFIGS[PREFILL_CFG]
+    L = args.L or cfg.L
+    chunk = cfg.chunk or 4096
+    inp = W.make_prefill(cfg, device="cuda", L=L, rows=(L - chunk, L))
+    torch.cuda.empty_cache()
+    T, S, H, k = inp["T"], inp["S"], inp["H"], inp["k"]
+    fused = args.path == "fused"
+    size = dsa.forward_fused_workspace_size if fused else dsa.forward_workspace_size
+    run = dsa.forward_fused if fused else dsa.forward
+    ws = torch.empty(size(T, S, inp["Hi"], H, k, chunk), dtype=torch.uint8, device="cuda")
+    out = torch.empty(T, H, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(T, H, dtype=torch.float32, device="cuda")
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+
+    def step():
+        run(inp["q8"], inp["q_scale"], inp["k8"], inp["k_scale"], inp["w"], inp["q"], inp["kv"], k,
+            inp["scale"], inp["sm_scale"], q_pos0=inp["q_pos0"], chunk=chunk, idx=idx, out=out,
+            lse=lse, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    e0, e1 = _ev(), _ev()
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    e1.synchronize()
+    st = dsa.get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the profile case: {dsa.STATUS.get(st, st)}")
+    line = {"profile": "chunk", "path": args.path, "rows": [L - chunk, L], "keys": S,
+            "ms_per_call": e0.elapsed_time(e1) / max(args.steps, 1),
+            "device_bytes": torch.cuda.memory_allocated()}
+    if fused:
+        line["fallback_rows"] = dsa.forward_fused_fallback_rows(ws, T, S, k, chunk)
+    print(json.dumps(line))
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.profile:
+        import sparse_attention_long_02_b200 as dsa
+        torch.cuda.set_device(0)
+        run_profile_case(args, dsa)
         return
     ranks = Ranks(args.gpus)
     import sparse_attention_long_02_b200 as dsa

@@ -403,10 +403,15 @@ long long sample_count(int S) {
   return (p >> 12) * 256 + std::min<long long>(p & 4095, 255) + 1;
 }
 
-// Workspace of the fused path, each part 256-byte aligned.
+// Workspace of the fused path, each part 256-byte aligned. The candidate
+// lists and failure lists are double-buffered by chunk parity, so the
+// selection of one chunk (side stream) overlaps the indexer passes of the
+// next (caller's stream).
 struct FusedLayout {
   long long M, ldm, ld;
-  size_t k8s, kss, sample, tau, cnt, ckey, cidx, fail, fail_total, scratch, idx, total;
+  size_t k8s, kss, sample, tau, cnt[2], ckey[2], cidx[2], fail[2], fail_total, scratch, idx,
+      total;
+  int nbuf;
 };
 
 FusedLayout fused_layout(int T, int S, int k, int chunk) {
@@ -425,10 +430,21 @@ FusedLayout fused_layout(int T, int S, int k, int chunk) {
   L.kss = take(static_cast<size_t>(L.M) * 4);
   L.sample = take(rows * L.ldm * 4);
   L.tau = take(rows * 4);
-  L.cnt = take(rows * 4);
-  L.ckey = take(rows * kFusedCandCap * 4);
-  L.cidx = take(rows * kFusedCandCap * 4);
-  L.fail = take(4 + rows * 4);
+  L.nbuf = rows < static_cast<size_t>(T) ? 2 : 1;
+  for (int b = 0; b < 2; ++b) {
+    const int u = b < L.nbuf ? b : 0;     // one chunk: both parities share a buffer
+    if (u != b) {
+      L.cnt[b] = L.cnt[0];
+      L.ckey[b] = L.ckey[0];
+      L.cidx[b] = L.cidx[0];
+      L.fail[b] = L.fail[0];
+      continue;
+    }
+    L.cnt[b] = take(rows * 4);
+    L.ckey[b] = take(rows * kFusedCandCap * 4);
+    L.cidx[b] = take(rows * kFusedCandCap * 4);
+    L.fail[b] = take(4 + rows * 4);
+  }
   L.fail_total = take(4);
   L.scratch = take(static_cast<size_t>(kFusedSlots) * L.ld * 4);
   L.idx = take(static_cast<size_t>(T) * k * 4);
@@ -577,13 +593,26 @@ int dsa_forward_fused(const void* q8, const float* q_scale, const void* k8, cons
                         cudaMemcpyDeviceToDevice, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.fail_total, 0, 4, st);
   if (e != cudaSuccess) return status_of(e);
-  for (int c0 = 0; c0 < T; c0 += rows) {
+  // Per chunk c (buffers of parity b = c & 1): on the caller's stream the
+  // sample pass, the thresholds and the filter pass; on the side stream the
+  // select and recompute kernels, beside the next chunk's passes. The filter
+  // pass of chunk c+2 rewrites buffers b, so it first waits for chunk c's
+  // selection; the attention waits for every selection.
+  std::unique_lock<std::mutex> lock(g_overlap_mu);
+  Overlap* ov = L.nbuf == 2 ? overlap_for_current_device() : nullptr;
+  if (!ov) lock.unlock();
+  cudaStream_t side = ov ? ov->side : st;
+  if (ov && ((e = cudaEventRecord(ov->start, st)) != cudaSuccess ||
+             (e = cudaStreamWaitEvent(ov->side, ov->start, 0)) != cudaSuccess))
+    return status_of(e);
+  int c = 0;
+  for (int c0 = 0; c0 < T; c0 += rows, ++c) {
+    const int b = c & 1;
     const int n = std::min(rows, T - c0);
     const uint8_t* q8c = static_cast<const uint8_t*>(q8) + static_cast<size_t>(c0) * Hi * 128;
     const float* qsc = q_scale ? q_scale + c0 : nullptr;
     const float* wc = w + static_cast<size_t>(c0) * Hi;
-    // 1. each row's scores against the sampled keys
-    // the sampled keys the chunk's last row sees
+    // 1. each row's scores against the sampled keys the chunk's last row sees
     const long long m_c =
         sample_count(static_cast<int>(std::min<long long>(static_cast<long long>(q_pos0) + c0 + n,
                                                           S)));
@@ -611,12 +640,12 @@ int dsa_forward_fused(const void* q8, const float* q_scale, const void* k8, cons
     F.sample = a.scores;
     F.ld_sample = L.ldm;
     F.tau = reinterpret_cast<unsigned*>(ws + L.tau);
-    F.cand_count = reinterpret_cast<unsigned*>(ws + L.cnt);
-    F.cand_key = reinterpret_cast<unsigned*>(ws + L.ckey);
-    F.cand_idx = reinterpret_cast<int*>(ws + L.cidx);
+    F.cand_count = reinterpret_cast<unsigned*>(ws + L.cnt[b]);
+    F.cand_key = reinterpret_cast<unsigned*>(ws + L.ckey[b]);
+    F.cand_idx = reinterpret_cast<int*>(ws + L.cidx[b]);
     F.cand_cap = kFusedCandCap;
-    F.fail_count = reinterpret_cast<unsigned*>(ws + L.fail);
-    F.fail_rows = reinterpret_cast<int*>(ws + L.fail) + 1;
+    F.fail_count = reinterpret_cast<unsigned*>(ws + L.fail[b]);
+    F.fail_rows = reinterpret_cast<int*>(ws + L.fail[b]) + 1;
     F.fail_total = reinterpret_cast<unsigned*>(ws + L.fail_total);
     F.q8 = q8c;
     F.q_scale = qsc;
@@ -629,24 +658,36 @@ int dsa_forward_fused(const void* q8, const float* q_scale, const void* k8, cons
     F.idx = idx + static_cast<size_t>(c0) * k;
     F.err = err;
     if (e == cudaSuccess) e = launch_fused_tau(F, st);
-    // 3. the filter-mode indexer: candidate lists instead of scores
-    if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.cnt, 0, static_cast<size_t>(n) * 4, st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.fail, 0, 4, st);
-    IndexerArgs b = a;
-    b.S = S;
-    b.k_scale = k_scale;
-    b.scores = nullptr;
-    b.ld = 0;
-    b.tau = F.tau;
-    b.cand_count = reinterpret_cast<unsigned*>(ws + L.cnt);
-    b.cand_key = reinterpret_cast<unsigned*>(ws + L.ckey);
-    b.cand_idx = reinterpret_cast<int*>(ws + L.cidx);
-    b.cand_cap = kFusedCandCap;
-    if (e == cudaSuccess) e = launch_indexer(b, q8c, k8b, S, st);
+    // 3. the filter-mode indexer: candidate lists instead of scores, into
+    // buffers b once chunk c-2's selection has read them
+    if (e == cudaSuccess && ov && c >= 2) e = cudaStreamWaitEvent(st, ov->topk_done[b], 0);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.cnt[b], 0, static_cast<size_t>(n) * 4, st);
+    IndexerArgs fa = a;
+    fa.S = S;
+    fa.k_scale = k_scale;
+    fa.scores = nullptr;
+    fa.ld = 0;
+    fa.tau = F.tau;
+    fa.cand_count = reinterpret_cast<unsigned*>(ws + L.cnt[b]);
+    fa.cand_key = reinterpret_cast<unsigned*>(ws + L.ckey[b]);
+    fa.cand_idx = reinterpret_cast<int*>(ws + L.cidx[b]);
+    fa.cand_cap = kFusedCandCap;
+    if (e == cudaSuccess) e = launch_indexer(fa, q8c, k8b, S, st);
     // 4. the exact selection among the candidates; 5. the rest recomputed
-    if (e == cudaSuccess) e = launch_fused_select(F, st);
-    if (e == cudaSuccess) e = launch_fused_fallback(F, st);
+    if (e == cudaSuccess && ov) {
+      e = cudaEventRecord(ov->idx_done[b], st);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ov->idx_done[b], 0);
+    }
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.fail[b], 0, 4, side);
+    if (e == cudaSuccess) e = launch_fused_select(F, side);
+    if (e == cudaSuccess) e = launch_fused_fallback(F, side);
+    if (e == cudaSuccess && ov) e = cudaEventRecord(ov->topk_done[b], side);
     if (e != cudaSuccess) return status_of(e);
+  }
+  if (ov) {
+    for (int b = 0; b < std::min(c, 2); ++b)
+      if ((e = cudaStreamWaitEvent(st, ov->topk_done[b], 0)) != cudaSuccess) return status_of(e);
+    lock.unlock();
   }
   return dsa_sparse_mla_fwd(q, kv, idx, T, S, H, k, sm_scale, out, lse, stream);
 }

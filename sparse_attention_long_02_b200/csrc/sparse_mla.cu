@@ -21,7 +21,8 @@
 //      table for the paged cache), the whole rows of the CTA's own 32 slots
 //      and the CTA's 256 value dims of the peer's 32 slots, up to three tiles
 //      ahead;
-//   2. warp 1 issues S = Q K_own^T (M=128 heads, N=32 keys, K=576) into TMEM;
+//   2. warp 1 issues S = Q K_own^T (M=128 heads, N=32 keys, K=576) into TMEM,
+//      one tile ahead of the PV product;
 //   3. eight softmax warps (thread = head, two warps per TMEM lane quarter,
 //      16 keys each) take the tile maximum of their own keys; the two CTAs
 //      swap their maxima one tile ahead (remote stores), so both use the same
@@ -324,8 +325,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
         mma_commit(smem_u32(&sm.kv_empty[st]));
         return true;
       };
-      // QK runs two tiles ahead of PV: the softmax warps take tile i+1's
-      // maximum while tile i is finished
+      // QK runs one tile ahead of PV: QK(i) needs only the softmax warps'
+      // read of tile i-1's logits, so they take tile i's maximum while the
+      // peer finishes tile i-1; PV(i-1) follows as soon as both P halves of
+      // tile i-1 are in, which frees tile i-1's ring stage a tile earlier
+      // than a deeper lead would
       int next_pv = 0;
       for (int i = 0; ok && i < ntiles; ++i) {
         const int st = i % kStages;
@@ -350,9 +354,9 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
           }
         }
         mma_commit(smem_u32(&sm.s_full));
-        if (i >= 2) {
-          if (!(ok = issue_pv(i - 2))) break;
-          next_pv = i - 1;
+        if (i >= 1) {
+          if (!(ok = issue_pv(i - 1))) break;
+          next_pv = i;
         }
       }
       while (ok && next_pv < ntiles && !*abort_flag && issue_pv(next_pv)) ++next_pv;

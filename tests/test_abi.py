@@ -129,14 +129,20 @@ def test_workspace_sizes(dsa):
         64 * 512 * 64 * 4 + 64 * 2048 * 4
     assert L.dsa_forward_workspace_size(0, 8, 4, 8, 4, 0) == 0
     # fused prefill: the sampled keys (the first 256 of every 4096) and their
-    # scales, per chunk row the sample scores, threshold, count and 4096
-    # candidates, the failure list, the call's failure total, 148 scratch score rows, and idx
+    # scales, per chunk row the sample scores and threshold, then twice (by
+    # chunk parity) the count, 4096 candidates and the failure list; the call's
+    # failure total, 148 scratch score rows, and idx
     r256 = lambda x: (x + 255) // 256 * 256
     T, S, k, rows = 131072, 131072, 2048, 4096
     M = 32 * 256
-    parts = [M * 128, M * 4, rows * M * 4, rows * 4, rows * 4, rows * 4096 * 4, rows * 4096 * 4,
-             4 + rows * 4, 4, 148 * S * 4, T * k * 4]
+    per_parity = [rows * 4, rows * 4096 * 4, rows * 4096 * 4, 4 + rows * 4]
+    parts = [M * 128, M * 4, rows * M * 4, rows * 4] + 2 * per_parity + \
+        [4, 148 * S * 4, T * k * 4]
     assert L.dsa_forward_fused_workspace_size(T, S, 64, 128, k, rows) == sum(r256(x) for x in parts)
+    # one chunk: a single set of candidate buffers
+    parts1 = [M * 128, M * 4, T * M * 4, T * 4] + [T * 4, T * 4096 * 4, T * 4096 * 4,
+                                                    4 + T * 4] + [4, 148 * S * 4, T * k * 4]
+    assert L.dsa_forward_fused_workspace_size(T, S, 64, 128, k, 0) == sum(r256(x) for x in parts1)
     assert L.dsa_forward_fused_workspace_size(T, S, 64, 128, 4096, rows) == 0
     # warm-up target: T * H rows of fp32 logits, S rounded up to 4
     assert L.dsa_attention_probs_workspace_size(2048, 2048, 128) == 2048 * 128 * 2048 * 4

@@ -102,7 +102,7 @@ def _normal(shape, g, device, dtype=torch.float32):
     return torch.randn(*shape, generator=g, device=device, dtype=torch.float32).to(dtype)
 
 
-def _plant(q: torch.Tensor, k: torch.Tensor, cfg: Config, g, device):
+def _plant(q: torch.Tensor, k: torch.Tensor, cfg: Config, g, device, t0q: int = 0, L: int = 0):
     """Correlate each block of queries with a few keys along a random direction.
 
     For block b (``plant_block`` queries), draw a unit vector u_b in R^128 and
@@ -110,22 +110,26 @@ def _plant(q: torch.Tensor, k: torch.Tensor, cfg: Config, g, device):
     prefix [0, block_start), the first block using [0, block_end)). Add a*u_b
     to every head of every query in the block and to each planted key, with
     a^2 = 3*sqrt(128), so a planted pair's dot product gains +3 sigma.
+    ``q`` may hold only the query rows [t0q, t0q + len(q)) of an L-token
+    prefill (L = 0: all rows); every block's keys are planted all the same.
     """
-    T = q.shape[0]
+    L = L or q.shape[0]
     a = math.sqrt(3.0 * math.sqrt(D_INDEX))
-    nblk = (T + cfg.plant_block - 1) // cfg.plant_block
+    nblk = (L + cfg.plant_block - 1) // cfg.plant_block
     for b in range(nblk):
         t0 = b * cfg.plant_block
-        t1 = min(T, t0 + cfg.plant_block)
+        t1 = min(L, t0 + cfg.plant_block)
         u = torch.randn(D_INDEX, generator=g, device=device)
         u = u / u.norm()
         hi = t0 if (cfg.plant_prefix and t0 > 0) else t1
         pos = torch.randint(0, hi, (cfg.plant_n,), generator=g, device=device)
-        q[t0:t1] += a * u
+        r0, r1 = max(t0, t0q) - t0q, min(t1, t0q + q.shape[0]) - t0q
+        if r0 < r1:
+            q[r0:r1] += a * u
         k.index_add_(0, pos, (a * u).expand(cfg.plant_n, D_INDEX).contiguous())
 
 
-def make_prefill(cfg: Config, device="cpu", L: int | None = None):
+def make_prefill(cfg: Config, device="cpu", L: int | None = None, rows=None):
     """Inputs for a causal prefill of ``L`` tokens (default: the config's L).
 
     Returns a dict with
@@ -133,11 +137,18 @@ def make_prefill(cfg: Config, device="cpu", L: int | None = None):
       k8 [L][128] uint8 (e4m3), k_scale [L] f32 or None, w [L][Hi] f32,
       q [L][H][576] bf16, kv [L][576] bf16,
       plus scale, sm_scale, k, q_pos0 (=0), T, S.
+    With ``rows`` = (t0, t1), the query-side tensors (q8, q_scale, w, q) hold
+    only the rows t0 .. t1-1 of that prefill (T = t1 - t0, q_pos0 = t0) and
+    the caches all L keys: the same shapes and distributions, drawn in
+    another order than the whole prefill's (so not the same values).
     """
     L = cfg.L if L is None else L
+    t0, t1 = rows if rows is not None else (0, L)
+    T = t1 - t0
     g = _gen(cfg.seed, device)
     Hi, H = cfg.Hi, cfg.H
     if cfg.grid:
+        assert rows is None, "the integer grid is drawn for whole prefills only"
         q8 = torch.randint(-8, 9, (L, Hi, D_INDEX), generator=g, device=device)
         k8 = torch.randint(-8, 9, (L, D_INDEX), generator=g, device=device)
         q8 = q8.float().to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
@@ -145,19 +156,19 @@ def make_prefill(cfg: Config, device="cpu", L: int | None = None):
         w = torch.randint(-4, 5, (L, Hi), generator=g, device=device).float() / 4.0
         q_scale = k_scale = None
     else:
-        qi = _normal((L, Hi, D_INDEX), g, device)
+        qi = _normal((T, Hi, D_INDEX), g, device)
         ki = _normal((L, D_INDEX), g, device)
         if cfg.plant_block:
-            _plant(qi, ki, cfg, g, device)
+            _plant(qi, ki, cfg, g, device, t0q=t0, L=L)
         q8, q_scale = fp8_per_token(qi, 2)
         k8, k_scale = fp8_per_token(ki, 1)
         del qi, ki
-        w = _normal((L, Hi), g, device) / 8.0        # N(0, 1/64)
-    q = _normal((L, H, D_QK), g, device, torch.bfloat16)
+        w = _normal((T, Hi), g, device) / 8.0        # N(0, 1/64)
+    q = _normal((T, H, D_QK), g, device, torch.bfloat16)
     kv = _normal((L, D_QK), g, device, torch.bfloat16)
     return dict(q8=q8, q_scale=q_scale, k8=k8, k_scale=k_scale, w=w.contiguous(),
                 q=q.contiguous(), kv=kv.contiguous(), scale=cfg.scale,
-                sm_scale=cfg.sm_scale, k=cfg.k, q_pos0=0, T=L, S=L,
+                sm_scale=cfg.sm_scale, k=cfg.k, q_pos0=t0, T=T, S=L,
                 Hi=Hi, H=H)
 
 
