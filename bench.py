@@ -368,8 +368,8 @@ def e2e_prefill(pf, steps):
     return ms, h2d, d2h
 
 
-def time_decode(dsa, steps, warmup):
-    cfg = W.CONFIGS[DECODE_CFG]
+def time_decode(dsa, steps, warmup, cfg_id=DECODE_CFG):
+    cfg = W.CONFIGS[cfg_id]
     inp = W.make_decode(cfg, device="cuda")
     g = inp
     B, nq, k = inp["B"], inp["nq"], inp["k"]
@@ -407,53 +407,112 @@ def time_decode(dsa, steps, warmup):
     if st != 0:
         raise RuntimeError(f"device error in decode: {dsa.STATUS.get(st, st)}")
     work = decode_work(inp["seq_len"].cpu().tolist(), nq, inp["Hi"], inp["H"], k)
-    return res, work, B * nq
+    return res, work, B * nq, inp
 
 
-def time_next(dsa, steps=3, warmup=2):
-    """Dense causal and sliding-window attention on the same sparse MLA
-    kernel (index sets from dsa_window_indices) beside the whole DSA path,
-    on the 16K prefill workload."""
-    cfg = W.CONFIGS[2]
-    inp = W.make_prefill(cfg, device="cuda")
-    L, H, k, sm = inp["T"], inp["H"], inp["k"], inp["sm_scale"]
-    q, kv = inp["q"], inp["kv"]
-    out = torch.empty(L, H, 512, dtype=torch.bfloat16, device="cuda")
-    lse = torch.empty(L, H, dtype=torch.float32, device="cuda")
-    pf = Prefill(dsa, cfg, inp)
-    swa_idx = dsa.window_indices(L, L, k, k)
-    chunk = 2048        # dense rows in chunks; a chunk's rows see keys up to its last row
-    dense_idx = [dsa.window_indices(chunk, L, c0 + chunk, c0 + chunk, q_pos0=c0)
-                 for c0 in range(0, L, chunk)]
-
-    def swa():
-        dsa.sparse_mla(q, kv, swa_idx, sm, out=out, lse=lse)
-
-    def dense():
-        for c, c0 in enumerate(range(0, L, chunk)):
-            dsa.sparse_mla(q[c0:c0 + chunk], kv, dense_idx[c], sm, out=out[c0:c0 + chunk],
-                           lse=lse[c0:c0 + chunk])
-
-    res = {"workload": f"prefill L={L} (config 2), MLA {H} heads over the 512+64 latent; "
-                       f"dsa = indexer + top-{k} + sparse MLA; swa = window {k}; "
-                       f"dense_causal = every causal key, rows in chunks of {chunk} "
-                       f"(1/9 of the slots are masked, past the diagonal)"}
-    for name, fn in (("dsa", pf.step), ("swa", swa), ("dense_causal", dense)):
-        for _ in range(warmup):
-            fn()
+def _time(fn, steps, warmup, flush=None):
+    """Median device time of fn (ms) over `steps` calls after `warmup`, an
+    optional L2 flush before each (outside the events)."""
+    for _ in range(warmup):
+        fn()
+    times = []
+    for _ in range(steps):
+        if flush is not None:
+            flush.zero_()
         e0, e1 = _ev(), _ev()
         e0.record()
-        for _ in range(steps):
-            fn()
+        fn()
         e1.record()
         e1.synchronize()
-        ms = e0.elapsed_time(e1) / steps
-        res[name] = {"ms": ms, "tokens_per_s": L / (ms * 1e-3)}
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def time_next(dsa, pf, path="scores"):
+    """DSA beside dense causal attention (the same MLA kernel with every causal
+    key, slots generated in the kernel) over the context length, for prefill
+    (prefixes of the 128K prefill's inputs: the first L rows against the first
+    L keys are an L-token causal prefill) and for decode (B = 64 sequences of
+    one context length, paged). Also sliding-window attention at 16K, the
+    projection and the warm-up objective."""
+    i = pf.inp
+    H, k, sm = i["H"], i["k"], i["sm_scale"]
+    res = {"workload": "prefill: the first L rows of the L=131072 prefill (4096-row chunks, k=2048, "
+                       "indexer 64x128 FP8, MLA 128 heads); dsa = " +
+                       ("dsa_forward_fused" if path == "fused" else "dsa_forward") +
+                       ", dense = dsa_dense_causal_mla (every causal key); decode: B=64 sequences "
+                       "of the given context, nq=1, paged, L2 flushed before each call"}
+    prefill = []
+    for L in (4096, 16384, 65536, 131072):
+        chunk = min(4096, L)
+        size = dsa.forward_fused_workspace_size if path == "fused" else dsa.forward_workspace_size
+        run = dsa.forward_fused if path == "fused" else dsa.forward
+        ws = torch.empty(size(L, L, i["Hi"], H, k, chunk), dtype=torch.uint8, device="cuda")
+        out = torch.empty(L, H, 512, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(L, H, dtype=torch.float32, device="cuda")
+        cut = lambda x: None if x is None else x[:L]
+
+        def dsa_call():
+            run(i["q8"][:L], cut(i["q_scale"]), i["k8"][:L], cut(i["k_scale"]), i["w"][:L],
+                i["q"][:L], i["kv"][:L], k, i["scale"], sm, chunk=chunk, out=out, lse=lse,
+                workspace=ws, return_idx=False)
+
+        def dense_call():
+            dsa.dense_causal_mla(i["q"][:L], i["kv"][:L], sm, out=out, lse=lse)
+
+        reps = 1 if L > 65536 else 2
+        t_dsa = _time(dsa_call, reps, 1)
+        t_dense = _time(dense_call, reps, 1)
+        prefill.append({"L": L, "dsa_ms": t_dsa, "dense_ms": t_dense,
+                        "dsa_tokens_per_s": L / (t_dsa * 1e-3),
+                        "dense_tokens_per_s": L / (t_dense * 1e-3), "speedup": t_dense / t_dsa})
+        del ws, out, lse
+        torch.cuda.empty_cache()
+    res["prefill"] = prefill
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    decode = []
+    for ctx in (4096, 16384, 32768, 65536, 131072):
+        cfg = W.Config(94, "decode_curve", "decode", k=2048, Hi=64, H=128, seed=7, B=64, ctx=ctx)
+        d = W.make_decode(cfg, device="cuda")
+        B, nq = d["B"], d["nq"]
+        ws = torch.empty(dsa.decode_workspace_size(B, nq, d["max_blocks"], d["Hi"], d["H"], 2048),
+                         dtype=torch.uint8, device="cuda")
+        out = torch.empty(B, nq, d["H"], 512, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(B, nq, d["H"], dtype=torch.float32, device="cuda")
+
+        def dsa_dec():
+            dsa.decode_paged(d["q8"], d["q_scale"], d["w"], d["q"], d["k8_pool"], d["k_scale_pool"],
+                             d["kv_pool"], d["block_table"], d["seq_len"], 2048, d["scale"],
+                             d["sm_scale"], out=out, lse=lse, workspace=ws)
+
+        def dense_dec():
+            dsa.dense_causal_mla_decode_paged(d["q"], d["kv_pool"], d["block_table"], d["seq_len"],
+                                              d["sm_scale"], out=out, lse=lse)
+
+        t_dsa = _time(dsa_dec, 5, 2, flush)
+        t_dense = _time(dense_dec, 5, 2, flush)
+        decode.append({"ctx": ctx, "dsa_ms": t_dsa, "dense_ms": t_dense,
+                       "dsa_queries_per_s": B * nq / (t_dsa * 1e-3),
+                       "dense_queries_per_s": B * nq / (t_dense * 1e-3),
+                       "speedup": t_dense / t_dsa})
+        del d, ws, out, lse
+        torch.cuda.empty_cache()
+    res["decode"] = decode
     st = dsa.get_device_error()
     if st != 0:
-        raise RuntimeError(f"device error in the window runs: {dsa.STATUS.get(st, st)}")
-    res["projection"] = time_projection(dsa, steps, warmup)
-    res["warmup_objective"] = time_warmup(dsa, steps, warmup)
+        raise RuntimeError(f"device error in the DSA-vs-dense runs: {dsa.STATUS.get(st, st)}")
+    # sliding-window attention (window k) at 16K, on the same MLA kernel
+    L = 16384
+    swa_idx = dsa.window_indices(L, L, k, k)
+    out = torch.empty(L, H, 512, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(L, H, dtype=torch.float32, device="cuda")
+    t_swa = _time(lambda: dsa.sparse_mla(i["q"][:L], i["kv"][:L], swa_idx, sm, out=out, lse=lse),
+                  3, 2)
+    res["swa_16k"] = {"window": k, "ms": t_swa, "tokens_per_s": L / (t_swa * 1e-3)}
+    del swa_idx, out, lse
+    torch.cuda.empty_cache()
+    res["projection"] = time_projection(dsa, 3, 2)
+    res["warmup_objective"] = time_warmup(dsa, 3, 2)
     return res
 
 
@@ -577,6 +636,34 @@ def oracle_sample(inp, n_rows=32, threads=None):
                 host_cpus=os.cpu_count())
 
 
+def oracle_decode_sample(inp, n_seqs=8, threads=None):
+    """Time the CPU oracle's paged decode on a sample of the batch's sequences,
+    stratified by context length (every n-th by length, so queries/s on the
+    sample estimates the whole batch's); rows run in parallel on host threads."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    threads = threads or os.cpu_count() or 1
+    lens = inp["seq_len"].cpu().numpy()
+    order = np.argsort(lens, kind="stable")
+    B, nq = len(lens), inp["nq"]
+    seqs = sorted({int(order[min(B - 1, int((i + 0.5) * B / n_seqs))]) for i in range(n_seqs)})
+    as_np = {"q8": np.uint8, "q_scale": np.float32, "w": np.float32, "q": np.uint16,
+             "k8_pool": np.uint8, "k_scale_pool": np.float32, "kv_pool": np.uint16,
+             "block_table": np.int32, "seq_len": np.int32}
+    host = dict(inp)
+    for name, dt in as_np.items():                  # one host copy, shared by the threads
+        host[name] = oracle._np(inp[name], dt)
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(lambda b: oracle.decode(host, seqs=[b]), seqs))
+    wall = time.perf_counter() - t0
+    ctx = [int(lens[b]) for b in seqs]
+    return dict(value=len(seqs) * nq / wall, unit="queries/s", cores=threads, kind="oracle",
+                sample=f"{len(seqs)} of the {B} sequences (every {B // len(seqs)}-th by context "
+                       f"length: {min(ctx)}..{max(ctx)} tokens), {nq} queries each, whole path per "
+                       f"query, {threads} threads; {wall:.1f} s wall", wall_s=wall)
+
+
 def cpu_model():
     """The host CPU's model name, from /proc/cpuinfo (None where it is absent)."""
     try:
@@ -626,7 +713,7 @@ def run_reference(args):
 def run_profile_case(args, dsa):
     """One small case per step, for ncu captures of single kernels (see --profile)."""
     if args.profile == "decode":
-        dres, dwork, nq = time_decode(dsa, max(args.steps, 1), args.warmup)
+        dres, dwork, nq, _ = time_decode(dsa, max(args.steps, 1), args.warmup)
         print(json.dumps({"profile": "decode", "ms": dres, "queries": nq,
                           "mla_bytes": dwork["mla_bytes"], "idx_bytes": dwork["idx_bytes"]}))
         return
@@ -742,7 +829,7 @@ def main():
             "roofline": roof, "stages": stages,
             "end_to_end_roofline": {"ms": 1e3 * t_roof, "frac": 1e3 * t_roof / ms}}
     if not args.no_decode:
-        dres, dwork, nqueries = time_decode(dsa, max(args.steps, 10), args.warmup)
+        dres, dwork, nqueries, dinp = time_decode(dsa, max(args.steps, 10), args.warmup)
         mla_gbs = dwork["mla_bytes"] / (dres["sparse_mla"] * 1e-3) / 1e9
         line["decode"] = {
             "workload": "B=64 x 32768, nq=1, paged (block 64), k=2048, 64x128 FP8 indexer, "
@@ -765,14 +852,31 @@ def main():
             "note": "indexer + top-k timed together, against the indexer's algorithmic bytes"}
         line["decode"]["end_to_end_roofline"] = {"ms": 1e3 * (t_idx + t_mla),
                                                  "frac": 1e3 * (t_idx + t_mla) / dres["total"]}
+        vres, vwork, vq, vinp = time_decode(dsa, max(args.steps, 10), args.warmup, cfg_id=5)
+        vgbs = vwork["mla_bytes"] / (vres["sparse_mla"] * 1e-3) / 1e9
+        line["decode_varlen"] = {
+            "workload": "B=128, contexts log-uniform in [512, 131072], nq=2 causal, paged, "
+                        "k=2048", "value": vq * ranks.world / (vres["total"] * 1e-3),
+            "unit": "queries/s", "ms": vres["total"],
+            "sparse_mla": {"ms": vres["sparse_mla"], "bound": "hbm", "achieved": vgbs,
+                           "peak": pk["hbm"], "unit": "GB/s", "frac": vgbs / pk["hbm"]}}
     if args.next:
-        line["next"] = time_next(dsa)
+        line["next"] = time_next(dsa, pf, args.path)
     if not args.no_e2e and not rows_mode:       # e2e: the default mode's whole prefill per GPU
         e_ms, h2d, d2h = e2e_prefill(pf, max(1, min(args.steps, 3)))
         line["e2e"] = {"value": tokens / (ranks.max(e_ms) / 1e3), "unit": "tokens/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     if ranks.rank == 0 and ranks.world == 1 and not args.no_cpu:
-        line["cpu_baseline"] = oracle_sample(inp)
+        cb = oracle_sample(inp)
+        one = oracle_sample(inp, n_rows=8, threads=1)
+        cb["single_thread"] = {k: one[k] for k in ("value", "unit", "cores", "sample", "wall_s")}
+        if not args.no_decode:
+            cb["decode"] = oracle_decode_sample(dinp)
+            cb["decode"]["workload"] = "decode B=64 x 32768, nq=1 (the GPU decode line's)"
+            vcb = oracle_decode_sample(vinp)
+            vcb["workload"] = "decode B=128, contexts log-uniform in [512, 131072], nq=2"
+            cb["decode_varlen"] = vcb
+        line["cpu_baseline"] = cb
     ranks.close()
     if ranks.rank == 0:
         print(json.dumps(line), flush=True)

@@ -260,6 +260,30 @@ int dsa_window_indices(int T, int S, int q_pos0, int window, int k, int32_t *idx
                        dsa_stream_t stream);
 
 /*
+ * Dense causal MLA, the full interface page 2 keeps beside DSA ("六、实测表现与
+ * 取舍"): the same kernel as dsa_sparse_mla_fwd with every causal key selected,
+ * the slots generated in the kernel (no index sets in memory). It is the
+ * baseline DSA is measured against: attention whose cost grows with the whole
+ * context, where DSA's grows with k (page 1, section "秘密武器").
+ *
+ * dsa_dense_causal_mla: query row t (position q_pos0 + t) attends to keys
+ *   0 .. min(q_pos0 + t, S - 1) of kv [S][576]; q, out, lse as for
+ *   dsa_sparse_mla_fwd.
+ * dsa_dense_causal_mla_decode_paged: query j of sequence b attends to its
+ *   sequence's keys 0 .. seq_len[b] - nq + j through the block table;
+ *   arguments as for dsa_sparse_mla_decode_paged without idx and k.
+ * Both return DSA_ERR_INVALID_ARG (nothing launched) for bad arguments and
+ * DSA_ERR_UNSUPPORTED for H outside 1 .. 128.
+ */
+int dsa_dense_causal_mla(const void *q, const void *kv, int T, int S, int H, int q_pos0,
+                         float sm_scale, void *out, float *lse, dsa_stream_t stream);
+int dsa_dense_causal_mla_decode_paged(const void *q, const void *kv_pool,
+                                      const int32_t *block_table, const int32_t *seq_len,
+                                      int B, int nq, int max_blocks, int nblk, int H,
+                                      float sm_scale, void *out, float *lse,
+                                      dsa_stream_t stream);
+
+/*
  * Whole prefill path: indexer -> top-k -> sparse MLA, the chain of steps 2
  * to 4 of the four-step workflow ("DeepSeek-V3.2-Exp 模型优势与 DSA 工作原理",
  * section 4: scores, top-k selection, attention over the selected positions

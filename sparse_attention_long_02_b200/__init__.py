@@ -65,6 +65,8 @@ _sig("dsa_decode_paged_noalloc", I32, P, P, P, P, P, P, P, P, P, I32, I32, I32, 
      I32, F32, F32, P, P, P, P)
 _sig("dsa_plan_prefill_chunks", I32, I32, I32, I32, I32, I32, I32, I32, I32, I32, P, I32)
 _sig("dsa_plan_decode_sequences", I32, P, I32, I32, I32, I32, I32, I32, I32, P, I32)
+_sig("dsa_dense_causal_mla", I32, P, P, I32, I32, I32, I32, F32, P, P, P)
+_sig("dsa_dense_causal_mla_decode_paged", I32, P, P, P, P, I32, I32, I32, I32, I32, F32, P, P, P)
 _sig("dsa_sparse_mla_decode_paged", I32, P, P, P, P, P, I32, I32, I32, I32, I32, I32, F32, P,
      P, P)
 
@@ -401,6 +403,37 @@ def sparse_mla_decode_paged(q, kv_pool, block_table, seq_len, idx, sm_scale, out
                                             kv_pool.shape[0], H, k, float(sm_scale), _p(out),
                                             _p(lse), _stream(stream)),
            "dsa_sparse_mla_decode_paged")
+    return out, lse
+
+
+def dense_causal_mla(q, kv, sm_scale, q_pos0=0, out=None, lse=None, stream=None):
+    """Dense causal MLA: row t attends to every key 0 .. min(q_pos0 + t, S - 1) -> (out, lse)."""
+    q, kv = _dev(q, torch.bfloat16), _dev(kv, torch.bfloat16)
+    T, H, S = q.shape[0], q.shape[1], kv.shape[0]
+    if out is None:
+        out = torch.empty(T, H, 512, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(T, H, dtype=torch.float32, device=q.device)
+    _check(_lib.dsa_dense_causal_mla(_p(q), _p(kv), T, S, H, q_pos0, float(sm_scale), _p(out),
+                                     _p(lse), _stream(stream)), "dsa_dense_causal_mla")
+    return out, lse
+
+
+def dense_causal_mla_decode_paged(q, kv_pool, block_table, seq_len, sm_scale, out=None, lse=None,
+                                  stream=None):
+    """Dense causal MLA of a paged decode: every key of each query's causal prefix."""
+    q, kv_pool = _dev(q, torch.bfloat16), _dev(kv_pool, torch.bfloat16)
+    block_table, seq_len = _dev(block_table, torch.int32), _dev(seq_len, torch.int32)
+    B, nq, H = q.shape[0], q.shape[1], q.shape[2]
+    if out is None:
+        out = torch.empty(B, nq, H, 512, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(B, nq, H, dtype=torch.float32, device=q.device)
+    _check(_lib.dsa_dense_causal_mla_decode_paged(_p(q), _p(kv_pool), _p(block_table),
+                                                  _p(seq_len), B, nq, block_table.shape[1],
+                                                  kv_pool.shape[0], H, float(sm_scale), _p(out),
+                                                  _p(lse), _stream(stream)),
+           "dsa_dense_causal_mla_decode_paged")
     return out, lse
 
 

@@ -351,9 +351,10 @@ int dsa_window_indices(int T, int S, int q_pos0, int window, int k, int32_t* idx
 static int mla_common(const void* q, const void* kv, const int32_t* idx, int T, int S, int H, int k,
                       float sm_scale, void* out, float* lse, const int32_t* block_table,
                       const int32_t* seq_len, int max_blocks, int nblk, int nq,
-                      cudaStream_t st) {
-  if (!q || !kv || !idx || !out || T < 0 || S < 0 || k <= 0 || (k & 3) || !(sm_scale > 0.f) ||
-      !aligned16(q) || !aligned16(kv) || !aligned16(idx) || !aligned16(out))
+                      cudaStream_t st, int dense = 0, int q_pos0 = 0) {
+  if (!q || !kv || (!idx && !dense) || !out || T < 0 || S < 0 || k <= 0 || (k & 3) ||
+      !(sm_scale > 0.f) || q_pos0 < 0 || !aligned16(q) || !aligned16(kv) || !aligned16(idx) ||
+      !aligned16(out))
     return DSA_ERR_INVALID_ARG;
   if (H < 1 || H > 128) return DSA_ERR_UNSUPPORTED;
   if (T == 0) return DSA_OK;
@@ -364,6 +365,8 @@ static int mla_common(const void* q, const void* kv, const int32_t* idx, int T, 
   a.k = k;
   a.sm_scale_log2 = sm_scale * 1.4426950408889634f;
   a.idx = idx;
+  a.dense = dense;
+  a.q_pos0 = q_pos0;
   a.block_table = block_table;
   a.seq_len = seq_len;
   a.max_blocks = max_blocks;
@@ -383,6 +386,24 @@ int dsa_sparse_mla_fwd(const void* q, const void* kv, const int32_t* idx, int T,
   if (S <= 0 && T > 0) return DSA_ERR_INVALID_ARG;
   return mla_common(q, kv, idx, T, S, H, k, sm_scale, out, lse, nullptr, nullptr, 0, 0, 1,
                     static_cast<cudaStream_t>(stream));
+}
+
+int dsa_dense_causal_mla(const void* q, const void* kv, int T, int S, int H, int q_pos0,
+                         float sm_scale, void* out, float* lse, dsa_stream_t stream) {
+  if (S <= 0 && T > 0) return DSA_ERR_INVALID_ARG;
+  return mla_common(q, kv, nullptr, T, S, H, 4, sm_scale, out, lse, nullptr, nullptr, 0, 0, 1,
+                    static_cast<cudaStream_t>(stream), 1, q_pos0);
+}
+
+int dsa_dense_causal_mla_decode_paged(const void* q, const void* kv_pool,
+                                      const int32_t* block_table, const int32_t* seq_len, int B,
+                                      int nq, int max_blocks, int nblk, int H, float sm_scale,
+                                      void* out, float* lse, dsa_stream_t stream) {
+  if (!block_table || !seq_len || B < 0 || nq < 1 || max_blocks < 1 || nblk < 1)
+    return DSA_ERR_INVALID_ARG;
+  return mla_common(q, kv_pool, nullptr, B * nq, max_blocks * 64, H, 4, sm_scale, out, lse,
+                    block_table, seq_len, max_blocks, nblk, nq, static_cast<cudaStream_t>(stream),
+                    1, 0);
 }
 
 int dsa_sparse_mla_decode_paged(const void* q, const void* kv_pool, const int32_t* block_table,

@@ -113,7 +113,10 @@ struct IndexerBwdArgs {
 struct MlaArgs {
   int T = 0, S = 0, H = 0, k = 0;         // query rows, keys (contiguous), heads, slots per row
   float sm_scale_log2 = 0.f;              // sm_scale * log2(e)
-  const int* idx = nullptr;               // [T][k]
+  const int* idx = nullptr;               // [T][k] (unused in dense mode)
+  // dense causal mode: row r's slots are every key it sees, 0 .. its position
+  // (q_pos0 + r, or the paged query's position); no index sets are read
+  int dense = 0, q_pos0 = 0;
   const int* block_table = nullptr;       // paged cache (decode) or null
   int max_blocks = 0, nblk = 0, nq = 1;
   const int* seq_len = nullptr;

@@ -131,13 +131,17 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
   const uint32_t rank = cluster_rank();
   const uint32_t peer = rank ^ 1u;
   const int c = static_cast<int>(rank);
-  const int r = blockIdx.x >> 1;                 // query row (one cluster per row)
+  // query row (one cluster per row); dense prefill rows run longest first
+  const int r = (A.dense && !A.block_table) ? A.T - 1 - static_cast<int>(blockIdx.x >> 1)
+                                            : static_cast<int>(blockIdx.x >> 1);
   const int seq = A.block_table ? r / A.nq : 0;
   // keys a slot may name: the causal prefix of the query (paged) or the cache
   int limit = A.S;
   if (A.block_table) limit = A.seq_len[seq] - A.nq + (r % A.nq) + 1;
-  const int ntiles = (A.k + kTileKeys - 1) / kTileKeys;
-  const int* sel = A.idx + static_cast<long long>(r) * A.k;
+  // slots of this row: the index set, or in dense mode every key it sees
+  const int nslots = !A.dense ? A.k : A.block_table ? limit : min(A.q_pos0 + r + 1, A.S);
+  const int ntiles = (nslots + kTileKeys - 1) / kTileKeys;
+  const int* sel = A.dense ? nullptr : A.idx + static_cast<long long>(r) * A.k;
   const int warp = warp_id(), lane = lane_id();
   const int dim0 = 256 * c;                      // first value dim of this CTA
   // Both CTAs of the pair normally take the same early exit; if they did not,
@@ -197,7 +201,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
     // Two-deep prefetch: the slots of tile i+2 and the block-table entries
     // of tile i+1 are loading while tile i is issued. Lane l holds own slot
     // l and peer slot l of a tile.
-    auto slot = [&](int j) { return j < A.k ? __ldg(sel + j) : -1; };
+    auto slot = [&](int j) { return j >= nslots ? -1 : A.dense ? j : __ldg(sel + j); };
     const int own0 = kOwnKeys * c + lane, peer0 = kOwnKeys * (c ^ 1) + lane;
     int vo = slot(own0), vp = slot(peer0);                                  // tile 0
     int bo = kv_block(A, vo, seq, limit), bp = kv_block(A, vp, seq, limit);

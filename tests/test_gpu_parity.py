@@ -451,6 +451,43 @@ def test_sliding_window_and_dense_causal_mla(dsa, window, k):
     assert_mla_close(out[rows], ref, lse[rows], ref_lse, lse_atol(q[rows], kv, 1 / 24, ref_lse, k))
 
 
+@pytest.mark.parametrize("T,S,q_pos0,H", [(300, 300, 0, 128), (100, 400, 300, 8), (70, 650, 580, 16)])
+def test_dense_causal_mla_range_mode(dsa, T, S, q_pos0, H):
+    """Dense causal attention with the slots generated in the kernel (no index
+    sets): against the oracle's sparse MLA over every key of each row's causal
+    prefix, on rows spanning several tiles, a ragged last tile and an offset."""
+    rng = np.random.default_rng(T + S + H)
+    q = torch.from_numpy(rng.normal(size=(T, H, 576))).to(torch.bfloat16)
+    kv = torch.from_numpy(rng.normal(size=(S, 576))).to(torch.bfloat16)
+    out, lse = dsa.dense_causal_mla(q.cuda(), kv.cuda(), 1 / 24, q_pos0=q_pos0)
+    no_device_error(dsa)
+    k = (S + 3) // 4 * 4
+    rows = sorted({0, 1, 63, 64, T // 2, T - 1})
+    ref, ref_lse = oracle.sparse_mla(q, kv, oracle.window(T, S, S, k, q_pos0=q_pos0), 1 / 24,
+                                     rows=rows)
+    assert_mla_close(out[rows], ref, lse[rows], ref_lse, lse_atol(q[rows], kv, 1 / 24, ref_lse, k))
+
+
+def test_dense_causal_mla_decode_paged_range_mode(dsa):
+    """The paged decode's dense attention: every key of each query's causal
+    prefix through the block table, against the oracle on the gathered sequence."""
+    inp = _small_decode([100, 2049, 5000, 64], 2, seed=12, H=128)
+    g = cuda(inp)
+    out, lse = dsa.dense_causal_mla_decode_paged(g["q"], g["kv_pool"], g["block_table"],
+                                                 g["seq_len"], inp["sm_scale"])
+    no_device_error(dsa)
+    kvp, table, lens = inp["kv_pool"], inp["block_table"].numpy(), inp["seq_len"].numpy()
+    for b in range(inp["B"]):
+        n = int(lens[b])
+        kv_seq = torch.from_numpy(
+            oracle.gather_sequence(kvp.view(torch.int16).numpy(), table[b], n)).view(torch.bfloat16)
+        k = (n + 3) // 4 * 4
+        idx = oracle.window(2, n, n, k, q_pos0=n - 2)
+        ref, ref_lse = oracle.sparse_mla(inp["q"][b], kv_seq, idx, inp["sm_scale"])
+        assert_mla_close(out[b], ref, lse[b], ref_lse,
+                         lse_atol(inp["q"][b], kv_seq, inp["sm_scale"], ref_lse, k))
+
+
 # ------------------------------------------------ projection (workflow step 1)
 
 @pytest.mark.parametrize("T,d,Hi", [(300, 200, 64), (129, 64, 4), (5, 8, 1)])

@@ -451,6 +451,27 @@ def test_warmup_target_rows_sum_to_one_and_match_softmax_and_attention():
     np.testing.assert_allclose(out[:, 0], p1 @ kv[:, :512].double().numpy(), rtol=1e-9, atol=1e-12)
 
 
+def test_warmup_target_is_the_mean_of_the_per_head_softmax_rows():
+    """The H-head target is the plain mean over heads of each head's own
+    library softmax of its masked logits, with heads of very different
+    sharpness so that any other weighting of the heads (a sum, one head, a
+    softmax of averaged logits, weights by head index) moves the result."""
+    rng = np.random.default_rng(43)
+    T, H = 10, 4
+    gains = torch.tensor([0.2, 1.0, 3.0, 8.0], dtype=torch.float64)
+    qf = torch.from_numpy(rng.normal(size=(T, H, 576))) * gains[None, :, None]
+    q, kv = qf.to(torch.bfloat16), _bf16(rng, (T, 576))
+    p = oracle.attention_probs(q, kv, 1 / 24)
+    mask = torch.ones(T, T, dtype=torch.bool).tril()
+    z = torch.einsum("thd,sd->ths", q.double(), kv.double()) / 24
+    per_head = torch.softmax(z.masked_fill(~mask[:, None, :], -np.inf), dim=-1)
+    np.testing.assert_allclose(p, per_head.mean(dim=1).numpy(), rtol=1e-10, atol=1e-14)
+    # the alternatives a mistake would produce differ from it
+    pooled = torch.softmax(z.mean(dim=1).masked_fill(~mask, -np.inf), dim=-1)
+    assert np.abs(p - pooled.numpy()).max() > 1e-3
+    assert np.abs(p - per_head[:, -1].numpy()).max() > 1e-3
+
+
 def test_warmup_kl_zero_at_the_target_and_gradient_by_finite_differences():
     rng = np.random.default_rng(42)
     R, n = 4, 17
