@@ -21,8 +21,9 @@
 //      table for the paged cache), the whole rows of the CTA's own 32 slots
 //      and the CTA's 256 value dims of the peer's 32 slots, up to three tiles
 //      ahead;
-//   2. warp 1 issues S = Q K_own^T (M=128 heads, N=32 keys, K=576) into TMEM,
-//      one tile ahead of the PV product;
+//   2. warp 1 issues S = Q K_own^T (M=128 heads, N=32 keys, K=576) into TMEM
+//      as soon as the tile is gathered and the previous logits are read,
+//      independently of the PV products;
 //   3. eight softmax warps (thread = head, two warps per TMEM lane quarter,
 //      16 keys each) take the tile maximum of their own keys; the two CTAs
 //      swap their maxima one tile ahead (remote stores), so both use the same
@@ -307,39 +308,8 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
       // wait runs out and both CTAs leave through their give-up paths
       if (ok && (debug_bits(err) & kDbgStallMla))
         ok = mbar_wait(smem_u32(&sm.o_done), 0, abort_flag, err);
-      auto issue_pv = [&](int i) -> bool {
-        const int st = i % kStages, b = i & 1;
-        if (!mbar_wait(smem_u32(&sm.p_own[b]), (i >> 1) & 1, abort_flag, err)) return false;
-        if (!mbar_wait<true>(smem_u32(&sm.p_peer[b]), (i >> 1) & 1, abort_flag, err)) return false;
-        tc_fence_after();
-        // keys of CTA h's slots: P from p[b][h], V from this CTA's own rows
-        // (h == c: their atoms 4c..4c+3) or from the peer rows' value dims
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t vbase =
-              smem_u32(sm.kv[st][h == c ? 4 * c : kOwnAtoms]);
-          const uint64_t vdesc = sdesc_sw128(vbase, kAtom, 1024);
-          const uint64_t pdesc = sdesc_sw64(smem_u32(sm.p[b][h]), 512);
-#pragma unroll
-          for (int kk = 0; kk < kOwnKeys / 16; ++kk)          // 16 keys: 32 B of P, 2 KB of V
-            mma_bf16(tmem + kColO, pdesc + 2 * kk, vdesc + (kk * 2048 >> 4), id_pv,
-                     (i > 0 || h > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(smem_u32(&sm.pv_done[b]));
-        mma_commit(smem_u32(&sm.kv_empty[st]));
-        return true;
-      };
-      // QK runs one tile ahead of PV: QK(i) needs only the softmax warps'
-      // read of tile i-1's logits, so they take tile i's maximum while the
-      // peer finishes tile i-1; PV(i-1) follows as soon as both P halves of
-      // tile i-1 are in, which frees tile i-1's ring stage a tile earlier
-      // than a deeper lead would
-      int next_pv = 0;
-      for (int i = 0; ok && i < ntiles; ++i) {
+      auto issue_qk = [&](int i) {
         const int st = i % kStages;
-        if (!mbar_wait(smem_u32(&sm.kv_full[st]), (i / kStages) & 1, abort_flag, err)) break;
-        // the softmax warps have read the previous tile's logits
-        if (i >= 1 && !mbar_wait(smem_u32(&sm.s_empty), (i - 1) & 1, abort_flag, err)) break;
         fence_proxy_async_smem();         // cp.async (generic) writes -> tensor-core reads
         tc_fence_after();
         const uint32_t d = tmem + kColS;
@@ -358,12 +328,56 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
           }
         }
         mma_commit(smem_u32(&sm.s_full));
-        if (i >= 1) {
-          if (!(ok = issue_pv(i - 1))) break;
-          next_pv = i;
+      };
+      auto issue_pv = [&](int i) {
+        const int st = i % kStages, b = i & 1;
+        tc_fence_after();
+        // keys of CTA h's slots: P from p[b][h], V from this CTA's own rows
+        // (h == c: their atoms 4c..4c+3) or from the peer rows' value dims
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t vbase =
+              smem_u32(sm.kv[st][h == c ? 4 * c : kOwnAtoms]);
+          const uint64_t vdesc = sdesc_sw128(vbase, kAtom, 1024);
+          const uint64_t pdesc = sdesc_sw64(smem_u32(sm.p[b][h]), 512);
+#pragma unroll
+          for (int kk = 0; kk < kOwnKeys / 16; ++kk)          // 16 keys: 32 B of P, 2 KB of V
+            mma_bf16(tmem + kColO, pdesc + 2 * kk, vdesc + (kk * 2048 >> 4), id_pv,
+                     (i > 0 || h > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&sm.pv_done[b]));
+        mma_commit(smem_u32(&sm.kv_empty[st]));
+      };
+      // QK(i) needs its gathered tile and the softmax warps' read of tile
+      // i-1's logits; PV(i) needs both P halves of tile i. Neither waits for
+      // the other: this thread polls both and issues whichever is ready, so a
+      // late P half from the peer holds back only the PV, never the next
+      // tile's logits. Both run in tile order; a stall of either longer than
+      // the wait limit gives up like any bounded wait.
+      int nq = 0, np = 0;
+      unsigned long long t_last = globaltimer();
+      while (ok && np < ntiles) {
+        bool moved = false;
+        if (nq < ntiles && mbar_test_wait(smem_u32(&sm.kv_full[nq % kStages]), (nq / kStages) & 1) &&
+            (nq == 0 || mbar_test_wait(smem_u32(&sm.s_empty), (nq - 1) & 1))) {
+          issue_qk(nq++);
+          moved = true;
+        }
+        if (np < nq && mbar_test_wait(smem_u32(&sm.p_own[np & 1]), (np >> 1) & 1) &&
+            mbar_test_wait_cluster(smem_u32(&sm.p_peer[np & 1]), (np >> 1) & 1)) {
+          issue_pv(np++);
+          moved = true;
+        }
+        if (moved) {
+          t_last = globaltimer();
+        } else if (*abort_flag) {
+          ok = false;
+        } else if (globaltimer() - t_last > kWaitLimitNs) {
+          *abort_flag = 1;
+          raise_error(err, kErrTimeout);
+          ok = false;
         }
       }
-      while (ok && next_pv < ntiles && !*abort_flag && issue_pv(next_pv)) ++next_pv;
       mma_commit(smem_u32(&sm.o_done));
       mbar_drain(smem_u32(&sm.o_done), 0);
     }
