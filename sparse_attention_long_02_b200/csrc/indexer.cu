@@ -151,8 +151,23 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_expect_tx(smem_u32(&sm.q_full), a.q_box_rows * 128);
       tma_load_2d(smem_u32(sm.q), &tm_q, smem_u32(&sm.q_full), 0, q0 * HI);
       int issued = 0;
+      // paged: the two physical blocks of a key tile, loaded a tile ahead so
+      // that the block-table read is off the copy-issue path
+      auto blocks = [&](int i, int (&pb)[2]) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int lb = 2 * (tile0 + i) + half;          // logical block
+          pb[half] = (i < ntiles && lb * 64 < key_limit)
+                         ? __ldg(a.block_table + static_cast<long long>(seq) * a.max_blocks + lb)
+                         : 0;
+        }
+      };
+      int pb_next[2] = {0, 0};
+      if (PAGED) blocks(0, pb_next);
       for (int i = 0; i < ntiles; ++i) {
         const int st = i % kStages;
+        int pb[2] = {pb_next[0], pb_next[1]};
+        if (PAGED) blocks(i + 1, pb_next);
         if (i >= kStages &&
             !mbar_wait(smem_u32(&sm.k_empty[st]), ((i / kStages) + 1) & 1, abort_flag, err))
           break;
@@ -161,16 +176,11 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int tile = tile0 + i;
         if (PAGED) {
           for (int half = 0; half < 2; ++half) {
-            const int lb = 2 * tile + half;               // logical block
-            int pb = 0;
-            if (lb * 64 < key_limit) {
-              pb = a.block_table[static_cast<long long>(seq) * a.max_blocks + lb];
-              if (pb < 0 || pb >= a.nblk) {
-                raise_error(err, kErrBounds);
-                pb = 0;
-              }
+            if (pb[half] < 0 || pb[half] >= a.nblk) {
+              raise_error(err, kErrBounds);
+              pb[half] = 0;
             }
-            tma_load_2d(smem_u32(sm.k[st]) + half * 64 * 128, &tm_k, full, 0, pb * 64);
+            tma_load_2d(smem_u32(sm.k[st]) + half * 64 * 128, &tm_k, full, 0, pb[half] * 64);
           }
         } else {
           tma_load_2d(smem_u32(sm.k[st]), &tm_k, full, 0, tile * kKeyTile);
