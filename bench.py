@@ -309,18 +309,22 @@ class RowShard:
     plan), each run as its own dsa_forward over the key prefix its rows see.
     The caches are whole on every GPU; no data crosses between GPUs."""
 
-    def __init__(self, dsa, cfg, inp, world, rank):
+    def __init__(self, dsa, cfg, inp, world, rank, path="fused"):
         self.dsa, self.inp = dsa, inp
         T, H, k = inp["T"], inp["H"], inp["k"]
         self.chunk = cfg.chunk or T
         self.starts = dsa.plan_prefill_chunks(T, inp["S"], inp["Hi"], H, k, self.chunk, world,
                                               rank)
-        self.ws = torch.empty(dsa.forward_workspace_size(self.chunk, inp["S"], inp["Hi"], H, k),
+        size = dsa.forward_fused_workspace_size if path == "fused" else dsa.forward_workspace_size
+        self.run = dsa.forward_fused if path == "fused" else dsa.forward
+        self.ws = torch.empty(size(self.chunk, inp["S"], inp["Hi"], H, k, self.chunk),
                               dtype=torch.uint8, device="cuda")
         self.out = torch.empty(T, H, 512, dtype=torch.bfloat16, device="cuda")
         self.lse = torch.empty(T, H, dtype=torch.float32, device="cuda")
         self.idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
-        self.launches = 3 * len(self.starts)       # indexer, top-k, sparse MLA per chunk
+        # per chunk: sample indexer, threshold, filter indexer, select, recompute and sparse
+        # MLA (fused), or indexer, top-k and sparse MLA (scores)
+        self.launches = (6 if path == "fused" else 3) * len(self.starts)
         self.rows = sum(min(self.chunk, T - c0) for c0 in self.starts)
 
     def step(self):
@@ -328,10 +332,11 @@ class RowShard:
         cut = lambda x, a, b: None if x is None else x[a:b]
         for c0 in self.starts:
             e = min(c0 + self.chunk, i["T"])
-            self.dsa.forward(i["q8"][c0:e], cut(i["q_scale"], c0, e), i["k8"][:e],
-                             cut(i["k_scale"], 0, e), i["w"][c0:e], i["q"][c0:e], i["kv"][:e],
-                             i["k"], i["scale"], i["sm_scale"], q_pos0=c0, idx=self.idx[c0:e],
-                             out=self.out[c0:e], lse=self.lse[c0:e], workspace=self.ws)
+            self.run(i["q8"][c0:e], cut(i["q_scale"], c0, e), i["k8"][:e],
+                     cut(i["k_scale"], 0, e), i["w"][c0:e], i["q"][c0:e], i["kv"][:e],
+                     i["k"], i["scale"], i["sm_scale"], q_pos0=c0, chunk=self.chunk,
+                     idx=self.idx[c0:e], out=self.out[c0:e], lse=self.lse[c0:e],
+                     workspace=self.ws)
 
 
 def time_steps(fn, steps, warmup, ranks, dsa, clock_gpu):
@@ -829,7 +834,7 @@ def main():
     L = inp["T"]
     shard = None
     if rows_mode:
-        shard = RowShard(dsa, cfg, inp, ranks.world, ranks.rank)
+        shard = RowShard(dsa, cfg, inp, ranks.world, ranks.rank, args.path)
         ms, clocks = time_steps(shard.step, args.steps, args.warmup, ranks, dsa, ranks.local)
         tokens = L
         del shard.ws, shard.out, shard.lse, shard.idx

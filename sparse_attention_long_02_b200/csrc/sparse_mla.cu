@@ -51,22 +51,21 @@ constexpr int kAtom = kOwnKeys * 128;           // 32 rows x 64 dims bf16, 128-B
 constexpr int kOwnAtoms = 9;                    // 8 latent + 1 rope atom of the own rows
 constexpr int kPeerAtoms = 4;                   // this CTA's 256 value dims of the peer's rows
 constexpr int kQAtom = 128 * 128;               // 128 heads x 64 dims bf16
-constexpr int kQTmemAtoms = 6;                  // Q dims [0, 384) live in TMEM
-constexpr int kQSmemAtoms = 3;                  // Q dims [384, 576) in shared memory
+constexpr int kQTmemAtoms = 7;                  // Q dims [0, 448) live in TMEM
 constexpr int kPHalf = 128 * kOwnKeys * 2;      // one CTA's P: 128 heads x 32 keys bf16
 constexpr int kGatherWarps = 6;                 // warps 0, 2, 3, 12, 13, 14
 constexpr int kSoftmaxWarps = 8;                // warps 4-11
 constexpr int kExchangeWarp = 15;
 constexpr uint32_t kColO = 0;                   // TMEM columns [0,256): output
-constexpr uint32_t kColQ = 256;                 // [256,448): Q dims [0,384), bf16 pairs
-constexpr uint32_t kColS = 448;                 // [448,512): logits of the own 32 keys, 2 buffers
+constexpr uint32_t kColQ = 256;                 // [256,480): Q dims [0,448), bf16 pairs
+constexpr uint32_t kColS = 480;                 // [480,512): logits of the own 32 keys
 constexpr float kRebase = 8.0f;                 // lazy rescale threshold (log2 units)
 
 struct MlaSmem {
   // stage = own rows (atoms 0-8), then the peer's rows' value dims (9-12)
   uint8_t kv[kStages][kOwnAtoms + kPeerAtoms][kAtom];
-  uint8_t p[2][kPHalf];                         // [slot half = owning CTA], 64-B swizzle
-  uint8_t q_s[kQSmemAtoms][kQAtom];             // Q dims [384,448), [448,512), [512,576)
+  uint8_t p[2][2][kPHalf];                      // [tile parity][slot half = owning CTA], 64-B swizzle
+  uint8_t q_s[2][kQAtom];                       // Q dims [448,512) and [512,576)
   float mx[2][128];                             // the peer's tile maxima, by tile parity
   float pair_max[2][2][128];                    // [parity][key half][head]
   float l_peer[128];                            // the peer's row sums (end)
@@ -75,27 +74,27 @@ struct MlaSmem {
   unsigned long long q_ready;                   // Q is in TMEM (staging slots free)
   unsigned long long kv_full[kStages];
   unsigned long long kv_empty[kStages];
-  unsigned long long s_full[2];                 // by logits buffer (tile parity)
-  unsigned long long s_empty[2];
+  unsigned long long s_full;
+  unsigned long long s_empty;
   unsigned long long pair;                      // both key halves posted (max, or l at the end)
   unsigned long long mx_full[2];                // the peer's tile maximum has landed
-  // one phase per tile each:
-  unsigned long long p_own;                     // this CTA's P half of the tile is written
-  unsigned long long p_peer;                    // the peer's P half has landed
-  unsigned long long p_acked;                   // the peer holds the P half sent from here
-  unsigned long long p_remote_free;             // the peer's PV no longer reads its P buffer
-  unsigned long long pv_done;                   // this CTA's PV of the tile has finished
+  unsigned long long p_own[2];                  // this CTA's P half of a tile is written
+  unsigned long long p_peer[2];                 // the peer's P half has landed
+  unsigned long long p_acked[2];                // the peer holds the P half sent from here
+  unsigned long long p_remote_free[2];          // the peer's PV no longer reads its p buffer
+  unsigned long long pv_done[2];                // this CTA's PV of a tile has finished
   unsigned long long l_full;                    // the peer's row sums have landed
   unsigned long long o_done;
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// Q's TMEM-bound atoms are staged in kv stages 1-2, which the gather first
-// fills after Q has moved into TMEM.
+// Q's TMEM-bound atoms are staged in kv stages 1-2 and the P buffers, which
+// are first written after Q has moved into TMEM.
 constexpr size_t kQStageOff = sizeof(uint8_t[kOwnAtoms + kPeerAtoms][kAtom]);
-static_assert(kQTmemAtoms * kQAtom <= 2 * kQStageOff, "Q staging fits stages 1-2");
-static_assert(kQTmemAtoms + kQSmemAtoms == kOwnAtoms, "Q split over TMEM and shared memory");
+static_assert(offsetof(MlaSmem, p) == kStages * kQStageOff, "P follows the ring");
+static_assert(kQStageOff + kQTmemAtoms * kQAtom <=
+                  offsetof(MlaSmem, q_s), "Q staging fits stages 1-2 and P");
 static_assert(kQStageOff % 1024 == 0 && kAtom % 1024 == 0 && kPHalf % 1024 == 0,
               "1024-B aligned tiles");
 static_assert(offsetof(MlaSmem, q_s) % 1024 == 0, "1024-B aligned Q atoms");
@@ -158,18 +157,17 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
       mbar_init(smem_u32(&sm.kv_full[i]), 32 * kGatherWarps + 1);
       mbar_init(smem_u32(&sm.kv_empty[i]), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&sm.s_full[b]), 1);
-      mbar_init(smem_u32(&sm.s_empty[b]), kSoftmaxWarps);
-    }
+    mbar_init(smem_u32(&sm.s_full), 1);
+    mbar_init(smem_u32(&sm.s_empty), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.pair), kSoftmaxWarps);
-    for (int b = 0; b < 2; ++b)
+    for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&sm.mx_full[b]), 128);        // one remote arrival per head
-    mbar_init(smem_u32(&sm.p_own), kSoftmaxWarps);
-    mbar_init(smem_u32(&sm.p_peer), 1);                // own expect_tx + the copied bytes
-    mbar_init(smem_u32(&sm.p_acked), 1);               // one arrival from the peer per tile
-    mbar_init(smem_u32(&sm.p_remote_free), 1);         // one arrival from the peer per tile
-    mbar_init(smem_u32(&sm.pv_done), 1);
+      mbar_init(smem_u32(&sm.p_own[b]), kSoftmaxWarps);
+      mbar_init(smem_u32(&sm.p_peer[b]), 1);           // own expect_tx + the copied bytes
+      mbar_init(smem_u32(&sm.p_acked[b]), 1);          // one arrival from the peer per use
+      mbar_init(smem_u32(&sm.p_remote_free[b]), 1);    // one arrival from the peer per use
+      mbar_init(smem_u32(&sm.pv_done[b]), 1);
+    }
     mbar_init(smem_u32(&sm.l_full), 128);
     mbar_init(smem_u32(&sm.o_done), 1);
     sm.abort_flag = aborted ? 1 : 0;
@@ -195,10 +193,10 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
     const int gw = warp == 0 ? 0 : warp <= 3 ? warp - 1 : warp - 9;   // 0..5
     if (warp == 0 && lane == 0) {
       const uint32_t qf = smem_u32(&sm.q_full);
-      mbar_expect_tx(qf, (kQTmemAtoms + kQSmemAtoms) * kQAtom);
+      mbar_expect_tx(qf, (kQTmemAtoms + 2) * kQAtom);
       for (int a = 0; a < kQTmemAtoms; ++a)
         tma_load_2d(smem_u32(q_stage + a * kQAtom), &tm_q, qf, 64 * a, r * A.H);
-      for (int a = 0; a < kQSmemAtoms; ++a)
+      for (int a = 0; a < 2; ++a)
         tma_load_2d(smem_u32(sm.q_s[a]), &tm_q, qf, 64 * (kQTmemAtoms + a), r * A.H);
     }
     // Two-deep prefetch: the slots of tile i+2 and the block-table entries
@@ -263,37 +261,41 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
     if (warp == 0 && lane == 0) mbar_drain(smem_u32(&sm.q_full), 0);
   } else if (warp == kExchangeWarp && !aborted) {
     // ---------------------------------------------------- exchange warp
-    // Tile i's P half goes from p[c] to the peer's p[c] in one bulk copy once
-    // it is written and the peer's PV of tile i-1 no longer reads that
-    // buffer. This warp also tells the peer when its half of tile i has
-    // landed here (its source may be rewritten) and when this CTA's PV of
-    // tile i has finished (it may send tile i+1). Cluster-scope releases for
-    // P come from this warp only.
+    // Tile i's P half goes from p[i&1][c] to the peer's p[i&1][c] in one bulk
+    // copy once it is written and the peer's PV of tile i-2 no longer reads
+    // that buffer. This warp also tells the peer when its half of tile i has
+    // landed here (its source may be rewritten) and when this CTA's PV of a
+    // tile has finished (it may send the tile two ahead). Cluster-scope
+    // releases for P come from this warp only.
     if (lane == 0) {
       int sent = 0;
       bool ok = true;
-      if (ntiles > 0) mbar_expect_tx(smem_u32(&sm.p_peer), kPHalf);          // tile 0
+      for (int j = 0; j < 2 && j < ntiles; ++j) mbar_expect_tx(smem_u32(&sm.p_peer[j]), kPHalf);
       for (int i = 0; ok && i < ntiles; ++i) {
-        if (!(ok = mbar_wait(smem_u32(&sm.p_own), i & 1, abort_flag, err))) break;
-        if (i >= 1 &&
-            !(ok = mbar_wait<true>(smem_u32(&sm.p_remote_free), (i - 1) & 1, abort_flag, err)))
+        const int b = i & 1;
+        if (!(ok = mbar_wait(smem_u32(&sm.p_own[b]), (i >> 1) & 1, abort_flag, err))) break;
+        if (i >= 2 &&
+            !(ok = mbar_wait<true>(smem_u32(&sm.p_remote_free[b]), ((i - 2) >> 1) & 1, abort_flag,
+                                   err)))
           break;
-        bulk_copy_to_peer(mapa(smem_u32(sm.p[c]), peer), smem_u32(sm.p[c]), kPHalf,
-                          mapa(smem_u32(&sm.p_peer), peer));
+        bulk_copy_to_peer(mapa(smem_u32(sm.p[b][c]), peer), smem_u32(sm.p[b][c]), kPHalf,
+                          mapa(smem_u32(&sm.p_peer[b]), peer));
         sent = i + 1;
-        if (!(ok = mbar_wait<true>(smem_u32(&sm.p_peer), i & 1, abort_flag, err))) break;
-        mbar_arrive_remote(mapa(smem_u32(&sm.p_acked), peer));
-        // armed before the peer may send tile i+1 (it waits for p_remote_free)
-        if (i + 1 < ntiles) mbar_expect_tx(smem_u32(&sm.p_peer), kPHalf);
-        if (!(ok = mbar_wait(smem_u32(&sm.pv_done), i & 1, abort_flag, err))) break;
-        mbar_arrive_remote(mapa(smem_u32(&sm.p_remote_free), peer));
+        if (!(ok = mbar_wait<true>(smem_u32(&sm.p_peer[b]), (i >> 1) & 1, abort_flag, err))) break;
+        mbar_arrive_remote(mapa(smem_u32(&sm.p_acked[b]), peer));
+        if (i + 2 < ntiles) mbar_expect_tx(smem_u32(&sm.p_peer[b]), kPHalf);     // tile i+2
+        if (i >= 1) {
+          const int j = i - 1;
+          if (!(ok = mbar_wait(smem_u32(&sm.pv_done[j & 1]), (j >> 1) & 1, abort_flag, err))) break;
+          mbar_arrive_remote(mapa(smem_u32(&sm.p_remote_free[j & 1]), peer));
+        }
       }
       // A copy reads this CTA's P buffer until it lands: wait for the peer's
-      // word on the last one before this CTA may leave (the softmax warps
-      // waited for every earlier one before rewriting the buffer).
-      if (sent > 0) {
-        const uint32_t bar = smem_u32(&sm.p_acked);
-        if (!mbar_wait<true>(bar, (sent - 1) & 1, abort_flag, err)) mbar_drain(bar, (sent - 1) & 1);
+      // word on the last two before this CTA may leave (the softmax warps
+      // waited for every earlier one before rewriting a buffer).
+      for (int j = sent > 2 ? sent - 2 : 0; j < sent; ++j) {
+        const uint32_t bar = smem_u32(&sm.p_acked[j & 1]);
+        if (!mbar_wait<true>(bar, (j >> 1) & 1, abort_flag, err)) mbar_drain(bar, (j >> 1) & 1);
       }
     }
   } else if (warp == 1 && !aborted) {
@@ -310,7 +312,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
         const int st = i % kStages;
         fence_proxy_async_smem();         // cp.async (generic) writes -> tensor-core reads
         tc_fence_after();
-        const uint32_t d = tmem + kColS + 32 * (i & 1);
+        const uint32_t d = tmem + kColS;
         for (int a = 0; a < kOwnAtoms; ++a) {
           const uint64_t kd = sdesc_sw128(smem_u32(sm.kv[st][a]), 0, 1024);
           if (a < kQTmemAtoms) {
@@ -325,10 +327,10 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
               mma_bf16(d, qd + 2 * kk, kd + 2 * kk, id_qk, 1u);
           }
         }
-        mma_commit(smem_u32(&sm.s_full[i & 1]));
+        mma_commit(smem_u32(&sm.s_full));
       };
       auto issue_pv = [&](int i) {
-        const int st = i % kStages;
+        const int st = i % kStages, b = i & 1;
         tc_fence_after();
         // keys of CTA h's slots: P from p[b][h], V from this CTA's own rows
         // (h == c: their atoms 4c..4c+3) or from the peer rows' value dims
@@ -337,13 +339,13 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
           const uint32_t vbase =
               smem_u32(sm.kv[st][h == c ? 4 * c : kOwnAtoms]);
           const uint64_t vdesc = sdesc_sw128(vbase, kAtom, 1024);
-          const uint64_t pdesc = sdesc_sw64(smem_u32(sm.p[h]), 512);
+          const uint64_t pdesc = sdesc_sw64(smem_u32(sm.p[b][h]), 512);
 #pragma unroll
           for (int kk = 0; kk < kOwnKeys / 16; ++kk)          // 16 keys: 32 B of P, 2 KB of V
             mma_bf16(tmem + kColO, pdesc + 2 * kk, vdesc + (kk * 2048 >> 4), id_pv,
                      (i > 0 || h > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(smem_u32(&sm.pv_done));
+        mma_commit(smem_u32(&sm.pv_done[b]));
         mma_commit(smem_u32(&sm.kv_empty[st]));
       };
       // QK(i) needs its gathered tile and the softmax warps' read of tile
@@ -357,12 +359,12 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
       while (ok && np < ntiles) {
         bool moved = false;
         if (nq < ntiles && mbar_test_wait(smem_u32(&sm.kv_full[nq % kStages]), (nq / kStages) & 1) &&
-            (nq < 2 || mbar_test_wait(smem_u32(&sm.s_empty[nq & 1]), ((nq - 2) >> 1) & 1))) {
+            (nq == 0 || mbar_test_wait(smem_u32(&sm.s_empty), (nq - 1) & 1))) {
           issue_qk(nq++);
           moved = true;
         }
-        if (np < nq && mbar_test_wait(smem_u32(&sm.p_own), np & 1) &&
-            mbar_test_wait_cluster(smem_u32(&sm.p_peer), np & 1)) {
+        if (np < nq && mbar_test_wait(smem_u32(&sm.p_own[np & 1]), (np >> 1) & 1) &&
+            mbar_test_wait_cluster(smem_u32(&sm.p_peer[np & 1]), (np >> 1) & 1)) {
           issue_pv(np++);
           moved = true;
         }
@@ -420,12 +422,12 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
     auto load_tile = [&](int j) -> bool {
       const int st = j % kStages;
       if (!warp_wait(smem_u32(&sm.kv_full[st]), (j / kStages) & 1, abort_flag, err)) return false;
-      if (!warp_wait(smem_u32(&sm.s_full[j & 1]), (j >> 1) & 1, abort_flag, err)) return false;
+      if (!warp_wait(smem_u32(&sm.s_full), j & 1, abort_flag, err)) return false;
       tc_fence_after();
-      tmem_ld16(tmem + lane_base + kColS + 32 * (j & 1) + 16 * g, s);
+      tmem_ld16(tmem + lane_base + kColS + 16 * g, s);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty[j & 1]));
+      if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty));
       // which of the own slots are selected (written by the gather warps
       // before kv_full(j))
       const unsigned valid = sm.valid[st] >> (16 * g);
@@ -461,11 +463,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
         }
         m_ref = mt;
       }
-      // p is free once this CTA's PV of tile i-1 has read it and the peer
-      // holds the half sent from it (this also lets the output be rescaled)
-      if (i >= 1 &&
-          !(ok = warp_wait(smem_u32(&sm.pv_done), (i - 1) & 1, abort_flag, err) &&
-                 warp_wait<true>(smem_u32(&sm.p_acked), (i - 1) & 1, abort_flag, err)))
+      // p[b] is free once this CTA's PV of tile i-2 has read it and the peer
+      // holds the half sent from it
+      if (i >= 2 &&
+          !(ok = warp_wait(smem_u32(&sm.pv_done[b]), ((i - 2) >> 1) & 1, abort_flag, err) &&
+                 warp_wait<true>(smem_u32(&sm.p_acked[b]), ((i - 2) >> 1) & 1, abort_flag, err)))
         break;
       {
         const bool live = m_ref > -INFINITY;
@@ -481,16 +483,19 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
         }
         // row h of this CTA's P half: 64 B, 16-B chunk q (keys 8q..8q+7) at
         // chunk q ^ ((h / 2) % 4)
-        uint4* prow = reinterpret_cast<uint4*>(sm.p[c] + h * 64);
+        uint4* prow = reinterpret_cast<uint4*>(sm.p[b][c] + h * 64);
         prow[(2 * g) ^ ((h >> 1) & 3)] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         prow[(2 * g + 1) ^ ((h >> 1) & 3)] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
       }
-      // a new reference maximum: PV of tile i-1 has finished (waited for
-      // above), so rescale this warp's half of the output. The TMEM loads and
-      // stores are warp-collective, so the whole warp takes the branch when
-      // any head re-bases (the others scale by alpha = 1).
+      // a new reference maximum: once PV of tile i-1 has finished, rescale
+      // this warp's half of the output. The TMEM loads and stores are
+      // warp-collective, so the whole warp takes the branch when any head
+      // re-bases (the others scale by alpha = 1).
       if (__any_sync(0xffffffffu, rescale)) {
+        if (i >= 1 && !(ok = warp_wait(smem_u32(&sm.pv_done[(i - 1) & 1]), ((i - 1) >> 1) & 1,
+                                       abort_flag, err)))
+          break;
         tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
@@ -505,7 +510,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
       fence_proxy_async_smem();           // P (generic writes) -> MMA and bulk-copy reads
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.p_own));
+      if (lane == 0) mbar_arrive(smem_u32(&sm.p_own[b]));
       // the next tile's maximum goes out while the peer finishes this one
       if (i + 1 < ntiles && !(ok = load_tile(i + 1))) break;
     }
@@ -514,7 +519,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
     // pair writes its 128 of this CTA's 256 output dims.
     const int last = ntiles - 1;
     if (ok && ntiles > 0 &&
-        warp_wait(smem_u32(&sm.pv_done), last & 1, abort_flag, err)) {
+        warp_wait(smem_u32(&sm.pv_done[last & 1]), (last >> 1) & 1, abort_flag, err)) {
       sm.pair_max[ntiles & 1][g][h] = l;
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.pair));
