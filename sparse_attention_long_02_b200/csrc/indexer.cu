@@ -275,7 +275,11 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               cs_key[qq * kCapS + slot] = key;
               cs_idx[qq * kCapS + slot] = static_cast<int>(s);
             }
-            const unsigned over = __ballot_sync(0xffffffffu, keep && !local);
+            // the warp's appends overflow the shared list only when its last
+            // slot does (warp-uniform test)
+            const unsigned over = base + __popc(ball) > static_cast<unsigned>(kCapS)
+                                      ? __ballot_sync(0xffffffffu, keep && !local)
+                                      : 0u;
             if (over) {
               unsigned gb = 0;
               if (lane == 0) gb = atomicAdd(a.cand_count + t, static_cast<unsigned>(__popc(over)));
