@@ -13,19 +13,23 @@
 // four e4m3 MMAs of K = 32. Each epilogue thread owns one key row of the
 // accumulator and reduces the heads of each query in registers, so the head
 // sum needs no cross-lane traffic. Two TMEM accumulator buffers and two
-// epilogue warpgroups let the MMA of key tile i+1 run under the epilogue of
-// tile i.
+// epilogue groups let the MMA of key tile i+1 run under the epilogue of tile
+// i; within a group, two warps share each key row, one per half of the
+// columns (whole queries each), so four epilogue warps per SM sub-partition
+// hide each other's TMEM-load and arithmetic latencies.
 //
-// Warp roles (384 threads): warp 0 = TMA producer, warp 1 = MMA issuer and
-// TMEM owner, warps 4-7 and 8-11 = epilogue groups 0 and 1 (a warp may only
-// touch TMEM lanes 32*(warp%4) .. +31).
+// Warp roles (576 threads = 18 warps): warp 0 = TMA producer, warp 1 = MMA
+// issuer and TMEM owner, warps 2-17 = epilogue: group (w-2)/4 % 2, column
+// half (w-2)/8. A warp may only touch TMEM lanes 32*(w%4) .. +31, and each
+// run of four consecutive warps covers the four lane quarters.
 #include "common.cuh"
 #include "dsa_internal.h"
 
 namespace dsa {
 namespace {
 
-constexpr int kIdxThreads = 384;
+constexpr int kIdxThreads = 576;
+static_assert(kIdxThreads / 32 == 2 + 16, "producer, MMA issuer and 16 epilogue warps");
 
 // Order-preserving 32-bit key of a float score (larger score, larger key).
 __device__ __forceinline__ uint32_t score_key(float f) {
@@ -57,11 +61,10 @@ struct IdxSmem {
   int abort_flag;
 };
 
-// 128 registers a thread (the epilogue fits without spills, and ran faster
-// than at the 158 the compiler picks alone): 384 x 128 leaves an SM room for
-// a 256-thread top-k CTA of the previous chunk beside this one.
+// 96 registers a thread: the register file is split over the four SM
+// sub-partitions (16384 each), and 18 warps put five on two of them.
 template <int HI, bool PAGED>
-__global__ void __maxnreg__(128)
+__global__ void __maxnreg__(96)
 indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const IndexerArgs a) {
   constexpr int QB = (256 / HI) < 64 ? (256 / HI) : 64;   // queries per CTA (prefill)
@@ -102,6 +105,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   if (nqb <= 0 || last_key < 0 || tile0 >= tile1) return;
   const int ntiles = tile1 - tile0;
   const int ncol = a.n_mma;                 // MMA N = padded QB*HI (or nq*HI)
+  // column halves per tile: two when each half holds whole queries (and
+  // whole TMEM loads), else one
+  const int nsplit = ((ncol / 2) % HI == 0 && (ncol / 2) % 32 == 0 && (HI < 32 || (ncol / 2) % 64 == 0)) ? 2 : 1;
   const uint32_t idesc = idesc_e4m3(128, ncol);
 
   const int warp = warp_id(), lane = lane_id();
@@ -113,7 +119,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.t_full[i]), 1);
-      mbar_init(smem_u32(&sm.t_empty[i]), 4);
+      mbar_init(smem_u32(&sm.t_empty[i]), 4 * nsplit);
     }
     mbar_init(smem_u32(&sm.mma_done), 1);
     sm.abort_flag = 0;
@@ -218,9 +224,11 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mma_commit(smem_u32(&sm.mma_done));
       mbar_drain(smem_u32(&sm.mma_done), 0);
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 2 && (warp - 2) / 8 < nsplit) {
     // --------------------------------------------------------- epilogue
-    const int g = (warp - 4) >> 2;                 // epilogue group = TMEM buffer
+    const int g = ((warp - 2) >> 2) & 1;           // epilogue group = TMEM buffer
+    const int hh = (warp - 2) >> 3;                // column half
+    const int cols = ncol / nsplit;                // columns of this warp: [hh*cols, +cols)
     const int row = 32 * (warp & 3) + lane;        // accumulator row = key in tile
     const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     // k_scale of this thread's key in tile i, fetched one tile ahead so the
@@ -301,10 +309,10 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // packed f32x2 FMAs over four independent accumulators
         float2 acc[4];
 #pragma unroll 1
-        for (int c = 0; c < ncol / 64; ++c) {
+        for (int c = hh * cols / 64; c < (hh + 1) * cols / 64; ++c) {
           float v[64];
           tmem_ld64(taddr + c * 64, v);
-          if (c == ncol / 64 - 1) release();
+          if (c == (hh + 1) * cols / 64 - 1) release();
           const float2* wp = reinterpret_cast<const float2*>(sm.w + c * 64);
 #pragma unroll
           for (int sub = 0; sub < 2; ++sub) {
@@ -326,10 +334,10 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
       } else {
 #pragma unroll 1
-        for (int c = 0; c < ncol / 32; ++c) {
+        for (int c = hh * cols / 32; c < (hh + 1) * cols / 32; ++c) {
           float v[32];
           tmem_ld32(taddr + c * 32, v);
-          if (c == ncol / 32 - 1) release();
+          if (c == (hh + 1) * cols / 32 - 1) release();
           const float* wp = sm.w + c * 32;
 #pragma unroll
           for (int qq = 0; qq < 32 / HI; ++qq) {
