@@ -49,6 +49,10 @@ struct IdxSmem {
   uint8_t q[256 * 128];                 // B operand: QB*HI rows x 128 B
   uint8_t k[kStages][kKTileBytes];      // A operand ring
   float w[256];                         // w[t,h]*scale*q_scale[t] for the CTA's queries
+  // the same for HI >= 32, by 32-column block b and lane group t0 = lane % 4:
+  // wt[b][t0][k] = w[32b + 4k + t0] (rows padded to 12 so that the four
+  // groups' 16-B loads fall in distinct banks)
+  float wt[8][4][12];
   uint32_t tau[64];                     // filter mode: the CTA's queries' thresholds
   uint32_t cand_n[64];                  // filter mode: entries in each query's list
   unsigned long long q_full;
@@ -140,6 +144,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       v = a.w[t * HI + h] * (a.scale * qs);
     }
     sm.w[j] = v;
+    sm.wt[j >> 5][j & 3][(j & 31) >> 2] = v;
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&sm.tmem_base), a.tmem_cols);
@@ -229,7 +234,11 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int g = ((warp - 2) >> 2) & 1;           // epilogue group = TMEM buffer
     const int hh = (warp - 2) >> 3;                // column half
     const int cols = ncol / nsplit;                // columns of this warp: [hh*cols, +cols)
-    const int row = 32 * (warp & 3) + lane;        // accumulator row = key in tile
+    // accumulator row (key in tile) whose score this thread emits: its own
+    // TMEM lane, or for HI >= 32 the lane the head-sum butterfly below leaves
+    // with it
+    const int t0 = lane & 3, t1 = lane >> 2;
+    const int row = 32 * (warp & 3) + (HI >= 32 ? t1 + 8 * (t0 & 1) + 16 * (t0 >> 1) : lane);
     const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     // k_scale of this thread's key in tile i, fetched one tile ahead so the
     // load's latency hides behind the previous tile's epilogue
@@ -305,31 +314,56 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         out[s] = (s <= pos) ? acc * ks : -INFINITY;
       };
       if constexpr (HI >= 32) {
-        // 64 columns per TMEM round trip; ReLU, then the weighted head sum in
-        // packed f32x2 FMAs over four independent accumulators
+        // 32 columns per pair of 16-lane TMEM loads: this thread holds
+        // columns 4k + t0 (k < 8) of the rows t1, t1+8, 16+t1, 24+t1 of its
+        // lane quarter, so each weight it loads serves four keys. ReLU, then
+        // the weighted sum over its 8 heads of each row (packed f32x2 FMAs);
+        // at the end of a query a butterfly over the four lanes t0 = 0..3
+        // sums the four lane groups' heads and leaves lane t0 with the total
+        // of row t1 + 8 (t0 % 2) + 16 (t0 / 2).
+        const uint32_t ta = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + g * ncol;
+        const uint32_t tb = ta + (16u << 16);
         float2 acc[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[e] = make_float2(0.f, 0.f);
 #pragma unroll 1
-        for (int c = hh * cols / 64; c < (hh + 1) * cols / 64; ++c) {
-          float v[64];
-          tmem_ld64(taddr + c * 64, v);
-          if (c == (hh + 1) * cols / 64 - 1) release();
-          const float2* wp = reinterpret_cast<const float2*>(sm.w + c * 64);
+        for (int c = hh * cols / 32; c < (hh + 1) * cols / 32; ++c) {
+          float v[32];
+          tmem_ld_16x128b_x8_pair(ta + c * 32, tb + c * 32, v);
+          if (c == (hh + 1) * cols / 32 - 1) release();
+          const float4* wq = reinterpret_cast<const float4*>(sm.wt[c][t0]);
 #pragma unroll
-          for (int sub = 0; sub < 2; ++sub) {
-            const int col0 = c * 64 + sub * 32;
-            if (col0 % HI == 0) {
+          for (int m = 0; m < 2; ++m) {
+            const float4 w4 = wq[m];                 // heads k = 4m .. 4m+3
+            const float2 wa = make_float2(w4.x, w4.y), wb = make_float2(w4.z, w4.w);
 #pragma unroll
-              for (int e = 0; e < 4; ++e) acc[e] = make_float2(0.f, 0.f);
+            for (int rr = 0; rr < 4; ++rr) {         // row rr: v[16 (rr/2) + 2k + rr%2]
+              const float* x = v + 16 * (rr >> 1) + (rr & 1);
+              const int k = 4 * m;
+              acc[rr] = __ffma2_rn(wa, make_float2(fmaxf(x[2 * k], 0.f), fmaxf(x[2 * k + 2], 0.f)),
+                                   acc[rr]);
+              acc[rr] = __ffma2_rn(wb, make_float2(fmaxf(x[2 * k + 4], 0.f), fmaxf(x[2 * k + 6], 0.f)),
+                                   acc[rr]);
             }
+          }
+          if ((c * 32 + 32) % HI == 0) {
+            float p[4];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float2 x =
-                  make_float2(fmaxf(v[32 * sub + 2 * j], 0.f), fmaxf(v[32 * sub + 2 * j + 1], 0.f));
-              acc[j & 3] = __ffma2_rn(wp[16 * sub + j], x, acc[j & 3]);
+            for (int rr = 0; rr < 4; ++rr) {
+              p[rr] = acc[rr].x + acc[rr].y;
+              acc[rr] = make_float2(0.f, 0.f);
             }
-            if ((col0 + 32) % HI == 0)
-              emit(col0 / HI, ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
-                                  ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y)));
+            // lanes t0 and t0^1 swap the rows the other keeps: even t0 keeps
+            // rows {0, 2} (t1, 16+t1), odd t0 rows {1, 3}
+            const bool odd = t0 & 1;
+            const float k0 = odd ? p[1] : p[0], k1 = odd ? p[3] : p[2];
+            const float s0 = odd ? p[0] : p[1], s1 = odd ? p[2] : p[3];
+            const float q0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 1);
+            const float q1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 1);
+            // then t0 and t0^2: t0 < 2 keeps the first, t0 >= 2 the second
+            const bool hi2 = t0 >> 1;
+            const float tot = (hi2 ? q1 : q0) + __shfl_xor_sync(0xffffffffu, hi2 ? q0 : q1, 2);
+            emit((c * 32) / HI, tot);
           }
         }
       } else {
