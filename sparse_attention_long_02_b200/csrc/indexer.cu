@@ -28,8 +28,8 @@
 namespace dsa {
 namespace {
 
-constexpr int kIdxThreads = 576;
-static_assert(kIdxThreads / 32 == 2 + 16, "producer, MMA issuer and 16 epilogue warps");
+constexpr int kIdxThreads = 320;
+static_assert(kIdxThreads / 32 == 2 + 8, "producer, MMA issuer and 8 epilogue warps");
 
 // Order-preserving 32-bit key of a float score (larger score, larger key).
 __device__ __forceinline__ uint32_t score_key(float f) {
@@ -68,7 +68,7 @@ struct IdxSmem {
 // 96 registers a thread: the register file is split over the four SM
 // sub-partitions (16384 each), and 18 warps put five on two of them.
 template <int HI, bool PAGED>
-__global__ void __maxnreg__(96)
+__global__ void __maxnreg__(168)
 indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const IndexerArgs a) {
   constexpr int QB = (256 / HI) < 64 ? (256 / HI) : 64;   // queries per CTA (prefill)
@@ -111,7 +111,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int ncol = a.n_mma;                 // MMA N = padded QB*HI (or nq*HI)
   // column halves per tile: two when each half holds whole queries (and
   // whole TMEM loads), else one
-  const int nsplit = ((ncol / 2) % HI == 0 && (ncol / 2) % 32 == 0 && (HI < 32 || (ncol / 2) % 64 == 0)) ? 2 : 1;
+  const int nsplit = 1;
   const uint32_t idesc = idesc_e4m3(128, ncol);
 
   const int warp = warp_id(), lane = lane_id();
@@ -253,6 +253,13 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       return __ldg(a.k_scale + s);
     };
     float ks_next = key_scale(g);
+    float wreg[64];
+    if constexpr (HI >= 32) {
+#pragma unroll
+      for (int b = 0; b < 8; ++b)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) wreg[8 * b + k] = b < ncol / 32 ? sm.wt[b][t0][k] : 0.f;
+    }
     const unsigned lane_lt = (1u << lane) - 1u;
     for (int i = g; i < ntiles; i += 2) {
       const float ks = ks_next;
@@ -326,16 +333,16 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         float2 acc[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[e] = make_float2(0.f, 0.f);
-#pragma unroll 1
-        for (int c = hh * cols / 32; c < (hh + 1) * cols / 32; ++c) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          if (c >= cols / 32) break;
           float v[32];
           tmem_ld_16x128b_x8_pair(ta + c * 32, tb + c * 32, v);
-          if (c == (hh + 1) * cols / 32 - 1) release();
-          const float4* wq = reinterpret_cast<const float4*>(sm.wt[c][t0]);
+          if (c == cols / 32 - 1) release();
 #pragma unroll
           for (int m = 0; m < 2; ++m) {
-            const float4 w4 = wq[m];                 // heads k = 4m .. 4m+3
-            const float2 wa = make_float2(w4.x, w4.y), wb = make_float2(w4.z, w4.w);
+            const float2 wa = make_float2(wreg[8 * c + 4 * m], wreg[8 * c + 4 * m + 1]);
+            const float2 wb = make_float2(wreg[8 * c + 4 * m + 2], wreg[8 * c + 4 * m + 3]);
 #pragma unroll
             for (int rr = 0; rr < 4; ++rr) {         // row rr: v[16 (rr/2) + 2k + rr%2]
               const float* x = v + 16 * (rr >> 1) + (rr & 1);
