@@ -10,18 +10,24 @@
 //
 // Tiling: keys sit on the MMA's M dimension (128 keys = 128 TMEM lanes),
 // queries x heads on N (QB queries x HI heads <= 256 columns), K = 128 is
-// four e4m3 MMAs of K = 32. Each epilogue thread owns one key row of the
-// accumulator and reduces the heads of each query in registers, so the head
-// sum needs no cross-lane traffic. Two TMEM accumulator buffers and two
-// epilogue groups let the MMA of key tile i+1 run under the epilogue of tile
-// i; within a group, two warps share each key row, one per half of the
-// columns (whole queries each), so four epilogue warps per SM sub-partition
-// hide each other's TMEM-load and arithmetic latencies.
+// four e4m3 MMAs of K = 32. Two TMEM accumulator buffers and two epilogue
+// groups let the MMA of key tile i+1 run under the epilogue of tile i.
 //
-// Warp roles (576 threads = 18 warps): warp 0 = TMA producer, warp 1 = MMA
-// issuer and TMEM owner, warps 2-17 = epilogue: group (w-2)/4 % 2, column
-// half (w-2)/8. A warp may only touch TMEM lanes 32*(w%4) .. +31, and each
-// run of four consecutive warps covers the four lane quarters.
+// Epilogue, HI >= 32 (the DSA configs): a thread reads its lane quarter's
+// accumulator with 16-lane TMEM loads, which give it four key rows x every
+// fourth column, so the folded weights w * scale * q_scale of its columns
+// (64 values for 256 columns) stay in registers for the whole CTA and each
+// serves four keys. ReLU and the weighted sum over its heads run in packed
+// f32x2 FMAs; a two-step butterfly over the four lanes that share the rows
+// completes each row's head sum. (Reading the weights from shared memory per
+// element instead kept the shared-memory pipe ~70% busy and cost ~27% of the
+// kernel.) HI < 32: a thread owns one key row and reduces whole queries in
+// registers.
+//
+// Warp roles (320 threads = 10 warps): warp 0 = TMA producer, warp 1 = MMA
+// issuer and TMEM owner, warps 2-9 = epilogue, group (w-2)/4 = TMEM buffer.
+// A warp may only touch TMEM lanes 32*(w%4) .. +31, and each run of four
+// consecutive warps covers the four lane quarters.
 #include "common.cuh"
 #include "dsa_internal.h"
 
@@ -40,8 +46,10 @@ constexpr int kKeyTile = 128;      // keys per MMA tile (M)
 constexpr int kStages = 4;         // key-tile ring depth
 constexpr int kKTileBytes = kKeyTile * 128;
 
-// Filter mode: each CTA first appends its candidates to per-query lists in
-// shared memory (this many bytes in all) and copies them out once at the end.
+// Filter mode: each CTA first appends its candidates to lists in shared memory
+// (this many bytes in all) and copies them out once at the end. For HI >= 32
+// each epilogue warp keeps its own list per query, with its counts in
+// registers, so an append needs no atomic; otherwise the lists are per query.
 constexpr int kCandSmemBytes = 64 * 1024;
 
 struct IdxSmem {
@@ -73,6 +81,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                const IndexerArgs a) {
   constexpr int QB = (256 / HI) < 64 ? (256 / HI) : 64;   // queries per CTA (prefill)
   constexpr int kCapS = kCandSmemBytes / (QB * 8);         // shared-memory entries per query
+  constexpr int kCapW = kCandSmemBytes / (8 * QB * 8);     // per epilogue warp and query (HI >= 32)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   IdxSmem& sm = *reinterpret_cast<IdxSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -109,9 +118,6 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   if (nqb <= 0 || last_key < 0 || tile0 >= tile1) return;
   const int ntiles = tile1 - tile0;
   const int ncol = a.n_mma;                 // MMA N = padded QB*HI (or nq*HI)
-  // column halves per tile: two when each half holds whole queries (and
-  // whole TMEM loads), else one
-  const int nsplit = 1;
   const uint32_t idesc = idesc_e4m3(128, ncol);
 
   const int warp = warp_id(), lane = lane_id();
@@ -123,7 +129,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.t_full[i]), 1);
-      mbar_init(smem_u32(&sm.t_empty[i]), 4 * nsplit);
+      mbar_init(smem_u32(&sm.t_empty[i]), 4);
     }
     mbar_init(smem_u32(&sm.mma_done), 1);
     sm.abort_flag = 0;
@@ -229,11 +235,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mma_commit(smem_u32(&sm.mma_done));
       mbar_drain(smem_u32(&sm.mma_done), 0);
     }
-  } else if (warp >= 2 && (warp - 2) / 8 < nsplit) {
+  } else if (warp >= 2) {
     // --------------------------------------------------------- epilogue
-    const int g = ((warp - 2) >> 2) & 1;           // epilogue group = TMEM buffer
-    const int hh = (warp - 2) >> 3;                // column half
-    const int cols = ncol / nsplit;                // columns of this warp: [hh*cols, +cols)
+    const int g = (warp - 2) >> 2;                 // epilogue group = TMEM buffer
     // accumulator row (key in tile) whose score this thread emits: its own
     // TMEM lane, or for HI >= 32 the lane the head-sum butterfly below leaves
     // with it
@@ -253,6 +257,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       return __ldg(a.k_scale + s);
     };
     float ks_next = key_scale(g);
+    // HI >= 32: the folded weights of this thread's columns, 32c + 4k + t0
+    // (c < 8, k < 8), in registers for the whole CTA
     float wreg[64];
     if constexpr (HI >= 32) {
 #pragma unroll
@@ -261,6 +267,10 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int k = 0; k < 8; ++k) wreg[8 * b + k] = b < ncol / 32 ? sm.wt[b][t0][k] : 0.f;
     }
     const unsigned lane_lt = (1u << lane) - 1u;
+    const int ew = warp - 2;                       // epilogue warp 0..7
+    unsigned wcnt[HI >= 32 ? QB : 1];              // this warp's appends per query (HI >= 32)
+#pragma unroll
+    for (int e = 0; e < (HI >= 32 ? QB : 1); ++e) wcnt[e] = 0;
     for (int i = g; i < ntiles; i += 2) {
       const float ks = ks_next;
       ks_next = key_scale(i + 2);
@@ -278,9 +288,10 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       };
       // Called by the whole warp with the same qq. Scores mode writes the
       // row; filter mode appends (order key, key) of every score at or above
-      // the query's threshold to the query's list in shared memory (one
-      // shared atomic per warp and query), or, once that list is full,
-      // straight to the row's list in global memory.
+      // the query's threshold to a list in shared memory (this warp's own for
+      // HI >= 32, else the query's, one shared atomic per warp and query),
+      // or, once that list is full, straight to the row's list in global
+      // memory.
       auto emit = [&](int qq, float acc) {
         if (qq >= nqb) return;
         const long long t = q0 + qq;
@@ -289,6 +300,33 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const uint32_t key = score_key(acc * ks);
           const bool keep = key_ok && s <= pos && key >= sm.tau[qq];
           const unsigned ball = __ballot_sync(0xffffffffu, keep);
+          if constexpr (HI >= 32) {
+            if (ball) {
+              const unsigned base = wcnt[qq];
+              const unsigned slot = base + __popc(ball & lane_lt);
+              const bool local = slot < static_cast<unsigned>(kCapW);
+              uint32_t* lk = cs_key + (ew * QB + qq) * kCapW;
+              int* li = cs_idx + (ew * QB + qq) * kCapW;
+              if (keep && local) {
+                lk[slot] = key;
+                li[slot] = static_cast<int>(s);
+              }
+              wcnt[qq] = base + __popc(ball);
+              const unsigned over = base + __popc(ball) > static_cast<unsigned>(kCapW)
+                                        ? __ballot_sync(0xffffffffu, keep && !local)
+                                        : 0u;
+              if (over) {
+                unsigned gb = 0;
+                if (lane == 0) gb = atomicAdd(a.cand_count + t, static_cast<unsigned>(__popc(over)));
+                gb = __shfl_sync(0xffffffffu, gb, 0) + __popc(over & lane_lt);
+                if (keep && !local && gb < static_cast<unsigned>(a.cand_cap)) {
+                  a.cand_key[t * a.cand_cap + gb] = key;
+                  a.cand_idx[t * a.cand_cap + gb] = static_cast<int>(s);
+                }
+              }
+            }
+            return;
+          }
           if (ball) {
             unsigned base = 0;
             if (lane == 0) base = atomicAdd(&sm.cand_n[qq], static_cast<unsigned>(__popc(ball)));
@@ -323,7 +361,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if constexpr (HI >= 32) {
         // 32 columns per pair of 16-lane TMEM loads: this thread holds
         // columns 4k + t0 (k < 8) of the rows t1, t1+8, 16+t1, 24+t1 of its
-        // lane quarter, so each weight it loads serves four keys. ReLU, then
+        // lane quarter, so each weight in wreg serves four keys. ReLU, then
         // the weighted sum over its 8 heads of each row (packed f32x2 FMAs);
         // at the end of a query a butterfly over the four lanes t0 = 0..3
         // sums the four lane groups' heads and leaves lane t0 with the total
@@ -335,10 +373,10 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int e = 0; e < 4; ++e) acc[e] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          if (c >= cols / 32) break;
+          if (c >= ncol / 32) break;
           float v[32];
           tmem_ld_16x128b_x8_pair(ta + c * 32, tb + c * 32, v);
-          if (c == cols / 32 - 1) release();
+          if (c == ncol / 32 - 1) release();
 #pragma unroll
           for (int m = 0; m < 2; ++m) {
             const float2 wa = make_float2(wreg[8 * c + 4 * m], wreg[8 * c + 4 * m + 1]);
@@ -375,10 +413,10 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
       } else {
 #pragma unroll 1
-        for (int c = hh * cols / 32; c < (hh + 1) * cols / 32; ++c) {
+        for (int c = 0; c < ncol / 32; ++c) {
           float v[32];
           tmem_ld32(taddr + c * 32, v);
-          if (c == (hh + 1) * cols / 32 - 1) release();
+          if (c == ncol / 32 - 1) release();
           const float* wp = sm.w + c * 32;
 #pragma unroll
           for (int qq = 0; qq < 32 / HI; ++qq) {
@@ -391,6 +429,30 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
       }
     }
+    // filter mode, HI >= 32: this warp's lists go to the rows' lists in
+    // global memory, one atomic per query
+    if constexpr (HI >= 32) {
+      if (!PAGED && a.tau) {
+        __syncwarp();
+#pragma unroll
+        for (int qq = 0; qq < QB; ++qq) {
+          const unsigned n = min(wcnt[qq], static_cast<unsigned>(kCapW));
+          if (qq >= nqb || n == 0) continue;
+          const long long t = q0 + qq;
+          unsigned gb = 0;
+          if (lane == 0) gb = atomicAdd(a.cand_count + t, n);
+          gb = __shfl_sync(0xffffffffu, gb, 0);
+          const uint32_t* lk = cs_key + (ew * QB + qq) * kCapW;
+          const int* li = cs_idx + (ew * QB + qq) * kCapW;
+          for (unsigned j = lane; j < n; j += 32) {
+            if (gb + j < static_cast<unsigned>(a.cand_cap)) {
+              a.cand_key[t * a.cand_cap + gb + j] = lk[j];
+              a.cand_idx[t * a.cand_cap + gb + j] = li[j];
+            }
+          }
+        }
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -398,10 +460,10 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc_fence_after();
     tmem_dealloc(tmem, a.tmem_cols);
   }
-  // filter mode: each query's shared-memory list goes to the row's list in
-  // global memory with one atomic (entries past the row's capacity are
-  // dropped; the count still tells the select kernel the row overflowed)
-  if (!PAGED && a.tau) {
+  // filter mode, HI < 32: each query's shared-memory list goes to the row's
+  // list in global memory with one atomic (entries past the row's capacity
+  // are dropped; the count still tells the select kernel the row overflowed)
+  if (HI < 32 && !PAGED && a.tau) {
     for (int qq = warp; qq < nqb; qq += kIdxThreads / 32) {
       const unsigned n = min(sm.cand_n[qq], static_cast<unsigned>(kCapS));
       if (n == 0) continue;
