@@ -173,6 +173,37 @@ def test_forward_fused_end_to_end_on_grid(dsa, cfg1, chunk):
                      lse_atol(inp["q"], inp["kv"], inp["sm_scale"], ref["lse"], inp["k"]))
 
 
+@pytest.mark.parametrize("L,Hi,k,chunk", [(1500, 64, 256, 512), (6000, 64, 2048, 2048),
+                                          (2000, 32, 512, 0)])
+def test_forward_fused_on_grid_wide_heads(dsa, L, Hi, k, chunk):
+    """The fused path with 32 and 64 indexer heads (the epilogue that gives
+    each thread four key rows and each warp its own candidate lists) on the
+    exact grid: every row's selection equals the chunked path's, and sampled
+    rows equal the oracle's. At k = 2048 over 6000 keys the rows keep more
+    candidates than a warp's shared-memory list holds, so appends also go
+    straight to the global lists."""
+    cfg = W.Config(92, "grid_wide", "prefill", k=k, Hi=Hi, H=8, seed=L + Hi, L=L, grid=True,
+                   scale=1.0 / 16, sm_scale=1.0 / 24)
+    inp = W.make_prefill(cfg)
+    g = cuda(inp)
+    out, lse, idx = dsa.forward_fused(g["q8"], None, g["k8"], None, g["w"], g["q"], g["kv"], k,
+                                      inp["scale"], inp["sm_scale"], chunk=chunk)
+    no_device_error(dsa)
+    _, _, idx_ref = dsa.forward(g["q8"], None, g["k8"], None, g["w"], g["q"], g["kv"], k,
+                                inp["scale"], inp["sm_scale"], chunk=chunk)
+    no_device_error(dsa)
+    got, exp = idx.cpu().numpy(), idx_ref.cpu().numpy()
+    for r in range(L):
+        assert set(got[r][got[r] >= 0]) == set(exp[r][exp[r] >= 0]), r
+    rows = np.unique(np.clip(np.array([0, 1, k - 1, k, k + 1, L // 2, chunk - 1, chunk,
+                                       L - 2, L - 1]), 0, L - 1))
+    ref = oracle.forward(inp, rows=rows)
+    for i, r in enumerate(rows):
+        assert set(got[r][got[r] >= 0]) == set(ref["idx"][i][ref["idx"][i] >= 0]), r
+    assert_mla_close(out[rows], ref["out"], lse[rows], ref["lse"],
+                     lse_atol(inp["q"][rows], inp["kv"], inp["sm_scale"], ref["lse"], k))
+
+
 def test_forward_fused_recomputes_rows_whose_threshold_misses(dsa):
     """Keys at the sampled positions (the first 256 of every 4096) hold each
     row's largest scores, all distinct from the rest, so the threshold taken
@@ -361,10 +392,11 @@ def _small_decode(lens, nq, seed, Hi=64, H=128, k=2048):
     return W.make_decode(cfg, lens=torch.tensor(lens))
 
 
-@pytest.mark.parametrize("lens,nq", [([100, 2048, 2049, 2050, 5000, 9000], 2),
-                                     ([64, 65, 4097, 3000], 1)])
-def test_decode_paged_vs_oracle(dsa, lens, nq):
-    inp = _small_decode(lens, nq, seed=len(lens) + nq)
+@pytest.mark.parametrize("lens,nq,Hi", [([100, 2048, 2049, 2050, 5000, 9000], 2, 64),
+                                        ([64, 65, 4097, 3000], 1, 64),
+                                        ([300, 2100, 4500], 2, 32)])
+def test_decode_paged_vs_oracle(dsa, lens, nq, Hi):
+    inp = _small_decode(lens, nq, seed=len(lens) + nq, Hi=Hi)
     g = cuda(inp)
     out, lse, idx = dsa.decode_paged(g["q8"], g["q_scale"], g["w"], g["q"], g["k8_pool"],
                                      g["k_scale_pool"], g["kv_pool"], g["block_table"],
