@@ -42,6 +42,15 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   const uint32_t b = __float_as_uint(f);
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
+// The float threshold equivalent to an order-key threshold: score_key(x) >= k
+// exactly when x >= key_threshold(k), for every score the epilogue forms (no
+// NaN, and no -0: its sums start at +0, and x - x rounds to +0). Keys at or
+// below that of -inf keep every score; keys above that of +inf keep none
+// (the result is a NaN, which compares false).
+__device__ __forceinline__ float key_threshold(uint32_t k) {
+  if (k <= 0x007fffffu) return -INFINITY;
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
 constexpr int kKeyTile = 128;      // keys per MMA tile (M)
 constexpr int kStages = 4;         // key-tile ring depth
 constexpr int kKTileBytes = kKeyTile * 128;
@@ -61,7 +70,7 @@ struct IdxSmem {
   // wt[b][t0][k] = w[32b + 4k + t0] (rows padded to 12 so that the four
   // groups' 16-B loads fall in distinct banks)
   float wt[8][4][12];
-  uint32_t tau[64];                     // filter mode: the CTA's queries' thresholds
+  float tau[64];                        // filter mode: the CTA's queries' thresholds
   uint32_t cand_n[64];                  // filter mode: entries in each query's list
   unsigned long long q_full;
   unsigned long long k_full[kStages];
@@ -138,7 +147,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   if (!PAGED && a.tau && threadIdx.x < QB) {
     const int qq = threadIdx.x;
     sm.cand_n[qq] = 0;
-    sm.tau[qq] = qq < nqb ? a.tau[q0 + qq] : 0xffffffffu;
+    sm.tau[qq] = key_threshold(qq < nqb ? a.tau[q0 + qq] : 0xffffffffu);
   }
   // folded per-(query, head) weights: w * scale * q_scale
   for (int j = threadIdx.x; j < ncol; j += blockDim.x) {
@@ -267,6 +276,10 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int k = 0; k < 8; ++k) wreg[8 * b + k] = b < ncol / 32 ? sm.wt[b][t0][k] : 0.f;
     }
     const unsigned lane_lt = (1u << lane) - 1u;
+    // filter mode, HI >= 32: the queries' thresholds in registers
+    float tau_r[HI >= 32 ? QB : 1];
+#pragma unroll
+    for (int e = 0; e < (HI >= 32 ? QB : 1); ++e) tau_r[e] = sm.tau[e];
     const int ew = warp - 2;                       // epilogue warp 0..7
     unsigned wcnt[HI >= 32 ? QB : 1];              // this warp's appends per query (HI >= 32)
 #pragma unroll
@@ -278,6 +291,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc_fence_after();
       const long long s = static_cast<long long>(tile0 + i) * kKeyTile + row;   // logical key
       const bool key_ok = s < key_limit;
+      // filter mode: the key is causal for query qq when qq >= sd
+      const int sd = static_cast<int>(s - pos0);
       const uint32_t taddr = tmem + lane_base + g * ncol;
       // hand the buffer back to the MMA as soon as its last columns are in
       // registers, so the next MMA into it overlaps the tail of this epilogue
@@ -297,9 +312,10 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const long long t = q0 + qq;
         const long long pos = pos0 + qq;
         if (!PAGED && a.tau) {
-          const uint32_t key = score_key(acc * ks);
-          const bool keep = key_ok && s <= pos && key >= sm.tau[qq];
+          const float sc = acc * ks;
+          const bool keep = key_ok && sd <= qq && sc >= (HI >= 32 ? tau_r[qq] : sm.tau[qq]);
           const unsigned ball = __ballot_sync(0xffffffffu, keep);
+          const uint32_t key = score_key(sc);
           if constexpr (HI >= 32) {
             if (ball) {
               const unsigned base = wcnt[qq];
