@@ -845,6 +845,10 @@ def main():
         ms, clocks = time_steps(pf.step, args.steps, args.warmup, ranks, dsa, ranks.local)
         tokens = L * ranks.world
     value = tokens / (ms / 1e3)
+    # rows of the last timed step whose threshold missed and that were
+    # recomputed on CUDA cores (the fused path keeps the count in its workspace)
+    fallback_rows = (dsa.forward_fused_fallback_rows(pf.ws, inp["T"], inp["S"], inp["k"], pf.chunk)
+                     if args.path == "fused" and not rows_mode else None)
 
     work = prefill_work(L, inp["Hi"], inp["H"], inp["k"])
     st = pf.stages()
@@ -881,6 +885,8 @@ def main():
     config["path"] = ("dsa_forward_fused: top-k fused into the indexer, no score rows in HBM"
                       if args.path == "fused" else
                       "dsa_forward: each chunk's scores in HBM, top-k beside the next indexer")
+    if fallback_rows is not None:
+        config["fallback_rows"] = fallback_rows
     if rows_mode:
         config["shard"] = (f"rows: the {math.ceil(L / pf.chunk)} chunks of one prefill over "
                            f"{ranks.world} GPU(s) by causal cost; rank 0 runs "
