@@ -507,7 +507,7 @@ cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const Index
   auto kern = indexer_kernel<HI, PAGED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
-  // the whole shared carveout, so a top-k CTA fits beside this one
+  // the whole shared carveout, so shared memory never keeps a CTA off an SM
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);

@@ -2,9 +2,9 @@
 //
 // Compiled as 512-thread CTAs (topk.cu: rows that have the GPU to
 // themselves) and as 256-thread CTAs (topk_narrow.cu: the chunks of a prefill,
-// whose selection runs on a side stream beside the next chunk's indexer; a
-// 256-thread CTA at <= 64 registers fits on an SM beside a 128-register
-// indexer CTA); fused_topk.cu uses its device functions only. The including
+// whose selection runs on a side stream while the next chunk's indexer runs,
+// taking SMs as the indexer's CTAs retire); fused_topk.cu uses its device
+// functions only. The including
 // file defines DSA_TOPK_THREADS and DSA_TOPK_MIN_CTAS, and DSA_TOPK_LAUNCH,
 // the name of the row-per-CTA kernel's launcher, where it wants that kernel.
 //
@@ -536,7 +536,7 @@ cudaError_t DSA_TOPK_LAUNCH(const TopkArgs& a, cudaStream_t st) {
   const size_t smem = sizeof(TopkSmem);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
-  // the whole shared carveout, so a CTA fits beside an indexer CTA
+  // the whole shared carveout, so shared memory never keeps a CTA off an SM
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
