@@ -394,7 +394,9 @@ def _small_decode(lens, nq, seed, Hi=64, H=128, k=2048):
 
 @pytest.mark.parametrize("lens,nq,Hi", [([100, 2048, 2049, 2050, 5000, 9000], 2, 64),
                                         ([64, 65, 4097, 3000], 1, 64),
-                                        ([300, 2100, 4500], 2, 32)])
+                                        ([300, 2100, 4500], 2, 32),
+                                        ([700, 2200, 2051], 3, 64),
+                                        ([2300, 5000], 4, 64)])
 def test_decode_paged_vs_oracle(dsa, lens, nq, Hi):
     inp = _small_decode(lens, nq, seed=len(lens) + nq, Hi=Hi)
     g = cuda(inp)
