@@ -82,10 +82,12 @@ struct IdxSmem {
   int abort_flag;
 };
 
-// 96 registers a thread: the register file is split over the four SM
-// sub-partitions (16384 each), and 18 warps put five on two of them.
+// Prefill: one CTA per SM, so the epilogue may keep its 64 weights in
+// registers (about 164 a thread). Paged: two CTAs per SM, which caps a thread
+// at 102 registers (96 used; the weights past the second block are read from
+// shared memory).
 template <int HI, bool PAGED>
-__global__ void __maxnreg__(168)
+__global__ void __launch_bounds__(kIdxThreads, PAGED ? 2 : 1)
 indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const IndexerArgs a) {
   constexpr int QB = (256 / HI) < 64 ? (256 / HI) : 64;   // queries per CTA (prefill)
@@ -268,12 +270,16 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     float ks_next = key_scale(g);
     // HI >= 32: the folded weights of this thread's columns, 32c + 4k + t0
     // (c < 8, k < 8), in registers for the whole CTA
-    float wreg[64];
+    // paged (decode) rows keep the first two blocks' weights in registers and
+    // read the rest from shared memory, so that two CTAs fit on an SM
+    constexpr int kWB = PAGED ? 2 : 8;
+    float wreg[8 * kWB];
     if constexpr (HI >= 32) {
 #pragma unroll
       for (int b = 0; b < 8; ++b)
 #pragma unroll
-        for (int k = 0; k < 8; ++k) wreg[8 * b + k] = b < ncol / 32 ? sm.wt[b][t0][k] : 0.f;
+        for (int k = 0; k < 8; ++k)
+          if (b < kWB) wreg[8 * b + k] = b < ncol / 32 ? sm.wt[b][t0][k] : 0.f;
     }
     const unsigned lane_lt = (1u << lane) - 1u;
     // filter mode, HI >= 32: the queries' thresholds in registers
@@ -395,8 +401,11 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           if (c == ncol / 32 - 1) release();
 #pragma unroll
           for (int m = 0; m < 2; ++m) {
-            const float2 wa = make_float2(wreg[8 * c + 4 * m], wreg[8 * c + 4 * m + 1]);
-            const float2 wb = make_float2(wreg[8 * c + 4 * m + 2], wreg[8 * c + 4 * m + 3]);
+            const float4 w4 =
+                c < kWB ? make_float4(wreg[(8 * c + 4 * m) % (8 * kWB)], wreg[(8 * c + 4 * m + 1) % (8 * kWB)],
+                                      wreg[(8 * c + 4 * m + 2) % (8 * kWB)], wreg[(8 * c + 4 * m + 3) % (8 * kWB)])
+                        : reinterpret_cast<const float4*>(sm.wt[c][t0])[m];
+            const float2 wa = make_float2(w4.x, w4.y), wb = make_float2(w4.z, w4.w);
 #pragma unroll
             for (int rr = 0; rr < 4; ++rr) {         // row rr: v[16 (rr/2) + 2k + rr%2]
               const float* x = v + 16 * (rr >> 1) + (rr & 1);
@@ -500,9 +509,12 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 template <int HI, bool PAGED>
 cudaError_t launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const IndexerArgs& a,
                        dim3 grid, cudaStream_t st) {
-  // Above half the SM's shared memory, so one CTA per SM: a second resident
-  // CTA would only queue on the TMEM allocation.
-  const size_t smem = std::max<size_t>(sizeof(IdxSmem) + 1024, 120 * 1024) +
+  // Prefill: above half the SM's shared memory, so one CTA per SM (a second
+  // would only queue on the TMEM allocation). Paged (decode): two CTAs per SM
+  // (96 registers, at most 256 TMEM columns each), so a batch's key slices
+  // fill the SMs in one wave instead of 1.7.
+  const size_t smem = (PAGED ? sizeof(IdxSmem) + 1024
+                             : std::max<size_t>(sizeof(IdxSmem) + 1024, 120 * 1024)) +
                       (a.tau ? kCandSmemBytes : 0);
   auto kern = indexer_kernel<HI, PAGED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
