@@ -113,6 +113,19 @@ def test_host_validation_rejects_before_launch(dsa):
     assert L.dsa_forward_fused(None, None, fake, None, fake, fake, fake, 8, 8, 4, 8, 0, 4, 0,
                                ctypes.c_float(1.0), ctypes.c_float(0.1), None, fake, None, fake,
                                1 << 40, None) == -1
+    # paged decode: more than 256 indexer columns (nq * Hi), too many MLA heads, no queries,
+    # k not a multiple of 4, workspace missing or too small; an empty batch is a no-op
+    def decode(nq=1, Hi=64, H=128, k=2048, B=2, ws=None, ws_bytes=0):
+        return L.dsa_decode_paged(fake, None, fake, fake, fake, None, fake, fake, fake, B, nq, 4,
+                                  8, Hi, H, k, ctypes.c_float(1.0), ctypes.c_float(0.1), None,
+                                  fake, None, ws, ws_bytes, None)
+    assert decode(nq=5) == -2
+    assert decode(H=129) == -2
+    assert decode(nq=0) == -1
+    assert decode(k=2046) == -1
+    assert decode() == -3
+    assert decode(ws=fake, ws_bytes=L.dsa_decode_paged_workspace_size(2, 1, 4, 64, 128, 2048) - 1) == -3
+    assert decode(B=0) == 0
     # empty problems are a no-op
     assert L.dsa_topk(fake, 0, 4, 4, 0, 4, fake, None) == 0
 
