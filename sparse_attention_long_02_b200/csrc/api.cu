@@ -351,7 +351,7 @@ int dsa_window_indices(int T, int S, int q_pos0, int window, int k, int32_t* idx
 static int mla_common(const void* q, const void* kv, const int32_t* idx, int T, int S, int H, int k,
                       float sm_scale, void* out, float* lse, const int32_t* block_table,
                       const int32_t* seq_len, int max_blocks, int nblk, int nq,
-                      cudaStream_t st, int dense = 0, int q_pos0 = 0) {
+                      cudaStream_t st, int dense = 0, int q_pos0 = 0, int compact = 0) {
   if (!q || !kv || (!idx && !dense) || !out || T < 0 || S < 0 || k <= 0 || (k & 3) ||
       !(sm_scale > 0.f) || q_pos0 < 0 || !aligned16(q) || !aligned16(kv) || !aligned16(idx) ||
       !aligned16(out))
@@ -367,6 +367,7 @@ static int mla_common(const void* q, const void* kv, const int32_t* idx, int T, 
   a.idx = idx;
   a.dense = dense;
   a.q_pos0 = q_pos0;
+  a.compact = compact;
   a.block_table = block_table;
   a.seq_len = seq_len;
   a.max_blocks = max_blocks;
@@ -414,6 +415,24 @@ int dsa_sparse_mla_decode_paged(const void* q, const void* kv_pool, const int32_
     return DSA_ERR_INVALID_ARG;
   return mla_common(q, kv_pool, idx, B * nq, max_blocks * 64, H, k, sm_scale, out, lse,
                     block_table, seq_len, max_blocks, nblk, nq, static_cast<cudaStream_t>(stream));
+}
+
+// The sparse MLA on a selection this library's top-k wrote: every row holds
+// its selected slots first, so a row that sees fewer than k keys walks only
+// those (rows of a contiguous cache at positions q_pos0 + r).
+static int mla_own_selection(const void* q, const void* kv, const int32_t* idx, int T, int S,
+                             int H, int k, int q_pos0, float sm_scale, void* out, float* lse,
+                             cudaStream_t st) {
+  if (S <= 0 && T > 0) return DSA_ERR_INVALID_ARG;
+  return mla_common(q, kv, idx, T, S, H, k, sm_scale, out, lse, nullptr, nullptr, 0, 0, 1, st, 0,
+                    q_pos0, 1);
+}
+static int mla_own_selection_paged(const void* q, const void* kv_pool, const int32_t* block_table,
+                                   const int32_t* seq_len, const int32_t* idx, int B, int nq,
+                                   int max_blocks, int nblk, int H, int k, float sm_scale,
+                                   void* out, float* lse, cudaStream_t st) {
+  return mla_common(q, kv_pool, idx, B * nq, max_blocks * 64, H, k, sm_scale, out, lse,
+                    block_table, seq_len, max_blocks, nblk, nq, st, 0, 0, 1);
 }
 
 namespace {
@@ -535,7 +554,7 @@ int dsa_forward(const void* q8, const float* q_scale, const void* k8, const floa
       s = topk_chunk(c0, scores[0], st, false);
       if (s != DSA_OK) return s;
     }
-    return dsa_sparse_mla_fwd(q, kv, idx, T, S, H, k, sm_scale, out, lse, st);
+    return mla_own_selection(q, kv, idx, T, S, H, k, q_pos0, sm_scale, out, lse, st);
   }
   // top-k of chunk c (side stream) runs beside the indexer of chunk c+1
   cudaError_t e = cudaEventRecord(ov->start, st);
@@ -558,7 +577,7 @@ int dsa_forward(const void* q8, const float* q_scale, const void* k8, const floa
   for (int b = 0; b < std::min(c, 2); ++b)
     if ((e = cudaStreamWaitEvent(st, ov->topk_done[b], 0)) != cudaSuccess) return status_of(e);
   lock.unlock();
-  return dsa_sparse_mla_fwd(q, kv, idx, T, S, H, k, sm_scale, out, lse, st);
+  return mla_own_selection(q, kv, idx, T, S, H, k, q_pos0, sm_scale, out, lse, st);
 }
 
 size_t dsa_forward_fused_workspace_size(int T, int S, int Hi, int H, int k, int chunk) {
@@ -710,7 +729,8 @@ int dsa_forward_fused(const void* q8, const float* q_scale, const void* k8, cons
       if ((e = cudaStreamWaitEvent(st, ov->topk_done[b], 0)) != cudaSuccess) return status_of(e);
     lock.unlock();
   }
-  return dsa_sparse_mla_fwd(q, kv, idx, T, S, H, k, sm_scale, out, lse, stream);
+  return mla_own_selection(q, kv, idx, T, S, H, k, q_pos0, sm_scale, out, lse,
+                           static_cast<cudaStream_t>(stream));
 }
 
 int dsa_forward_fused_fallback_rows(const void* workspace, int T, int S, int k, int chunk,
@@ -783,8 +803,8 @@ int dsa_decode_paged(const void* q8, const float* q_scale, const float* w, const
   if (s != DSA_OK) return s;
   s = run_topk(scores, rows, 0, ld, 0, seq_len, nq, k, idx, st);
   if (s != DSA_OK) return s;
-  return dsa_sparse_mla_decode_paged(q, kv_pool, block_table, seq_len, idx, B, nq, max_blocks,
-                                     nblk, H, k, sm_scale, out, lse, stream);
+  return mla_own_selection_paged(q, kv_pool, block_table, seq_len, idx, B, nq, max_blocks, nblk,
+                                 H, k, sm_scale, out, lse, st);
 }
 
 }  // extern "C"

@@ -117,6 +117,10 @@ struct MlaArgs {
   // dense causal mode: row r's slots are every key it sees, 0 .. its position
   // (q_pos0 + r, or the paged query's position); no index sets are read
   int dense = 0, q_pos0 = 0;
+  // the index sets hold their selected slots first (the library's own
+  // top-k): a row walks only min(k, keys it sees) slots, since the rest are
+  // -1. Row r of a contiguous cache sits at position q_pos0 + r.
+  int compact = 0;
   const int* block_table = nullptr;       // paged cache (decode) or null
   int max_blocks = 0, nblk = 0, nq = 1;
   const int* seq_len = nullptr;

@@ -139,8 +139,12 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaArgs A) {
   // keys a slot may name: the causal prefix of the query (paged) or the cache
   int limit = A.S;
   if (A.block_table) limit = A.seq_len[seq] - A.nq + (r % A.nq) + 1;
-  // slots of this row: the index set, or in dense mode every key it sees
-  const int nslots = !A.dense ? A.k : A.block_table ? limit : min(A.q_pos0 + r + 1, A.S);
+  // keys the row sees, and its slots: every such key in dense mode, else
+  // the index set (only its first min(k, keys) entries when the sets hold
+  // their selected slots first, the rest being -1; at least one, so that a
+  // row that sees no key still writes its zero output and -inf lse)
+  const int row_keys = A.block_table ? limit : min(A.q_pos0 + r + 1, A.S);
+  const int nslots = A.dense ? row_keys : A.compact ? max(1, min(A.k, row_keys)) : A.k;
   const int ntiles = (nslots + kTileKeys - 1) / kTileKeys;
   const int* sel = A.dense ? nullptr : A.idx + static_cast<long long>(r) * A.k;
   const int warp = warp_id(), lane = lane_id();
